@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""SplitZip lossless BF16 KV codec on B200 -- benchmark.
+
+One step = the whole hot path over one batch: exponent histogram + top-16
+codebook of every tensor, container write of every tensor, then decode of
+every container back to BF16.  The workload is the Llama-3-8B-shaped KV
+cache at 32K tokens (32 layers x {K,V} x 8 heads x 32768 tokens x 128 dim,
+4 GiB, one codebook per (layer, K/V) tensor), synthetic and seeded (kvgen).
+
+Rank 0 prints one JSON line.  `value` is round-trip throughput: uncompressed
+bytes that went through encode and decode, over all ranks, per second of the
+max-over-ranks device time.  Encode and decode are also reported alone.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl splitzip|reference]
+
+--impl reference times the CPU oracle (test infrastructure, plain C, one
+thread) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kvgen  # noqa: E402
+
+METRIC = "encode / decode GB/s (uncompressed) and % of HBM roofline; compression ratio"
+WORKLOAD = 2
+HEADER = 48
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="splitzip", choices=["splitzip", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def workload_config():
+    layers, tokens = kvgen.CONTIGUOUS[WORKLOAD]
+    n = kvgen.HEADS * tokens * kvgen.HEAD_DIM
+    return {
+        "workload": "llama3-8b-kv-32k",
+        "shape": "[%d layers][K,V][%d heads][%d tokens][%d dim] bf16" % (layers, kvgen.HEADS, tokens, kvgen.HEAD_DIM),
+        "tensors": 2 * layers,
+        "elems_per_tensor": n,
+        "bytes": 2 * 2 * layers * n,
+        "codebooks": "one per (layer, K/V) tensor",
+        "seed": "0x%X" % (kvgen.SEED_BASE + WORKLOAD),
+        "l2": "inputs (4 GiB) exceed the 126 MB L2; no flush between steps",
+    }
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [t.strip() for t in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The CPU oracle on bounded samples: each step encodes and decodes one
+    (layer, K/V) tensor of the workload, single-threaded."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cfg = workload_config()
+    n = cfg["elems_per_tensor"]
+    cache = {}
+
+    def tensor(i):
+        if i not in cache:
+            cache[i] = kvgen.contiguous_tensor(WORKLOAD, i // 2, i % 2)
+        return cache[i]
+
+    times = []
+    for s in range(args.warmup + args.steps):
+        x = tensor(s % cfg["tensors"])
+        t0 = time.perf_counter()
+        blob = oracle.encode(x)
+        y = oracle.decode(blob, n)
+        dt = time.perf_counter() - t0
+        assert y[0] == x[0]
+        if s >= args.warmup:
+            times.append(dt)
+        if len(cache) > 4:
+            cache.pop(next(iter(cache)))
+    per_step = float(np.mean(times))
+    value = 2 * n / per_step / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u16", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "each step: oracle encode + decode of one 64 MiB (layer, K/V) tensor, "
+                                   "tensors taken in order"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(host_cache, seconds):
+    """The oracle as it stands (one thread) on the first tensors of the
+    workload until about `seconds` of CPU work have run."""
+    import oracle
+    oracle.build()
+    n = host_cache.shape[1]
+    done, t_total = 0, 0.0
+    while done < host_cache.shape[0] and t_total < seconds:
+        x = host_cache[done].view(np.uint16)
+        t0 = time.perf_counter()
+        blob = oracle.encode(x)
+        oracle.decode(blob, n)
+        t_total += time.perf_counter() - t0
+        done += 1
+    return {"value": round(2 * n * done / t_total / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "oracle encode + decode of the first %d of %d (layer, K/V) tensors (%.1f s)"
+                      % (done, host_cache.shape[0], t_total)}
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import lossless_bf16_kv_splitzip_b200 as sz
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    cfg = workload_config()
+    S, n = cfg["tensors"], cfg["elems_per_tensor"]
+    U = 2 * S * n  # uncompressed bytes per step on this rank
+
+    # inputs: generated on the host straight into pinned memory, then resident in HBM
+    h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
+    kvgen.contiguous_cache(WORKLOAD, out=h_in.numpy().view(np.uint16))
+    d_in = h_in.to(dev, non_blocking=False)
+    d_out = torch.empty_like(d_in)
+    plan = sz.BatchPlan([n] * S, n, device=dev)
+    in_ptrs = torch.tensor([d_in.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=dev)
+    out_ptrs = torch.tensor([d_out.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plan.histogram(in_ptrs, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        plan.encode_only(in_ptrs, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        plan.decode(out_ptrs, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(plan.enc_status.abs().sum()) or int(plan.dec_status.abs().sum()):
+        raise RuntimeError("device status: encode %s decode %s" % (plan.enc_status.tolist(), plan.dec_status.tolist()))
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    clocks = ClockSampler(vis.split(",")[local] if vis else str(local))
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.25)  # let the sampler take its first reading
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize(dev)
+    clock_info = clocks.stop()
+    barrier()
+
+    t_hist = np.array([e[0].elapsed_time(e[1]) for e in evs]) / 1e3
+    t_enc = np.array([e[1].elapsed_time(e[2]) for e in evs]) / 1e3
+    t_dec = np.array([e[2].elapsed_time(e[3]) for e in evs]) / 1e3
+    total_s = evs[0][0].elapsed_time(evs[-1][3]) / 1e3
+    ms_step = total_s / args.steps * 1e3
+    if world > 1:
+        t = torch.tensor([ms_step, t_hist.mean(), t_enc.mean(), t_dec.mean()], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, th, te, td = t.tolist()
+    else:
+        th, te, td = float(t_hist.mean()), float(t_enc.mean()), float(t_dec.mean())
+
+    # ---- results of the last step: sizes, ratio, statuses, round trip
+    sizes = plan.sizes.cpu().numpy().astype(np.int64)
+    assert int(plan.enc_status.abs().sum()) == 0 and int(plan.dec_status.abs().sum()) == 0
+    comp = int(sizes.sum())
+    esc = int(((sizes - (HEADER + n + (n + 1) // 2)) // 5).sum())
+    round_trip_ok = bool(torch.equal(d_out, d_in))
+
+    # ---- bit-exact check of sampled containers against the oracle (rank 0)
+    parity = None
+    if rank == 0:
+        import oracle
+        sample = [0, 1, S - 2, S - 1]
+        ok = True
+        for k in sample:
+            off = int(plan.out_offset[k])
+            got = plan.container[off: off + int(sizes[k])].cpu().numpy().tobytes()
+            ok &= got == oracle.encode(h_in[k].numpy().view(np.uint16))
+        parity = {"containers_bit_exact_vs_oracle": ok, "sampled_tensors": sample,
+                  "decode_round_trip_all_tensors": round_trip_ok}
+
+    # ---- roofline (algorithmic bytes / event time, per phase)
+    peak, peak_kind = measured_peak()
+    phases = {
+        "histogram+select": (2 * S * n, th),
+        "encode_kernel": (2 * S * n + comp, te),
+        "decode": (comp + 2 * S * n, td),
+    }
+    roof = {}
+    for name, (b, t) in phases.items():
+        a = b / t / 1e9
+        roof[name] = {"achieved": round(a, 1), "frac": round(a / peak, 4), "ms": round(t * 1e3, 4),
+                      "algorithmic_bytes": b}
+    dom = max(phases, key=lambda k: phases[k][1])
+    enc_e2e_bytes = 2 * S * n + comp
+    encode_s = th + te
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": roof[dom]["achieved"], "peak": peak, "unit": "GB/s",
+                "frac": roof[dom]["frac"], "traffic": None, "peak_kind": peak_kind + " (copy, MEASURED_PEAKS.json)"
+                if peak_kind == "measured" else "fallback"}
+
+    # ---- end to end: pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        h_cont = torch.empty(comp + 256 * S, dtype=torch.uint8, pin_memory=True)
+        h_out = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
+        coffs = np.concatenate([[0], np.cumsum(sizes)])
+        times = []
+        for it in range(args.e2e_steps + 1):
+            barrier()
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            d_in.copy_(h_in, non_blocking=True)
+            plan.histogram(in_ptrs, stream)
+            plan.encode_only(in_ptrs, stream)
+            sz_host = plan.sizes.cpu().numpy()  # the caller needs the sizes to move the bytes
+            for k in range(S):
+                off = int(plan.out_offset[k])
+                h_cont[int(coffs[k]): int(coffs[k]) + int(sz_host[k])].copy_(
+                    plan.container[off: off + int(sz_host[k])], non_blocking=True)
+            for k in range(S):
+                off = int(plan.out_offset[k])
+                plan.container[off: off + int(sz_host[k])].copy_(
+                    h_cont[int(coffs[k]): int(coffs[k]) + int(sz_host[k])], non_blocking=True)
+            plan.decode(out_ptrs, stream)
+            h_out.copy_(d_out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it > 0:  # first pass warms the copy engines
+                times.append(e0.elapsed_time(e1) / 1e3)
+        assert torch.equal(h_out, h_in)
+        e2e_s = float(np.mean(times))
+        if world > 1:
+            t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = t.item()
+        e2e = {"value": round(world * U / e2e_s / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(2 * S * n + comp), "d2h_bytes_per_step": int(comp + 2 * S * n + 8 * S),
+               "ms_per_step": round(e2e_s * 1e3, 2),
+               "path": "pinned host -> H2D input -> encode -> D2H containers -> H2D containers -> decode "
+                       "-> D2H BF16, through the C ABI"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(h_in.numpy(), args.cpu_seconds)
+
+    if rank == 0:
+        value = world * U / (ms_step / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u16", "data": "synthetic", "config": cfg,
+            "encode_gbs": round(U / encode_s / 1e9, 2), "decode_gbs": round(U / td / 1e9, 2),
+            "encode_roofline_frac": round(enc_e2e_bytes / encode_s / 1e9 / peak, 4),
+            "decode_roofline_frac": roof["decode"]["frac"],
+            "ratio": round(U / comp, 5), "escape_frac": round(esc / (S * n), 6),
+            "roofline": roofline, "roofline_phases": roof,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps,
+            "clocks": clock_info, "parity": parity,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

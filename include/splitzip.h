@@ -1,0 +1,270 @@
+/*
+ * splitzip.h -- C ABI of the SplitZip lossless BF16 KV-cache codec for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "SplitZip: Ultra Fast Lossless KV Compression for Disaggregated LLM
+ * Serving" (gist.science explainer, French and Japanese pages).
+ *   - section 1 "La structure de la Note": a BF16 number is a sign, an 8-bit
+ *     exponent and a 7-bit mantissa;
+ *   - section 2 "La decouverte secrete": mantissas look random, exponents
+ *     repeat;
+ *   - section 3 "La strategie SplitZip": the 16 most common exponents get a
+ *     fixed 4-bit code, two codes share a byte, and every other exponent is
+ *     written as an escape note (position, raw exponent);
+ *   - section 4 "Pourquoi est-ce rapide ?": fixed-length codes make encode a
+ *     straight pass; decode looks each code up, recombines it with sign and
+ *     mantissa and overwrites the escaped places;
+ *   - "Les Resultats": the round trip is lossless, bit for bit.
+ *
+ * ------------------------------------------------------------------------
+ * Container format (the pages fix no bytes; this library defines them).
+ * All integers little-endian.  H = 48 header bytes.
+ *
+ *   off  0  magic "SZKV"              4 bytes  'S','Z','K','V'
+ *   off  4  version = 1               u8
+ *   off  5  dtype   = 1 (BF16)        u8
+ *   off  6  flags   = 0               u16
+ *   off  8  n_elems                   u64
+ *   off 16  n_escapes  (e)            u64
+ *   off 24  codebook[16]              u8: exponent of code k, k = 0..15
+ *   off 40  reserved = 0              8 bytes
+ *   off 48  sm[n]         sign in bit 7, mantissa in bits 6..0
+ *           codes[ceil(n/2)]  element 2j in the low nibble of byte j,
+ *                         element 2j+1 in the high nibble; an odd count
+ *                         leaves the last high nibble 0
+ *           pos[e]        u32 element indices, strictly ascending
+ *           rawexp[e]     u8 exponent of element pos[k]
+ *   size = 48 + n + ceil(n/2) + 5e
+ *
+ * Codebook: the 256 exponents ordered by (count descending, exponent
+ * ascending); code k is the k-th.  An element whose exponent is not in the
+ * codebook is an escape: its nibble is the placeholder 0 and it gets one
+ * (pos, rawexp) record.  Hence e = n - (sum of the 16 codebook counts).
+ * The top 16 of 256 bins hold at least ceil(n/16) elements, so the worst
+ * case is size <= 48 + n + ceil(n/2) + 5(n - ceil(n/16)) (SZ_MAX_BYTES).
+ * ------------------------------------------------------------------------
+ *
+ * Conventions for every entry point:
+ *   - "d_" pointers are CUDA device pointers on the current device; "h_"
+ *     pointers are host pointers.  The caller owns every buffer, including
+ *     the workspace; the library never allocates device memory and never
+ *     synchronises the stream.  Work is enqueued on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream) and runs asynchronously.
+ *   - Errors the host can see (null pointer, size, alignment, workspace or
+ *     capacity too small, launch failure) are returned at once and nothing
+ *     is enqueued.  Errors only the device can see (corrupt container,
+ *     workspace histogram that does not describe the input, a lookback wait
+ *     that ran out) are written as an sz_status to the caller's d_status
+ *     word(s), which the call first sets to SZ_OK.  A container whose status
+ *     is not SZ_OK must not be used.
+ *   - Vector path: device buffers must be 16-byte aligned (SZ_ERR_ALIGN
+ *     otherwise); there is no scalar fallback for misaligned buffers.
+ *   - Element counts are limited to n < 2^32 (escape positions are u32).
+ */
+#ifndef SPLITZIP_H
+#define SPLITZIP_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t sz_status;
+
+#define SZ_OK 0
+#define SZ_ERR_NULL (-1)           /* a required pointer is NULL */
+#define SZ_ERR_TOO_LARGE (-2)      /* n >= 2^32, or a size overflows */
+#define SZ_ERR_CAPACITY (-3)       /* output buffer smaller than needed */
+#define SZ_ERR_ALIGN (-4)          /* buffer not 16-byte aligned, page size not a multiple of 64 */
+#define SZ_ERR_CORRUPT (-5)        /* container malformed, or input != workspace histogram */
+#define SZ_ERR_CUDA (-6)           /* a CUDA runtime call failed */
+#define SZ_ERR_DEVICE_TIMEOUT (-7) /* a bounded device-side wait ran out */
+#define SZ_ERR_INVALID (-8)        /* bad argument (codebook with repeats, counts) */
+#define SZ_ERR_WORKSPACE (-9)      /* workspace smaller than planned */
+
+#define SZ_HEADER_BYTES 48u
+
+/* Worst-case container size for n elements (see the format above). */
+#define SZ_MAX_BYTES(n) \
+    (48ull + (uint64_t)(n) + ((uint64_t)(n) + 1) / 2 + 5ull * ((uint64_t)(n) - ((uint64_t)(n) + 15) / 16))
+
+/* ------------------------------------------------------------------ plan */
+/*
+ * sz_plan -- sizes for one tensor of n_elems BF16 values.
+ *   *max_compressed_bytes  worst-case container size (SZ_MAX_BYTES)
+ *   *workspace_bytes       device workspace needed by every single-tensor
+ *                          call below for this n (one workspace serves the
+ *                          histogram, encode and decode of one tensor)
+ * Host only; never touches the device.  SZ_ERR_TOO_LARGE if n >= 2^32.
+ */
+sz_status sz_plan(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes);
+
+/* ------------------------------------------------------------- histogram */
+/*
+ * sz_histogram_codebook -- exponent histogram and top-16 codebook
+ * (explainer section 3, the "Top 16" list).
+ *   d_in            n BF16 values (uint16 bit patterns), 16-byte aligned
+ *   d_codebook16    out: 16 bytes, codebook[k] = exponent of code k
+ *   d_hist256_or_null  optional out: uint32[256] exponent counts
+ *   d_ws, ws_bytes  workspace of at least sz_plan's size, 16-byte aligned.
+ *                   The histogram stays in the workspace: sz_encode of the
+ *                   same input reads it from there to size the escape
+ *                   stream, so the same workspace must be passed to it.
+ * n may be 0 (codebook = exponents 0..15).
+ */
+sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_codebook16,
+                                uint32_t *d_hist256_or_null, void *d_ws, uint64_t ws_bytes,
+                                void *stream);
+
+/* ---------------------------------------------------------------- encode */
+/*
+ * sz_encode -- write the container of d_in[0..n) (explainer section 3:
+ * sign+mantissa bytes, 4-bit codes two per byte, escape records).
+ *   d_codebook16    16 distinct exponents (normally from
+ *                   sz_histogram_codebook; any 16 distinct exponents are
+ *                   accepted, repeats give SZ_ERR_INVALID in *d_status)
+ *   d_out, out_cap  container buffer, 16-byte aligned.  out_cap must be at
+ *                   least 48 + n + ceil(n/2) (host check); the device checks
+ *                   the exact size against out_cap (SZ_ERR_CAPACITY).
+ *                   sz_plan's max_compressed_bytes always suffices for a
+ *                   codebook from sz_histogram_codebook.
+ *   d_out_bytes     out: uint64 container size (0 on a device error)
+ *   d_status_or_null  out: int32 device status (SZ_OK, SZ_ERR_CORRUPT when
+ *                   the workspace histogram does not describe d_in,
+ *                   SZ_ERR_CAPACITY, SZ_ERR_INVALID, SZ_ERR_DEVICE_TIMEOUT)
+ *   d_ws, ws_bytes  the workspace passed to sz_histogram_codebook for this
+ *                   same input (its histogram gives the escape count).
+ * The escape stream is compacted in element order across tiles by a
+ * decoupled lookback whose waits are bounded (SZ_ERR_DEVICE_TIMEOUT).
+ */
+sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
+                    uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status_or_null, void *d_ws,
+                    uint64_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------- decode */
+/*
+ * sz_decode -- rebuild d_out[0..n) from a container (explainer section 4:
+ * look the code up, recombine with sign and mantissa, overwrite escapes).
+ *   d_in, in_bytes  container bytes, 16-byte aligned; in_bytes may exceed
+ *                   the container size (the rest is ignored)
+ *   d_out           n uint16 outputs, 16-byte aligned
+ *   d_status        out (required): int32 device status; SZ_ERR_CORRUPT for
+ *                   a bad magic/version/dtype/flags/reserved field, a
+ *                   header n other than n, a size above in_bytes, repeated
+ *                   codebook entries, escape positions out of range or not
+ *                   strictly ascending, an escaped exponent that is in the
+ *                   codebook, or a nonzero placeholder / odd-tail nibble.
+ *                   d_out holds no meaningful data unless it reads SZ_OK.
+ *   d_ws, ws_bytes  workspace of sz_plan's size (per-tile escape offsets).
+ */
+sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uint64_t n,
+                    int32_t *d_status, void *d_ws, uint64_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------- batched/paged */
+/*
+ * A batch is a list of segments; each segment is one logical stream (one
+ * (layer, K/V) tensor, or one request's paged KV) with its own codebook and
+ * its own container.  A segment's stream is a run of pages of page_elems
+ * elements taken in page-list order (the last page may be partial); a
+ * contiguous tensor is one page of n elements, or several pages pointing
+ * into it.
+ */
+typedef struct sz_segment {
+    uint64_t n_elems;    /* elements in the segment's stream (< 2^32) */
+    uint64_t page_begin; /* index of the segment's first page in the page-pointer array */
+    uint64_t out_offset; /* byte offset of its container in the container buffer */
+    uint64_t tile_begin; /* first global tile index of the segment */
+} sz_segment;
+
+/*
+ * sz_plan_batched -- fill h_segs[0..n_segs) from the segment lengths.
+ *   h_seg_elems     n_segs element counts
+ *   page_elems      elements per page; a multiple of 64 when any segment
+ *                   spans more than one page (SZ_ERR_ALIGN otherwise)
+ *   h_segs          out: the segment table (pages numbered consecutively,
+ *                   containers at 256-byte aligned offsets, each slot
+ *                   SZ_MAX_BYTES(n_elems) long); copy it to the device for
+ *                   the batched calls
+ *   *total_pages    out: page pointers the page array must hold
+ *   *n_tiles        out: tiles of the whole batch (pass to the calls below)
+ *   *out_bytes      out: container buffer size
+ *   *workspace_bytes out: device workspace for the batched calls
+ * Host only.
+ */
+sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t page_elems,
+                          sz_segment *h_segs, uint64_t *total_pages, uint64_t *n_tiles,
+                          uint64_t *out_bytes, uint64_t *workspace_bytes);
+
+/*
+ * sz_histogram_codebook_batched -- exponent histogram and top-16 codebook
+ * of every segment (two kernel launches for the whole batch).  The
+ * codebooks and escape counts stay in the workspace for sz_encode_batched.
+ *   d_segs          the table from sz_plan_batched, in device memory
+ *   n_tiles         from sz_plan_batched
+ *   d_pages         device array of page pointers (16-byte aligned pages)
+ *   d_codebooks_or_null  optional out: uint8[n_segs][16]
+ *   d_status        out: int32[n_segs] device status per segment (set to
+ *                   SZ_OK first; SZ_ERR_ALIGN for a misaligned page)
+ */
+sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                                        const uint16_t *const *d_pages, uint64_t page_elems,
+                                        uint8_t *d_codebooks_or_null, int32_t *d_status, void *d_ws,
+                                        uint64_t ws_bytes, void *stream);
+
+/*
+ * sz_encode_batched -- write every segment's container (one kernel launch
+ * for the whole batch), with the codebooks that sz_histogram_codebook_batched
+ * left in the same workspace for the same pages.
+ *   d_out, out_cap  container buffer (16-byte aligned); segment k's
+ *                   container starts at d_out + d_segs[k].out_offset
+ *   d_out_bytes     out: uint64[n_segs] container sizes (0 on error)
+ *   d_status        in/out: int32[n_segs]; keeps the histogram call's
+ *                   errors and adds the encode's (first error wins)
+ */
+sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                            const uint16_t *const *d_pages, uint64_t page_elems, uint8_t *d_out,
+                            uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
+                            uint64_t ws_bytes, void *stream);
+
+/*
+ * sz_decode_batched -- decode every segment's container into its pages.
+ *   d_in, in_cap    container buffer; segment k's container starts at
+ *                   d_in + d_segs[k].out_offset and may use the rest of
+ *                   the buffer
+ *   d_pages         device array of destination page pointers (16-byte
+ *                   aligned), laid out like the encode's source pages
+ *   d_status        out: int32[n_segs] device status per segment
+ */
+sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                            const uint8_t *d_in, uint64_t in_cap, uint16_t *const *d_pages,
+                            uint64_t page_elems, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
+                            void *stream);
+
+/* ------------------------------------------------------------ diagnostics */
+/*
+ * sz_set_wait_limit_ns -- upper bound, in nanoseconds of device time, of
+ * every device-side wait (the encode's lookback on a predecessor tile).
+ * Default 1e9 (one second).  A wait that runs out sets
+ * SZ_ERR_DEVICE_TIMEOUT in the segment's status and the kernel returns.
+ * Applies to calls made after it, process-wide.
+ */
+sz_status sz_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * sz_debug_set_flags -- test hook.  Bit 0: tiles never publish their
+ * escape counts, so every lookback wait runs out (exercises the timeout
+ * path without faulting anything).  0 restores normal operation.
+ */
+sz_status sz_debug_set_flags(uint32_t flags);
+
+/* Tile size in elements used by every kernel (16384). */
+uint64_t sz_tile_elems(void);
+
+/* Library version string, e.g. "splitzip-b200 1.0 sm_100a". */
+const char *sz_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPLITZIP_H */

@@ -1,0 +1,288 @@
+"""SplitZip lossless BF16 KV-cache codec for NVIDIA B200 -- Python binding.
+
+The codec itself is the CUDA library ``libsplitzip.so`` (C ABI in
+``include/splitzip.h``).  The functions named ``sz_*`` below map one to one
+onto its entry points and only marshal arguments: device pointers are taken
+from torch tensors (or plain ints), the stream from torch's current stream.
+Every step of encode and decode runs in the library's kernels; there is no
+CPU or PyTorch fallback, and a missing or unbuildable library raises.
+
+The helpers at the end (``encode``, ``decode``, ``BatchPlan``) only allocate
+buffers with torch and call the ``sz_*`` functions.
+
+Method: "SplitZip: Ultra Fast Lossless KV Compression for Disaggregated LLM
+Serving" (gist.science explainer), sections 1-4.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+
+import numpy as np
+
+from ._build import LIB_PATH, build, is_stale
+
+__all__ = [
+    "SzError", "sz_plan", "sz_histogram_codebook", "sz_encode", "sz_decode", "sz_plan_batched",
+    "sz_histogram_codebook_batched", "sz_encode_batched", "sz_decode_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags",
+    "sz_tile_elems", "sz_version", "encode", "decode", "BatchPlan", "lib", "HEADER_BYTES",
+    "max_bytes", "STATUS",
+]
+
+HEADER_BYTES = 48
+STATUS = {
+    0: "SZ_OK", -1: "SZ_ERR_NULL", -2: "SZ_ERR_TOO_LARGE", -3: "SZ_ERR_CAPACITY",
+    -4: "SZ_ERR_ALIGN", -5: "SZ_ERR_CORRUPT", -6: "SZ_ERR_CUDA", -7: "SZ_ERR_DEVICE_TIMEOUT",
+    -8: "SZ_ERR_INVALID", -9: "SZ_ERR_WORKSPACE",
+}
+for _code, _name in STATUS.items():
+    globals()[_name] = _code
+
+
+class SzError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (%d)" % (where, STATUS.get(status, "?"), status))
+
+
+class sz_segment(ctypes.Structure):
+    _fields_ = [("n_elems", ctypes.c_uint64), ("page_begin", ctypes.c_uint64),
+                ("out_offset", ctypes.c_uint64), ("tile_begin", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libsplitzip.so (built in-tree on first use if missing)."""
+    global _lib
+    if _lib is None:
+        if is_stale():
+            build()
+        L = ctypes.CDLL(LIB_PATH)
+        u64, u32, i32, vp = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_void_p
+        pu64 = ctypes.POINTER(ctypes.c_uint64)
+        sig = {
+            "sz_plan": [u64, pu64, pu64],
+            "sz_histogram_codebook": [vp, u64, vp, vp, vp, u64, vp],
+            "sz_encode": [vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
+            "sz_decode": [vp, u64, vp, u64, vp, vp, u64, vp],
+            "sz_plan_batched": [u32, vp, u64, vp, pu64, pu64, pu64, pu64],
+            "sz_histogram_codebook_batched": [u32, vp, u64, vp, u64, vp, vp, vp, u64, vp],
+            "sz_encode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, vp, u64, vp],
+            "sz_decode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, u64, vp],
+            "sz_set_wait_limit_ns": [u64],
+            "sz_debug_set_flags": [u32],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = i32
+        L.sz_tile_elems.argtypes = []
+        L.sz_tile_elems.restype = u64
+        L.sz_version.argtypes = []
+        L.sz_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def header_symbols(header_text: str):
+    """Entry points declared in include/splitzip.h."""
+    return sorted(set(re.findall(r"^\s*(?:sz_status|uint64_t|const char \*)\s*(sz_\w+)\(", header_text,
+                                 flags=re.M)))
+
+
+# ------------------------------------------------------------ marshalling
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        return x.data_ptr()
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    raise TypeError("expected a tensor, an int address or None, got %r" % type(x))
+
+
+def _s(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise SzError(st, where)
+
+
+# --------------------------------------------------------------- entry points
+def sz_plan(n: int):
+    """-> (max_compressed_bytes, workspace_bytes)"""
+    a, b = ctypes.c_uint64(), ctypes.c_uint64()
+    _check(lib().sz_plan(n, ctypes.byref(a), ctypes.byref(b)), "sz_plan")
+    return a.value, b.value
+
+
+def sz_histogram_codebook(d_in, n, d_codebook16, d_hist256=None, d_ws=None, ws_bytes=0, stream=None):
+    _check(lib().sz_histogram_codebook(_p(d_in), n, _p(d_codebook16), _p(d_hist256), _p(d_ws), ws_bytes,
+                                       _s(stream)), "sz_histogram_codebook")
+
+
+def sz_encode(d_in, n, d_codebook16, d_out, out_cap, d_out_bytes, d_status=None, d_ws=None, ws_bytes=0,
+              stream=None):
+    _check(lib().sz_encode(_p(d_in), n, _p(d_codebook16), _p(d_out), out_cap, _p(d_out_bytes), _p(d_status),
+                           _p(d_ws), ws_bytes, _s(stream)), "sz_encode")
+
+
+def sz_decode(d_in, in_bytes, d_out, n, d_status, d_ws, ws_bytes, stream=None):
+    _check(lib().sz_decode(_p(d_in), in_bytes, _p(d_out), n, _p(d_status), _p(d_ws), ws_bytes, _s(stream)),
+           "sz_decode")
+
+
+def sz_plan_batched(seg_elems, page_elems: int):
+    """-> (segs: ctypes array of sz_segment, total_pages, n_tiles, out_bytes, workspace_bytes)"""
+    n = len(seg_elems)
+    elems = (ctypes.c_uint64 * max(n, 1))(*[int(v) for v in seg_elems])
+    segs = (sz_segment * max(n, 1))()
+    tp, nt, ob, wb = (ctypes.c_uint64() for _ in range(4))
+    _check(lib().sz_plan_batched(n, ctypes.addressof(elems), page_elems, ctypes.addressof(segs),
+                                 ctypes.byref(tp), ctypes.byref(nt), ctypes.byref(ob), ctypes.byref(wb)),
+           "sz_plan_batched")
+    return segs, tp.value, nt.value, ob.value, wb.value
+
+
+def sz_histogram_codebook_batched(n_segs, d_segs, n_tiles, d_pages, page_elems, d_codebooks, d_status, d_ws,
+                                  ws_bytes, stream=None):
+    _check(lib().sz_histogram_codebook_batched(n_segs, _p(d_segs), n_tiles, _p(d_pages), page_elems,
+                                               _p(d_codebooks), _p(d_status), _p(d_ws), ws_bytes, _s(stream)),
+           "sz_histogram_codebook_batched")
+
+
+def sz_encode_batched(n_segs, d_segs, n_tiles, d_pages, page_elems, d_out, out_cap, d_out_bytes, d_status,
+                      d_ws, ws_bytes, stream=None):
+    _check(lib().sz_encode_batched(n_segs, _p(d_segs), n_tiles, _p(d_pages), page_elems, _p(d_out), out_cap,
+                                   _p(d_out_bytes), _p(d_status), _p(d_ws), ws_bytes, _s(stream)),
+           "sz_encode_batched")
+
+
+def sz_decode_batched(n_segs, d_segs, n_tiles, d_in, in_cap, d_pages, page_elems, d_status, d_ws, ws_bytes,
+                      stream=None):
+    _check(lib().sz_decode_batched(n_segs, _p(d_segs), n_tiles, _p(d_in), in_cap, _p(d_pages), page_elems,
+                                   _p(d_status), _p(d_ws), ws_bytes, _s(stream)), "sz_decode_batched")
+
+
+def sz_set_wait_limit_ns(limit_ns: int):
+    _check(lib().sz_set_wait_limit_ns(limit_ns), "sz_set_wait_limit_ns")
+
+
+def sz_debug_set_flags(flags: int):
+    _check(lib().sz_debug_set_flags(flags), "sz_debug_set_flags")
+
+
+def sz_tile_elems() -> int:
+    return int(lib().sz_tile_elems())
+
+
+def sz_version() -> str:
+    return lib().sz_version().decode()
+
+
+def max_bytes(n: int) -> int:
+    return HEADER_BYTES + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
+
+
+# ------------------------------------------------------------ torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _u16_view(x):
+    torch = _torch()
+    if x.dtype in (torch.bfloat16, torch.float16, torch.int16):
+        return x.view(torch.int16)
+    if x.dtype == torch.uint16:
+        return x
+    raise TypeError("expected a 16-bit tensor, got %s" % x.dtype)
+
+
+def encode(x, stream=None, workspace=None):
+    """Encode a contiguous 16-bit CUDA tensor.  Returns (container uint8
+    tensor sized for the worst case, size int64 tensor [1], status int32
+    tensor [1]) -- all on the device, nothing synchronised."""
+    torch = _torch()
+    x = _u16_view(x.contiguous())
+    n = x.numel()
+    cap, wsb = sz_plan(n)
+    dev = x.device
+    ws = workspace if workspace is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
+    cb = torch.empty(16, dtype=torch.uint8, device=dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    size = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sz_histogram_codebook(x, n, cb, None, ws, wsb, stream)
+    sz_encode(x, n, cb, out, cap, size, status, ws, wsb, stream)
+    return out, size, status
+
+
+def decode(container, n, out=None, stream=None, workspace=None):
+    """Decode a container (uint8 CUDA tensor) of n elements into an int16
+    tensor (bit patterns).  Returns (out, status int32 tensor [1])."""
+    torch = _torch()
+    dev = container.device
+    _, wsb = sz_plan(n)
+    ws = workspace if workspace is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty(n, dtype=torch.int16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sz_decode(container, container.numel(), out, n, status, ws, wsb, stream)
+    return out, status
+
+
+class BatchPlan:
+    """Buffers of one batched encode/decode: the segment table (host and
+    device), container buffer, workspace, per-segment sizes and statuses."""
+
+    def __init__(self, seg_elems, page_elems, device="cuda"):
+        torch = _torch()
+        self.seg_elems = [int(v) for v in seg_elems]
+        self.page_elems = int(page_elems)
+        segs, self.total_pages, self.n_tiles, self.out_bytes, self.ws_bytes = sz_plan_batched(
+            self.seg_elems, self.page_elems)
+        self.n_segs = len(self.seg_elems)
+        self.h_segs = segs
+        raw = np.frombuffer(bytes(segs), dtype=np.uint64).reshape(-1, 4)[: self.n_segs]
+        self.out_offset = raw[:, 2].copy()
+        self.tile_begin = raw[:, 3].copy()
+        self.page_begin = raw[:, 1].copy()
+        self.d_segs = torch.from_numpy(raw.copy().view(np.int64)).to(device)
+        self.container = torch.empty(max(self.out_bytes, 16), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
+        self.sizes = torch.zeros(max(self.n_segs, 1), dtype=torch.int64, device=device)
+        self.codebooks = torch.zeros((max(self.n_segs, 1), 16), dtype=torch.uint8, device=device)
+        self.enc_status = torch.zeros(max(self.n_segs, 1), dtype=torch.int32, device=device)
+        self.dec_status = torch.zeros(max(self.n_segs, 1), dtype=torch.int32, device=device)
+
+    def histogram(self, d_page_ptrs, stream=None):
+        sz_histogram_codebook_batched(self.n_segs, self.d_segs, self.n_tiles, d_page_ptrs, self.page_elems,
+                                      self.codebooks, self.enc_status, self.ws, self.ws.numel(), stream)
+
+    def encode_only(self, d_page_ptrs, stream=None):
+        sz_encode_batched(self.n_segs, self.d_segs, self.n_tiles, d_page_ptrs, self.page_elems, self.container,
+                          self.container.numel(), self.sizes, self.enc_status, self.ws, self.ws.numel(), stream)
+
+    def encode(self, d_page_ptrs, stream=None):
+        self.histogram(d_page_ptrs, stream)
+        self.encode_only(d_page_ptrs, stream)
+
+    def decode(self, d_page_ptrs, stream=None):
+        sz_decode_batched(self.n_segs, self.d_segs, self.n_tiles, self.container, self.container.numel(),
+                          d_page_ptrs, self.page_elems, self.dec_status, self.ws, self.ws.numel(), stream)
+
+    def container_bytes(self, k: int, size: int) -> "np.ndarray":
+        off = int(self.out_offset[k])
+        return self.container[off: off + size].cpu().numpy()

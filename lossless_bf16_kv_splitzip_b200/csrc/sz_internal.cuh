@@ -1,0 +1,246 @@
+// sz_internal.cuh -- shared device-side definitions of the SplitZip B200
+// kernels: tile geometry, the tile -> (segment, page, offset) mapping, the
+// per-segment metadata record and small PTX helpers.
+//
+// Method: "SplitZip: Ultra Fast Lossless KV Compression for Disaggregated LLM
+// Serving" (gist.science explainer), sections 1-4; container layout as
+// documented in include/splitzip.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "splitzip.h"
+
+namespace sz {
+
+// ---------------------------------------------------------------- geometry
+// A tile is the unit of work of one CTA iteration: 256 threads x 4 chunks x
+// 16 elements.  A thread's chunk c covers tile elements
+// [(c*256 + tid)*16, +16), so one warp-wide 16-byte access is 512
+// contiguous bytes of input (two per chunk) or of sm output (one per chunk).
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 16;
+constexpr int kChunks = 4;
+constexpr uint32_t kTile = kThreads * kChunk * kChunks;  // 16384 elements
+constexpr uint64_t kHeader = 48;
+constexpr uint32_t kMaxSmemSegs = 1024;  // segment starts cached in shared memory
+
+// Per-segment record kept in the workspace between kernels (32 bytes).
+struct SegMeta {
+    uint8_t codebook[16];
+    uint64_t n_escapes;  // e = n - sum of the codebook's counts
+    uint32_t valid;      // 1 when the 16 entries are distinct
+    uint32_t pad;
+};
+static_assert(sizeof(SegMeta) == 32, "SegMeta layout");
+
+// Lookback tile-status word: flag in bits 63..62, count in bits 31..0.
+constexpr uint64_t kFlagAggregate = 1ull << 62;
+constexpr uint64_t kFlagPrefix = 2ull << 62;
+constexpr uint64_t kFlagMask = 3ull << 62;
+
+constexpr uint32_t kDebugNoPublish = 1u;
+
+__host__ __device__ inline uint64_t container_size(uint64_t n, uint64_t e) {
+    return kHeader + n + (n + 1) / 2 + 5 * e;
+}
+__host__ __device__ inline uint64_t div_up(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+__host__ __device__ inline uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
+__host__ __device__ inline uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__host__ __device__ inline uint32_t umin32(uint32_t a, uint32_t b) { return a < b ? a : b; }
+
+// Tiles of a segment of n elements in pages of page_elems: every page is cut
+// into tiles of kTile elements (its last tile may be short).
+__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems) {
+    return div_up(page_elems, kTile);
+}
+__host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems) {
+    if (n == 0) return 0;
+    const uint64_t full = n / page_elems, rem = n % page_elems;
+    return full * tiles_per_page(page_elems) + div_up(rem, kTile);
+}
+
+// ------------------------------------------------------------ tile lookup
+// Where the tiles come from.  Single-tensor calls use one implicit segment
+// (one page = the whole tensor); batched calls read the segment table.
+struct Batch {
+    const sz_segment *segs;  // nullptr for a single tensor
+    uint32_t n_segs;
+    uint64_t page_elems;
+    uint64_t n_tiles;
+    sz_segment single;       // the implicit segment of a single-tensor call
+};
+
+struct TileRef {
+    uint32_t seg;
+    uint64_t local;    // tile index within the segment
+    uint64_t n;        // elements of the segment
+    uint64_t page;     // page index within the segment
+    uint64_t elem0;    // first element of the tile in the segment's stream
+    uint64_t in_page;  // offset of the tile within its page (elements)
+    uint32_t len;      // elements in the tile
+};
+
+// Segment-start cache: tile_begin of every segment in shared memory when
+// the batch is small enough, else binary search in global memory.
+struct SegCache {
+    uint64_t tile_begin[kMaxSmemSegs + 1];
+};
+
+__device__ inline void seg_cache_fill(SegCache &c, const Batch &b) {
+    if (b.segs == nullptr || b.n_segs > kMaxSmemSegs) return;
+    for (uint32_t i = threadIdx.x; i < b.n_segs; i += blockDim.x) c.tile_begin[i] = b.segs[i].tile_begin;
+    if (threadIdx.x == 0) c.tile_begin[b.n_segs] = b.n_tiles;
+    __syncthreads();
+}
+
+__device__ inline uint32_t find_segment(const SegCache &c, const Batch &b, uint64_t tile) {
+    if (b.segs == nullptr) return 0;
+    uint32_t lo = 0, hi = b.n_segs;  // largest k with tile_begin[k] <= tile
+    if (b.n_segs <= kMaxSmemSegs) {
+        while (hi - lo > 1) {
+            const uint32_t mid = (lo + hi) >> 1;
+            if (c.tile_begin[mid] <= tile) lo = mid; else hi = mid;
+        }
+    } else {
+        while (hi - lo > 1) {
+            const uint32_t mid = (lo + hi) >> 1;
+            if (b.segs[mid].tile_begin <= tile) lo = mid; else hi = mid;
+        }
+    }
+    return lo;
+}
+
+__device__ inline sz_segment load_segment(const Batch &b, uint32_t k) {
+    sz_segment s;
+    if (b.segs == nullptr) {
+        s.n_elems = b.single.n_elems;
+        s.page_begin = b.single.page_begin;
+        s.out_offset = b.single.out_offset;
+        s.tile_begin = b.single.tile_begin;
+    } else {
+        const sz_segment *g = b.segs + k;
+        s.n_elems = g->n_elems;
+        s.page_begin = g->page_begin;
+        s.out_offset = g->out_offset;
+        s.tile_begin = g->tile_begin;
+    }
+    return s;
+}
+
+__device__ inline TileRef resolve_tile(const Batch &b, const sz_segment &s, uint32_t k, uint64_t tile) {
+    TileRef r;
+    r.seg = k;
+    r.local = tile - s.tile_begin;
+    r.n = s.n_elems;
+    const uint64_t tpp = tiles_per_page(b.page_elems);
+    r.page = r.local / tpp;
+    r.in_page = (r.local % tpp) * kTile;
+    r.elem0 = r.page * b.page_elems + r.in_page;
+    const uint64_t page_len = umin64(b.page_elems, r.n - r.page * b.page_elems);
+    r.len = (uint32_t)umin64(kTile, page_len - r.in_page);
+    return r;
+}
+
+// Tile (within its segment) that holds element p.
+__device__ inline uint64_t tile_of_element(uint64_t p, uint64_t page_elems) {
+    return (p / page_elems) * tiles_per_page(page_elems) + (p % page_elems) / kTile;
+}
+
+// ------------------------------------------------------------ status words
+__device__ inline void set_status(int32_t *status, int32_t code) {
+    if (status != nullptr) atomicCAS(reinterpret_cast<int *>(status), 0, code);
+}
+
+// --------------------------------------------------------------- PTX bits
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Streaming loads/stores: each byte is touched once by the kernel.
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void st_stream_v4(void *p, uint4 v) {
+    __stcs(reinterpret_cast<uint4 *>(p), v);
+}
+__device__ __forceinline__ void st_stream_u64(void *p, uint64_t v) {
+    __stcs(reinterpret_cast<unsigned long long *>(p), (unsigned long long)v);
+}
+
+// Read a little-endian u32 at any byte address.
+__device__ __forceinline__ uint32_t load_u32_any(const uint8_t *p) {
+    if ((reinterpret_cast<uintptr_t>(p) & 3) == 0) return *reinterpret_cast<const uint32_t *>(p);
+    return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
+}
+__device__ __forceinline__ uint64_t load_u64_le(const uint8_t *p) {
+    uint64_t v = 0;
+    for (int b = 7; b >= 0; --b) v = (v << 8) | p[b];
+    return v;
+}
+
+// ------------------------------------------------------- launch arguments
+struct HistArgs {
+    Batch batch;
+    const uint16_t *const *pages;  // batched: page pointers; single: &base in `base`
+    const uint16_t *base;          // single-tensor input
+    uint32_t *hist;                // [n_segs][256]
+    uint64_t tiles_per_cta;
+    int32_t *status;               // [n_segs] or nullptr
+};
+
+struct SelectArgs {
+    uint32_t n_segs;
+    const sz_segment *segs;  // nullptr: single segment of `single_n` elements
+    uint64_t single_n;
+    const uint32_t *hist;    // [n_segs][256]
+    SegMeta *meta;           // [n_segs]
+    uint8_t *codebooks_out;  // optional [n_segs][16]
+    uint32_t *hist_out;      // optional [256] (single only)
+};
+
+struct EncodeArgs {
+    Batch batch;
+    const uint16_t *const *pages;
+    const uint16_t *base;
+    uint8_t *out;
+    uint64_t out_cap;
+    uint64_t *out_bytes;    // [n_segs]
+    int32_t *status;        // [n_segs] or nullptr
+    const SegMeta *meta;    // [n_segs]
+    uint64_t *tile_status;  // [n_tiles]
+    unsigned long long *ticket;
+    uint64_t wait_limit_ns;
+    uint32_t debug_flags;
+};
+
+struct DecodeArgs {
+    Batch batch;
+    uint16_t *const *pages;  // batched destination pages
+    uint16_t *base;          // single-tensor output
+    const uint8_t *in;
+    uint64_t in_cap;         // bytes available from d_in (single: in_bytes)
+    int32_t *status;         // [n_segs]
+    uint32_t *tile_start;    // per segment: tiles+1 escape start indices
+};
+
+}  // namespace sz

@@ -1,0 +1,122 @@
+"""The C-ABI library loads, exports every entry point of include/splitzip.h,
+and its host-only logic (plans, argument checks) behaves as documented.
+No call here reaches the device: every argument error is caught before the
+first CUDA call, and sz_plan / sz_plan_batched are host arithmetic."""
+import ctypes
+import os
+
+import pytest
+
+import lossless_bf16_kv_splitzip_b200 as sz
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "splitzip.h")
+
+
+def test_library_exports_every_declared_symbol():
+    names = sz.header_symbols(open(HEADER).read())
+    assert {"sz_plan", "sz_histogram_codebook", "sz_encode", "sz_decode", "sz_plan_batched",
+            "sz_histogram_codebook_batched", "sz_encode_batched", "sz_decode_batched"} <= set(names)
+    L = ctypes.CDLL(sz.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert sz.sz_version().startswith("splitzip-b200")
+    assert sz.sz_tile_elems() == 16384
+
+
+def test_library_is_built_for_sm100a():
+    # the cubin is embedded for sm_100a; the host code reports its target
+    assert "sm_100a" in sz.sz_version()
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 16385, 1 << 25, (1 << 32) - 2])
+def test_plan_worst_case_bound(n):
+    cap, ws = sz.sz_plan(n)
+    assert cap == 48 + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
+    tiles = -(-n // 16384)
+    assert ws >= 1280 + 8 * tiles + 4 * (tiles + 1)
+    assert ws % 256 == 0
+
+
+def test_plan_rejects_too_large():
+    with pytest.raises(sz.SzError) as e:
+        sz.sz_plan(1 << 32)
+    assert e.value.status == sz.SZ_ERR_TOO_LARGE
+
+
+def test_plan_batched_layout():
+    elems = [16384 * 3, 0, 16384 * 5 + 64, 100]
+    segs, pages, tiles, out, ws = sz.sz_plan_batched(elems, 16384)
+    rows = [(s.n_elems, s.page_begin, s.out_offset, s.tile_begin) for s in segs][: len(elems)]
+    assert [r[0] for r in rows] == elems
+    assert [r[1] for r in rows] == [0, 3, 3, 9]
+    assert [r[3] for r in rows] == [0, 3, 3, 9]
+    assert pages == 10 and tiles == 10
+    off = 0
+    for r, n in zip(rows, elems):
+        assert r[2] == off and r[2] % 256 == 0
+        off += -(-sz.max_bytes(n) // 256) * 256
+    assert out == off
+    assert ws > 0
+
+
+def test_plan_batched_tiles_inside_pages():
+    # page of 40000 elements: tiles of 16384, 16384, 7232 per page
+    segs, pages, tiles, out, ws = sz.sz_plan_batched([100000], 40000)
+    assert pages == 3
+    assert tiles == 3 + 3 + 2  # 2 full pages x 3 tiles, last page of 20000: 2 tiles
+
+
+def test_plan_batched_page_alignment():
+    with pytest.raises(sz.SzError) as e:
+        sz.sz_plan_batched([1000], 100)  # several pages of 100 elements
+    assert e.value.status == sz.SZ_ERR_ALIGN
+    sz.sz_plan_batched([50], 100)  # one partial page: fine
+
+
+# ---- host-side argument errors (fake addresses are never dereferenced)
+A = 1 << 40  # a 16-byte aligned fake device address
+
+
+def _status(f, *args):
+    return f(*args)
+
+
+def test_encode_argument_errors():
+    L = sz.lib()
+    cap, ws = sz.sz_plan(1000)
+    # null output
+    assert L.sz_encode(A, 1000, A, None, cap, A, None, A, ws, None) == sz.SZ_ERR_NULL
+    # misaligned output
+    assert L.sz_encode(A, 1000, A, A + 4, cap, A, None, A, ws, None) == sz.SZ_ERR_ALIGN
+    # misaligned input
+    assert L.sz_encode(A + 2, 1000, A, A, cap, A, None, A, ws, None) == sz.SZ_ERR_ALIGN
+    # capacity below 48 + n + ceil(n/2)
+    assert L.sz_encode(A, 1000, A, A, 48 + 1000 + 499, A, None, A, ws, None) == sz.SZ_ERR_CAPACITY
+    # workspace too small
+    assert L.sz_encode(A, 1000, A, A, cap, A, None, A, ws - 1, None) == sz.SZ_ERR_WORKSPACE
+    # too large
+    assert L.sz_encode(A, 1 << 32, A, A, cap, A, None, A, ws, None) == sz.SZ_ERR_TOO_LARGE
+
+
+def test_histogram_and_decode_argument_errors():
+    L = sz.lib()
+    cap, ws = sz.sz_plan(1000)
+    assert L.sz_histogram_codebook(None, 1000, A, None, A, ws, None) == sz.SZ_ERR_NULL
+    assert L.sz_histogram_codebook(A, 1000, A, None, A + 8, ws, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_histogram_codebook(A, 1000, A, None, A, 16, None) == sz.SZ_ERR_WORKSPACE
+    assert L.sz_decode(A, cap, A, 1000, None, A, ws, None) == sz.SZ_ERR_NULL  # status required
+    assert L.sz_decode(A + 1, cap, A, 1000, A, A, ws, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_decode(A, cap, A, 1000, A, A, 0, None) == sz.SZ_ERR_WORKSPACE
+
+
+def test_batched_argument_errors():
+    L = sz.lib()
+    assert L.sz_encode_batched(0, None, 0, None, 16384, None, 0, None, None, None, 0, None) == sz.SZ_OK
+    assert L.sz_encode_batched(2, A, 4, A, 16384, A, 1 << 20, A, None, A, 1 << 20, None) == sz.SZ_ERR_NULL
+    assert L.sz_encode_batched(2, A, 4, A, 0, A, 1 << 20, A, A, A, 1 << 20, None) == sz.SZ_ERR_INVALID
+    assert L.sz_encode_batched(2, A, 4, A, 16384, A + 8, 1 << 20, A, A, A, 1 << 20, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_histogram_codebook_batched(2, A, 4, A, 16384, None, None, A, 1 << 20, None) == sz.SZ_ERR_NULL
+    assert L.sz_histogram_codebook_batched(2, A, 4, A, 16384, None, A, A, 16, None) == sz.SZ_ERR_WORKSPACE
+    assert L.sz_decode_batched(2, A, 4, A + 4, 1 << 20, A, 16384, A, A, 1 << 20, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_decode_batched(2, A, 4, A, 1 << 20, A, 16384, A, A, 16, None) == sz.SZ_ERR_WORKSPACE
