@@ -49,21 +49,24 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--tensors", type=int, default=0,
+                   help="time only the first T (layer, K/V) tensors (a smaller case for profiling)")
     return p.parse_args()
 
 
-def workload_config():
+def workload_config(tensors=0):
     layers, tokens = kvgen.CONTIGUOUS[WORKLOAD]
     n = kvgen.HEADS * tokens * kvgen.HEAD_DIM
+    t = 2 * layers if tensors <= 0 else min(tensors, 2 * layers)
     return {
-        "workload": "llama3-8b-kv-32k",
+        "workload": "llama3-8b-kv-32k" if t == 2 * layers else "llama3-8b-kv-32k, first %d tensors" % t,
         "shape": "[%d layers][K,V][%d heads][%d tokens][%d dim] bf16" % (layers, kvgen.HEADS, tokens, kvgen.HEAD_DIM),
-        "tensors": 2 * layers,
+        "tensors": t,
         "elems_per_tensor": n,
-        "bytes": 2 * 2 * layers * n,
+        "bytes": 2 * t * n,
         "codebooks": "one per (layer, K/V) tensor",
         "seed": "0x%X" % (kvgen.SEED_BASE + WORKLOAD),
-        "l2": "inputs (4 GiB) exceed the 126 MB L2; no flush between steps",
+        "l2": "inputs (%d MiB) exceed the 126 MB L2; no flush between steps" % (2 * t * n >> 20),
     }
 
 
@@ -215,13 +218,16 @@ def main():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    cfg = workload_config()
+    cfg = workload_config(args.tensors)
     S, n = cfg["tensors"], cfg["elems_per_tensor"]
     U = 2 * S * n  # uncompressed bytes per step on this rank
 
     # inputs: generated on the host straight into pinned memory, then resident in HBM
     h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
-    kvgen.contiguous_cache(WORKLOAD, out=h_in.numpy().view(np.uint16))
+    kvgen.contiguous_cache(WORKLOAD, layers=S // 2 if S % 2 == 0 else None,
+                           out=h_in.numpy().view(np.uint16)) if S % 2 == 0 else \
+        [h_in[k].numpy().view(np.uint16).__setitem__(slice(None), kvgen.contiguous_tensor(WORKLOAD, k // 2, k % 2))
+         for k in range(S)]
     d_in = h_in.to(dev, non_blocking=False)
     d_out = torch.empty_like(d_in)
     plan = sz.BatchPlan([n] * S, n, device=dev)

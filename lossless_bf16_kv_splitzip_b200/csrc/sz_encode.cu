@@ -65,7 +65,16 @@ __device__ __forceinline__ uint32_t byte_of(uint4 v, int b) {  // b is a compile
     return (w >> (8 * (b & 3))) & 0xFFu;
 }
 
-__device__ __forceinline__ int chunk_elem_of_bit(int i) { return 4 * (i & 7) + (i >> 3); }
+// Escape mask in element order (bit j = element j), from the interleaved
+// layout above: for each quad q, bits 8b + q (b = 0..3) are gathered by one
+// multiply -- the four products of 1 + 2^7 + 2^14 + 2^21 do not overlap, and
+// bits 21..24 receive b = 0..3 in order.
+__device__ __forceinline__ uint32_t esc_in_element_order(uint32_t m) {
+    uint32_t r = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r |= ((((m >> q) & 0x01010101u) * 0x00204081u) >> 21 & 0xFu) << (4 * q);
+    return r;
+}
 
 __device__ __forceinline__ uint32_t esc_bit_of_elem(int j) { return 1u << (8 * (j & 3) + (j >> 2)); }
 
@@ -325,13 +334,12 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
         uint32_t chunk_base = 0;
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
-            uint32_t m = esc[c];
+            uint32_t m = esc[c] ? esc_in_element_order(esc[c]) : 0u;
             uint64_t idx = (uint64_t)tile_excl + chunk_base + field16(thr_excl, c);
             chunk_base += field16(tile_tot, c);
-            while (m) {
-                const int bit = __ffs(m) - 1;
+            while (m) {  // ascending element order
+                const int j = __ffs(m) - 1;
                 m &= m - 1;
-                const int j = chunk_elem_of_bit(bit);
                 const uint64_t p = r.elem0 + (uint64_t)(c * kThreads + tid) * kChunk + j;
                 if (idx >= e_total) {  // more escapes than the histogram said
                     set_status(status, SZ_ERR_CORRUPT);
