@@ -224,10 +224,12 @@ def main():
 
     # inputs: generated on the host straight into pinned memory, then resident in HBM
     h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
-    kvgen.contiguous_cache(WORKLOAD, layers=S // 2 if S % 2 == 0 else None,
-                           out=h_in.numpy().view(np.uint16)) if S % 2 == 0 else \
-        [h_in[k].numpy().view(np.uint16).__setitem__(slice(None), kvgen.contiguous_tensor(WORKLOAD, k // 2, k % 2))
-         for k in range(S)]
+    host = h_in.numpy().view(np.uint16)
+    if S % 2 == 0:
+        kvgen.contiguous_cache(WORKLOAD, layers=S // 2, out=host)
+    else:
+        for k in range(S):
+            host[k] = kvgen.contiguous_tensor(WORKLOAD, k // 2, k % 2)
     d_in = h_in.to(dev, non_blocking=False)
     d_out = torch.empty_like(d_in)
     plan = sz.BatchPlan([n] * S, n, device=dev)
