@@ -132,8 +132,7 @@ def sz_histogram_codebook(d_in, n, d_codebook16, d_hist256=None, d_ws=None, ws_b
                                        _s(stream)), "sz_histogram_codebook")
 
 
-def sz_encode(d_in, n, d_codebook16, d_out, out_cap, d_out_bytes, d_status=None, d_ws=None, ws_bytes=0,
-              stream=None):
+def sz_encode(d_in, n, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, ws_bytes, stream=None):
     _check(lib().sz_encode(_p(d_in), n, _p(d_codebook16), _p(d_out), out_cap, _p(d_out_bytes), _p(d_status),
                            _p(d_ws), ws_bytes, _s(stream)), "sz_encode")
 

@@ -9,8 +9,6 @@
 namespace sz {
 cudaError_t launch_hist(const HistArgs &a, bool batched, int grid, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
-cudaError_t launch_prepare(const uint8_t *codebook, const uint32_t *hist, uint64_t n, SegMeta *meta,
-                           cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, int grid, cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
@@ -55,39 +53,23 @@ bool device_info(DeviceInfo &out) {
 uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// ---- single-tensor workspace layout
-//   [0, 1024)        exponent histogram, u32[256]
-//   [1024, 1056)     SegMeta
-//   [1056, 1064)     tile ticket
-//   [1280, +8T)      lookback tile status, u64[T]
-//   [D, +4(T+1))     decode tile escape starts, D = round_up(1280 + 8T, 256)
-struct SingleWs {
-    uint64_t tiles, hist, meta, ticket, status, starts, total;
+// ---- workspace layout for S segments and T tiles (256-byte aligned parts)
+//   seg_hist   u32[S][256]     exponent counts per segment
+//   meta       SegMeta[S]      codebook and escape count per segment
+//   tile_hist  u32[T][256]     exponent counts per tile
+//   tile_off   u32[T]          first escape index of each tile
+//   sub_start  u32[4T + S]     first escape index of each sub-tile (decode)
+struct Ws {
+    uint64_t seg_hist, meta, tile_hist, tile_off, sub_start, total;
 };
-SingleWs single_ws(uint64_t n) {
-    SingleWs w;
-    w.tiles = segment_tiles(n, n > 0 ? n : 1);
-    w.hist = 0;
-    w.meta = 1024;
-    w.ticket = 1056;
-    w.status = 1280;
-    w.starts = round_up(w.status + 8 * w.tiles, kAlign);
-    w.total = round_up(w.starts + 4 * (w.tiles + 1), kAlign);
-    return w;
-}
-
-// ---- batched workspace layout (S segments, T tiles), 256-byte aligned parts
-struct BatchWs {
-    uint64_t hist, meta, ticket, status, starts, total;
-};
-BatchWs batch_ws(uint64_t n_segs, uint64_t n_tiles) {
-    BatchWs w;
-    w.hist = 0;
-    w.meta = round_up(w.hist + 1024 * n_segs, kAlign);
-    w.ticket = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
-    w.status = w.ticket + kAlign;
-    w.starts = round_up(w.status + 8 * n_tiles, kAlign);
-    w.total = round_up(w.starts + 4 * (n_tiles + n_segs), kAlign);
+Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
+    Ws w;
+    w.seg_hist = 0;
+    w.meta = round_up(w.seg_hist + 1024 * n_segs, kAlign);
+    w.tile_hist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
+    w.tile_off = round_up(w.tile_hist + 1024 * n_tiles, kAlign);
+    w.sub_start = round_up(w.tile_off + 4 * n_tiles, kAlign);
+    w.total = round_up(w.sub_start + 4 * (4 * n_tiles + n_segs), kAlign);
     return w;
 }
 
@@ -96,6 +78,7 @@ Batch single_batch(uint64_t n) {
     b.segs = nullptr;
     b.n_segs = 1;
     b.page_elems = n > 0 ? n : 1;
+    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems);
     b.n_tiles = segment_tiles(n, b.page_elems);
     b.single.n_elems = n;
     b.single.page_begin = 0;
@@ -104,12 +87,29 @@ Batch single_batch(uint64_t n) {
     return b;
 }
 
+Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, uint64_t page_elems) {
+    Batch b{};
+    b.segs = d_segs;
+    b.n_segs = n_segs;
+    b.page_elems = page_elems;
+    b.tiles_per_page = (uint32_t)tiles_per_page(page_elems);
+    b.n_tiles = n_tiles;
+    return b;
+}
+
+Ws single_ws(uint64_t n) { return ws_layout(1, single_batch(n).n_tiles); }
+
+template <class T>
+T *at(void *ws, uint64_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
 sz_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SZ_OK : SZ_ERR_CUDA; }
 
-#define SZ_TRY_CUDA(call)                              \
-    do {                                               \
-        cudaError_t _e = (call);                       \
-        if (_e != cudaSuccess) return SZ_ERR_CUDA;     \
+#define SZ_TRY_CUDA(call)                          \
+    do {                                           \
+        cudaError_t _e = (call);                   \
+        if (_e != cudaSuccess) return SZ_ERR_CUDA; \
     } while (0)
 
 }  // namespace
@@ -129,58 +129,64 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
     if (!d_codebook16 || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
     if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const SingleWs w = single_ws(n);
+    const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
-    SZ_TRY_CUDA(cudaMemsetAsync(ws + w.hist, 0, 1024, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024, s));
     HistArgs h{};
     h.batch = single_batch(n);
     h.base = d_in;
-    h.hist = reinterpret_cast<uint32_t *>(ws + w.hist);
+    h.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
+    h.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
     h.status = nullptr;
     SZ_TRY_CUDA(launch_hist(h, false, dev.sms * dev.hist_occ, s));
     SelectArgs sa{};
-    sa.n_segs = 1;
-    sa.segs = nullptr;
-    sa.single_n = n;
-    sa.hist = h.hist;
-    sa.meta = reinterpret_cast<SegMeta *>(ws + w.meta);
+    sa.batch = h.batch;
+    sa.seg_hist = h.seg_hist;
+    sa.tile_hist = h.tile_hist;
+    sa.meta = at<SegMeta>(d_ws, w.meta);
+    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
+    sa.codebook_in = nullptr;
     sa.codebooks_out = d_codebook16;
     sa.hist_out = d_hist256_or_null;
     return cuda_status(launch_select(sa, s));
 }
 
 sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
-                    uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status_or_null, void *d_ws,
-                    uint64_t ws_bytes, void *stream) {
-    if (!d_codebook16 || !d_out || !d_out_bytes || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
+                    uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
+                    void *stream) {
+    if (!d_codebook16 || !d_out || !d_out_bytes || !d_status || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
     if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
-    const SingleWs w = single_ws(n);
+    const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
-    SZ_TRY_CUDA(cudaMemsetAsync(ws + w.ticket, 0, (w.status - w.ticket) + 8 * w.tiles, s));
     SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
-    if (d_status_or_null) SZ_TRY_CUDA(cudaMemsetAsync(d_status_or_null, 0, sizeof(int32_t), s));
-    SegMeta *meta = reinterpret_cast<SegMeta *>(ws + w.meta);
-    SZ_TRY_CUDA(launch_prepare(d_codebook16, reinterpret_cast<const uint32_t *>(ws + w.hist), n, meta, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
+    // escape count and per-tile escape offsets for this codebook, from the
+    // histograms sz_histogram_codebook left in the workspace
+    SelectArgs sa{};
+    sa.batch = single_batch(n);
+    sa.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
+    sa.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
+    sa.meta = at<SegMeta>(d_ws, w.meta);
+    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
+    sa.codebook_in = d_codebook16;
+    SZ_TRY_CUDA(launch_select(sa, s));
     EncodeArgs a{};
-    a.batch = single_batch(n);
+    a.batch = sa.batch;
     a.base = d_in;
     a.out = d_out;
     a.out_cap = out_cap;
     a.out_bytes = d_out_bytes;
-    a.status = d_status_or_null;
-    a.meta = meta;
-    a.tile_status = reinterpret_cast<uint64_t *>(ws + w.status);
-    a.ticket = reinterpret_cast<unsigned long long *>(ws + w.ticket);
+    a.status = d_status;
+    a.meta = sa.meta;
+    a.tile_off = sa.tile_off;
     a.wait_limit_ns = g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
     return cuda_status(launch_encode(a, false, dev.sms * dev.enc_occ, s));
@@ -191,12 +197,11 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     if (!d_in || !d_status || !d_ws || (n > 0 && !d_out)) return SZ_ERR_NULL;
     if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
     if (!aligned16(d_in) || (n > 0 && !aligned16(d_out)) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const SingleWs w = single_ws(n);
+    const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
     DecodeArgs a{};
     a.batch = single_batch(n);
@@ -204,7 +209,9 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     a.in = d_in;
     a.in_cap = in_bytes;
     a.status = d_status;
-    a.tile_start = reinterpret_cast<uint32_t *>(ws + w.starts);
+    a.sub_start = at<uint32_t>(d_ws, w.sub_start);
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
     SZ_TRY_CUDA(launch_esc_index(a, false, s));
     return cuda_status(launch_decode(a, false, dev.sms * dev.dec_occ, s));
 }
@@ -234,17 +241,8 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
     *total_pages = pages;
     *n_tiles = tiles;
     *out_bytes = out;
-    *workspace_bytes = batch_ws(n_segs, tiles).total;
+    *workspace_bytes = ws_layout(n_segs, tiles).total;
     return SZ_OK;
-}
-
-static Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, uint64_t page_elems) {
-    Batch b{};
-    b.segs = d_segs;
-    b.n_segs = n_segs;
-    b.page_elems = page_elems;
-    b.n_tiles = n_tiles;
-    return b;
 }
 
 sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
@@ -255,25 +253,26 @@ sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_seg
     if (!d_segs || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const BatchWs w = batch_ws(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
-    SZ_TRY_CUDA(cudaMemsetAsync(ws + w.hist, 0, 1024 * (uint64_t)n_segs, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 * (uint64_t)n_segs, s));
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
     HistArgs h{};
     h.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
     h.pages = d_pages;
-    h.hist = reinterpret_cast<uint32_t *>(ws + w.hist);
+    h.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
+    h.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
     h.status = d_status;
     SZ_TRY_CUDA(launch_hist(h, true, dev.sms * dev.hist_occ, s));
     SelectArgs sa{};
-    sa.n_segs = n_segs;
-    sa.segs = d_segs;
-    sa.hist = h.hist;
-    sa.meta = reinterpret_cast<SegMeta *>(ws + w.meta);
+    sa.batch = h.batch;
+    sa.seg_hist = h.seg_hist;
+    sa.tile_hist = h.tile_hist;
+    sa.meta = at<SegMeta>(d_ws, w.meta);
+    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
     sa.codebooks_out = d_codebooks_or_null;
     return cuda_status(launch_select(sa, s));
 }
@@ -286,13 +285,11 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     if (!d_segs || !d_out || !d_out_bytes || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const BatchWs w = batch_ws(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
-    SZ_TRY_CUDA(cudaMemsetAsync(ws + w.ticket, 0, (w.status - w.ticket) + 8 * n_tiles, s));
     SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, 8 * (uint64_t)n_segs, s));
     EncodeArgs a{};
     a.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
@@ -301,9 +298,8 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.out_cap = out_cap;
     a.out_bytes = d_out_bytes;
     a.status = d_status;
-    a.meta = reinterpret_cast<const SegMeta *>(ws + w.meta);
-    a.tile_status = reinterpret_cast<uint64_t *>(ws + w.status);
-    a.ticket = reinterpret_cast<unsigned long long *>(ws + w.ticket);
+    a.meta = at<SegMeta>(d_ws, w.meta);
+    a.tile_off = at<uint32_t>(d_ws, w.tile_off);
     a.wait_limit_ns = g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
     return cuda_status(launch_encode(a, true, dev.sms * dev.enc_occ, s));
@@ -316,12 +312,11 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     if (!d_segs || !d_in || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_in) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const BatchWs w = batch_ws(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = static_cast<uint8_t *>(d_ws);
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
     DecodeArgs a{};
     a.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
@@ -329,7 +324,9 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.in = d_in;
     a.in_cap = in_cap;
     a.status = d_status;
-    a.tile_start = reinterpret_cast<uint32_t *>(ws + w.starts);
+    a.sub_start = at<uint32_t>(d_ws, w.sub_start);
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
     SZ_TRY_CUDA(launch_esc_index(a, true, s));
     return cuda_status(launch_decode(a, true, dev.sms * dev.dec_occ, s));
 }
@@ -346,6 +343,6 @@ sz_status sz_debug_set_flags(uint32_t flags) {
 
 uint64_t sz_tile_elems(void) { return kTile; }
 
-const char *sz_version(void) { return "splitzip-b200 1.0 sm_100a"; }
+const char *sz_version(void) { return "splitzip-b200 1.1 sm_100a"; }
 
 }  // extern "C"

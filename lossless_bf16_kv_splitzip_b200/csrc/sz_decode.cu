@@ -5,13 +5,22 @@
 // sign and mantissa, and, where an escape note exists, overwrites that
 // place with the raw exponent -- linear work with no detours.
 //
-// Two launches: (1) every tile finds where its escapes start in the
-// ascending position stream (one binary search per tile, all tiles in
-// parallel); (2) every tile decodes its elements in registers, patches its
-// escapes there, and writes the BF16 values with 16-byte stores.  The
-// escape list of each tile is checked as it is used: ascending, inside the
-// tile, raw exponent outside the codebook, placeholder code 0 -- together
-// with monotone tile starts this proves the whole stream well formed.
+// Two launches.  (1) esc_index_kernel: for every 16,384-element sub-tile,
+// the index of its first escape in the ascending position stream (one
+// binary search per sub-tile, all in parallel); it also checks each
+// segment's header.  (2) decode_kernel, warp-specialised like the encode:
+//   producer warp   TMA bulk copies of the sub-tile's sm bytes (16 KiB) and
+//                   codes (8 KiB) into a 3-stage ring; its 32 lanes also
+//                   load the sub-tile's escape records, check them (inside
+//                   the sub-tile, strictly ascending, raw exponent outside
+//                   the codebook) and store them in the stage together with
+//                   a chunk -> first-escape map;
+//   8 consumer warps turn codes + sm bytes into BF16 with register-only
+//                   PRMT lookups, patch their chunk's escapes in registers
+//                   (checking the placeholder code is 0), and write 16-byte
+//                   stores.
+// Monotone sub-tile starts plus in-sub-tile checks prove the whole escape
+// stream well formed.  Every mbarrier wait is bounded.
 #include "sz_internal.cuh"
 
 namespace sz {
@@ -21,10 +30,11 @@ struct Header {
     uint64_t n, e;
     uint64_t cb_lo, cb_hi;  // codebook bytes 0-7 and 8-15, little-endian
     bool ok;
+    bool misaligned;        // container not on a 16-byte boundary: not read at all
 };
 
-__device__ __forceinline__ uint32_t cb_entry(const Header &h, int k) {  // k compile-time after unrolling
-    return (uint32_t)(((k < 8) ? h.cb_lo : h.cb_hi) >> (8 * (k & 7))) & 0xFFu;
+__device__ __forceinline__ uint32_t cb_entry(uint64_t lo, uint64_t hi, int k) {  // k compile-time after unrolling
+    return (uint32_t)(((k < 8) ? lo : hi) >> (8 * (k & 7))) & 0xFFu;
 }
 
 // Parse and check the fixed fields of the container at c (cap bytes
@@ -32,63 +42,61 @@ __device__ __forceinline__ uint32_t cb_entry(const Header &h, int k) {  // k com
 __device__ inline Header read_header(const uint8_t *c, uint64_t cap, uint64_t n) {
     Header h{};
     h.ok = false;
-    if (cap < kHeader) return h;
+    h.misaligned = (reinterpret_cast<uintptr_t>(c) & 15) != 0;
+    if (h.misaligned || cap < kHeader) return h;
     const uint64_t w0 = *reinterpret_cast<const uint64_t *>(c);
     h.n = *reinterpret_cast<const uint64_t *>(c + 8);
     h.e = *reinterpret_cast<const uint64_t *>(c + 16);
     h.cb_lo = *reinterpret_cast<const uint64_t *>(c + 24);
     h.cb_hi = *reinterpret_cast<const uint64_t *>(c + 32);
     const uint64_t rsv = *reinterpret_cast<const uint64_t *>(c + 40);
-    h.ok = w0 == 0x00000101564B5A53ull && rsv == 0 && h.n == n && n < (1ull << 32) && h.e <= n &&
-           container_size(n, h.e) <= cap;
-    return h;
-}
-
-__device__ inline bool codebook_distinct(const Header &h) {
-    bool ok = true;
+    bool distinct = true;
 #pragma unroll
     for (int i = 0; i < 16; ++i)
 #pragma unroll
-        for (int k = i + 1; k < 16; ++k) ok &= cb_entry(h, i) != cb_entry(h, k);
-    return ok;
+        for (int k = i + 1; k < 16; ++k) distinct &= cb_entry(h.cb_lo, h.cb_hi, i) != cb_entry(h.cb_lo, h.cb_hi, k);
+    h.ok = w0 == 0x00000101564B5A53ull && rsv == 0 && h.n == n && n < (1ull << 32) && h.e <= n &&
+           container_size(n, h.e) <= cap && distinct;
+    return h;
 }
 
-// ----------------------------------------------------- per-tile escape index
-// Entry j of segment k (j = 0..tiles_k) = index of the first escape whose
-// position is >= the first element of tile j (entry tiles_k = e).  Entries
-// of segment k start at tile_begin_k + k.  One thread per entry.
+// ------------------------------------------------- per-sub-tile escape index
+// Entry j of segment k (j = 4*tile + sub, j = 0..4*tiles_k) = index of the
+// first escape whose position is >= the first element of that sub-tile
+// (sub-tiles past a short tile's end start at the tile's end); entry
+// 4*tiles_k = e.  Entries of segment k start at 4*tile_begin_k + k.
 template <bool kBatched>
 __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint64_t n_entries) {
     __shared__ uint64_t s_entry_begin[kMaxSmemSegs + 1];
     const uint32_t ns = kBatched ? a.batch.n_segs : 1u;
     const bool cached = kBatched && ns <= kMaxSmemSegs;
     if (cached) {
-        for (uint32_t i = threadIdx.x; i < ns; i += blockDim.x) s_entry_begin[i] = a.batch.segs[i].tile_begin + i;
-        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < ns; i += blockDim.x)
+            s_entry_begin[i] = 4 * a.batch.segs[i].tile_begin + i;
     }
+    __syncthreads();
     const uint64_t j_glob = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j_glob >= n_entries) return;
     uint32_t k = 0;
-    if (kBatched) {  // largest k with tile_begin_k + k <= j_glob
+    if (kBatched) {  // largest k with 4*tile_begin_k + k <= j_glob
         uint32_t lo = 0, hi = ns;
         while (hi - lo > 1) {
             const uint32_t mid = (lo + hi) >> 1;
-            const uint64_t b = cached ? s_entry_begin[mid] : a.batch.segs[mid].tile_begin + mid;
+            const uint64_t b = cached ? s_entry_begin[mid] : 4 * a.batch.segs[mid].tile_begin + mid;
             if (b <= j_glob) lo = mid; else hi = mid;
         }
         k = lo;
     }
     const sz_segment seg = load_segment(a.batch, k);
-    const uint64_t j = j_glob - (seg.tile_begin + k);
+    const uint64_t j = j_glob - (4 * seg.tile_begin + k);
     const uint64_t tiles = segment_tiles(seg.n_elems, a.batch.page_elems);
-    int32_t *status = a.status + k;
-    uint32_t *ts = a.tile_start + seg.tile_begin + k;
-    if (j > tiles) return;
+    uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k;
+    if (j > 4 * tiles) return;
     const uint64_t cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
     const uint8_t *c = a.in + seg.out_offset;
     const Header h = read_header(c, cap, seg.n_elems);
-    if (j == tiles) {  // the sentinel thread reports the header of its segment
-        if (!h.ok || !codebook_distinct(h)) set_status(status, SZ_ERR_CORRUPT);
+    if (j == 4 * tiles) {  // the sentinel thread reports the header of its segment
+        if (!h.ok) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
         ts[j] = h.ok ? (uint32_t)h.e : 0u;
         return;
     }
@@ -96,9 +104,9 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
         ts[j] = 0;
         return;
     }
+    const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / 4);
+    const uint64_t first = r.elem0 + umin32((uint32_t)(j % 4) * kSub, r.len);
     const uint64_t n = h.n, e = h.e;
-    const uint64_t tpp = tiles_per_page(a.batch.page_elems);
-    const uint64_t first = (j / tpp) * a.batch.page_elems + (j % tpp) * kTile;
     const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
     uint64_t lo = 0, hi = e;  // first index with pos >= first
     while (lo < hi) {
@@ -119,14 +127,15 @@ struct DecTables {
     uint32_t hA, hB, hC, hD, lA, lB;
 };
 
-__device__ inline DecTables make_tables(const Header &hd) {
+__device__ inline DecTables make_tables(uint64_t cb_lo, uint64_t cb_hi) {
     DecTables t;
     uint32_t h[4] = {0, 0, 0, 0}, l[2] = {0, 0};
 #pragma unroll
-    for (int k = 0; k < 16; ++k) h[k >> 2] |= (cb_entry(hd, k) >> 1) << (8 * (k & 3));
+    for (int k = 0; k < 16; ++k) h[k >> 2] |= (cb_entry(cb_lo, cb_hi, k) >> 1) << (8 * (k & 3));
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-        l[j >> 2] |= (((cb_entry(hd, j) & 1u) << 6) | ((cb_entry(hd, j + 8) & 1u) << 7)) << (8 * (j & 3));
+        l[j >> 2] |= (((cb_entry(cb_lo, cb_hi, j) & 1u) << 6) | ((cb_entry(cb_lo, cb_hi, j + 8) & 1u) << 7))
+                     << (8 * (j & 3));
     t.hA = h[0]; t.hB = h[1]; t.hC = h[2]; t.hD = h[3];
     t.lA = l[0]; t.lB = l[1];
     return t;
@@ -170,171 +179,336 @@ __device__ __forceinline__ void patch_elem(uint4 &o0, uint4 &o1, int j, uint32_t
 #undef SZ_PATCH
 }
 
-constexpr int kEscBatch = 2048;  // escapes staged in shared memory per round
+// 256-bit codebook membership, 8 words, selected without local memory.
+__device__ __forceinline__ bool in_set8(const uint32_t s[8], uint32_t x) {
+    const uint32_t w = x >> 5;
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v = (w == (uint32_t)i) ? s[i] : v;
+    return (v >> (x & 31)) & 1u;
+}
 
+constexpr int kDecStages = 3;
+constexpr uint32_t kEscCap = 1024;  // escapes staged per sub-tile; more: consumers stream them
+constexpr uint16_t kNoEsc = 0xFFFFu;
+
+constexpr uint32_t kDFlagEnd = 1u;
+constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
+constexpr uint32_t kDFlagStaged = 4u;   // escapes are in the stage (else consumers stream them)
+
+struct DecMeta {
+    uint16_t *dst;      // global destination of the sub-tile's first element
+    const uint8_t *c;   // the segment's container
+    uint64_t elem0;     // first element of the sub-tile in the segment stream
+    uint64_t n, e;
+    uint64_t cb_lo, cb_hi;
+    uint32_t seg, len, flags, lo, cnt, pad;
+};
+
+struct __align__(128) DecShared {
+    uint8_t sm[kDecStages][kSub];
+    uint8_t codes[kDecStages][kSub / 2];
+    uint16_t esc_pos[kDecStages][kEscCap];  // sub-tile-local offsets
+    uint16_t chunk_first[kDecStages][kThreads * kChunks];
+    uint8_t esc_raw[kDecStages][kEscCap];
+    DecMeta meta[kDecStages];
+    uint64_t full[kDecStages];
+    uint64_t empty[kDecStages];
+    SegCache segc;
+    uint32_t inset[8];
+    int go;
+};
+
+// ------------------------------------------------------------ producer
 template <bool kBatched>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a) {
-    __shared__ SegCache s_segc;
-    __shared__ uint16_t s_epos[kEscBatch];  // tile-local offsets
-    __shared__ uint8_t s_eraw[kEscBatch];
-    __shared__ uint32_t s_inset[8];         // codebook membership bitmap
-
-    const int tid = threadIdx.x;
-    if (kBatched) seg_cache_fill(s_segc, a.batch);
-
+__device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
+    const int lane = threadIdx.x & 31;
+    if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
+    const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
+    const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
+    uint32_t j = 0;
     uint32_t cur = 0xFFFFFFFFu;
     sz_segment seg{};
     Header h{};
-    bool seg_ok = false;
-    DecTables T{};
+    uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const uint8_t *c = nullptr;
-
-    for (uint64_t tile = blockIdx.x; tile < a.batch.n_tiles; tile += gridDim.x) {
-        const uint32_t k = find_segment(s_segc, a.batch, tile);
-        int32_t *status = a.status + k;
+    bool tma_ok = false, pos_aligned = false;
+    for (uint64_t t = t_begin; t < t_end; ++t) {
+        const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
-            __syncthreads();  // done with the previous segment's shared bitmap
+            cur = k;
             seg = load_segment(a.batch, k);
             const uint64_t cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
             c = a.in + seg.out_offset;
             h = read_header(c, cap, seg.n_elems);
-            seg_ok = h.ok && codebook_distinct(h);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cbset[i] = 0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const uint32_t x = cb_entry(h.cb_lo, h.cb_hi, q);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cbset[i] |= ((x >> 5) == (uint32_t)i) ? (1u << (x & 31)) : 0u;
+            }
+            tma_ok = (seg.n_elems % 16) == 0;  // code stream 16-byte aligned (container is)
+            pos_aligned = ((kHeader + h.n + (h.n + 1) / 2) & 3) == 0;
+            if (!h.ok && lane == 0) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
+        }
+        if (!h.ok) continue;
+        const TileRef r = resolve_tile(a.batch, seg, k, t);
+        uint16_t *dst = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
+        const bool dst_aligned = (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
+        if (!dst_aligned && lane == 0) set_status(a.status + k, SZ_ERR_ALIGN);
+        const uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k + 4 * (uint64_t)r.local;
+        const uint8_t *pos = c + kHeader + h.n + (h.n + 1) / 2;
+        const uint8_t *raw = pos + 4 * h.e;
+        for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
+            const int s = (int)(j % kDecStages);
+            bool ok = true;
+            if (j >= (uint32_t)kDecStages && lane == 0)
+                ok = mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns);
+            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+            if (!ok) {
+                if (lane == 0) set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
+                return;
+            }
+            const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
+            const uint32_t len = umin32(kSub, r.len - sub * kSub);
+            uint32_t lo = ts[sub], hi = ts[sub + 1];
+            if (hi < lo || hi > h.e || hi - lo > len) {  // sub-tile starts not monotone
+                if (lane == 0) set_status(a.status + k, SZ_ERR_CORRUPT);
+                hi = lo = 0;
+            }
+            const uint32_t cnt = hi - lo;
+            const bool staged = cnt <= kEscCap;
+            if (staged) {
+                uint16_t *cf = sh.chunk_first[s];
+                for (uint32_t i = lane; i < (uint32_t)(kThreads * kChunks); i += 32) cf[i] = kNoEsc;
+                __syncwarp();
+                for (uint32_t i = lane; i < cnt; i += 32) {
+                    const uint64_t p = pos_aligned ? *reinterpret_cast<const uint32_t *>(pos + 4 * (uint64_t)(lo + i))
+                                                   : load_u32_any(pos + 4 * (uint64_t)(lo + i));
+                    const uint32_t x = raw[lo + i];
+                    const uint64_t pp = i == 0 ? 0 : load_u32_any(pos + 4 * (uint64_t)(lo + i - 1));
+                    bool bad = p < elem0 || p - elem0 >= len || in_set8(cbset, x) || (i > 0 && pp >= p);
+                    if (bad) set_status(a.status + k, SZ_ERR_CORRUPT);
+                    const uint32_t local = bad ? kNoEsc : (uint32_t)(p - elem0);
+                    sh.esc_pos[s][i] = (uint16_t)local;
+                    sh.esc_raw[s][i] = (uint8_t)x;
+                    const bool first = i == 0 || pp < elem0 || ((uint32_t)(pp - elem0) >> 4) != (local >> 4);
+                    if (!bad && first) cf[local >> 4] = (uint16_t)i;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                DecMeta &m = sh.meta[s];
+                m.dst = dst_aligned ? dst + sub * kSub : nullptr;
+                m.c = c;
+                m.elem0 = elem0;
+                m.n = h.n;
+                m.e = h.e;
+                m.cb_lo = h.cb_lo;
+                m.cb_hi = h.cb_hi;
+                m.seg = k;
+                m.len = len;
+                m.lo = lo;
+                m.cnt = cnt;
+                const bool tma = tma_ok && len == kSub;
+                m.flags = (tma ? kDFlagInSmem : 0u) | (staged ? kDFlagStaged : 0u);
+                if (tma) {
+                    mbar_arrive_expect_tx(&sh.full[s], kSub + kSub / 2);
+                    tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
+                    tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
+                } else {
+                    mbar_arrive(&sh.full[s]);
+                }
+            }
+            __syncwarp();
+        }
+    }
+    const int s = (int)(j % kDecStages);
+    bool ok = true;
+    if (j >= (uint32_t)kDecStages && lane == 0)
+        ok = mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns);
+    if (lane == 0 && ok) {
+        sh.meta[s].flags = kDFlagEnd;
+        mbar_arrive(&sh.full[s]);
+    }
+}
+
+// ------------------------------------------------------------ consumers
+template <bool kBatched>
+__device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t cur = 0xFFFFFFFFu;
+    DecTables T{};
+    for (uint32_t j = 0;; ++j) {
+        const int s = (int)(j % kDecStages);
+        if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
+        consumer_sync();
+        if (!sh.go) {  // the same decision in every consumer thread
+            if (tid == 0 && a.batch.n_tiles > 0) {
+                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.tiles_per_cta, a.batch.n_tiles - 1);
+                set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
+            }
+            return;
+        }
+        const DecMeta m = sh.meta[s];
+        if (m.flags & kDFlagEnd) return;
+        if (m.seg != cur) {
+            T = make_tables(m.cb_lo, m.cb_hi);
             if (tid < 8) {
                 uint32_t w = 0;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t e = cb_entry(h, i);
-                    if ((e >> 5) == (uint32_t)tid) w |= 1u << (e & 31);
+                for (int q = 0; q < 16; ++q) {
+                    const uint32_t x = cb_entry(m.cb_lo, m.cb_hi, q);
+                    if ((x >> 5) == (uint32_t)tid) w |= 1u << (x & 31);
                 }
-                s_inset[tid] = w;
+                sh.inset[tid] = w;
             }
-            T = make_tables(h);
-            cur = k;
-            if (tid == 0 && !seg_ok) set_status(status, SZ_ERR_CORRUPT);
-            __syncthreads();
+            cur = m.seg;
+            consumer_sync();
         }
-        if (!seg_ok) continue;
-
-        const TileRef r = resolve_tile(a.batch, seg, k, tile);
-        uint16_t *dst = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
-        const bool dst_aligned = (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
-        const uint8_t *in_sm = c + kHeader + r.elem0;
-        const uint8_t *codes_base = c + kHeader + r.n;
-        const bool codes_aligned = (r.n % 8) == 0;
-        const uint8_t *pos = c + kHeader + r.n + (r.n + 1) / 2;
-        const uint8_t *raw = pos + 4 * h.e;
-        const uint32_t *ts = a.tile_start + seg.tile_begin + k;
-        uint32_t lo = ts[r.local], hi = ts[r.local + 1];
-        if (!dst_aligned && tid == 0) set_status(status, SZ_ERR_ALIGN);
-        if (hi < lo || hi > h.e || hi - lo > r.len) {  // tile starts not monotone
-            if (tid == 0) set_status(status, SZ_ERR_CORRUPT);
-            hi = lo = 0;
-        }
+        int32_t *status = a.status + m.seg;
+        const bool in_smem = (m.flags & kDFlagInSmem) != 0;
+        const bool codes_aligned = (m.n % 8) == 0;
+        const uint8_t *in_sm = m.c + kHeader + m.elem0;
+        const uint8_t *codes_base = m.c + kHeader + m.n;
 
         // ---- decode all chunks into registers
         uint4 o[2 * kChunks];
         uint64_t cw[kChunks];
-        const bool fast = r.len == kTile && codes_aligned && dst_aligned;
-        if (fast) {
-            uint4 smv[kChunks];
 #pragma unroll
-            for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                smv[q] = ld_stream_v4(in_sm + off);
-                cw[q] = __ldcs(reinterpret_cast<const unsigned long long *>(codes_base + (r.elem0 + off) / 2));
+        for (int q = 0; q < kChunks; ++q) {
+            const uint32_t ci = q * kThreads + tid;
+            const uint32_t off = ci * kChunk;
+            const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
+            uint4 smv = make_uint4(0, 0, 0, 0);
+            uint64_t codes = 0;
+            if (in_smem) {
+                smv = *reinterpret_cast<const uint4 *>(sh.sm[s] + off);
+                codes = *reinterpret_cast<const unsigned long long *>(sh.codes[s] + off / 2);
+            } else if (cnt == (uint32_t)kChunk && codes_aligned) {
+                smv = ld_stream_v4(in_sm + off);
+                codes = *reinterpret_cast<const unsigned long long *>(codes_base + (m.elem0 + off) / 2);
+            } else if (cnt) {
+                uint32_t sw[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int jj = 0; jj < kChunk; ++jj)
+                    if (jj < (int)cnt) sw[jj >> 2] |= (uint32_t)in_sm[off + jj] << (8 * (jj & 3));
+                smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+                const uint8_t *cb = codes_base + (m.elem0 + off) / 2;
+#pragma unroll
+                for (int b = 0; b < kChunk / 2; ++b)
+                    if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
+                // odd element count: the unused high nibble must be 0
+                if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+                if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
             }
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) decode_chunk(smv[q], cw[q], T, o[2 * q], o[2 * q + 1]);
-        } else {
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                const uint32_t cnt = off < r.len ? umin32(kChunk, r.len - off) : 0u;
-                uint4 smv = make_uint4(0, 0, 0, 0);
-                uint64_t codes = 0;
-                if (cnt == (uint32_t)kChunk && codes_aligned) {
-                    smv = ld_stream_v4(in_sm + off);
-                    codes = *reinterpret_cast<const unsigned long long *>(codes_base + (r.elem0 + off) / 2);
-                } else if (cnt) {
-                    uint32_t sw[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int j = 0; j < kChunk; ++j)
-                        if (j < (int)cnt) sw[j >> 2] |= (uint32_t)in_sm[off + j] << (8 * (j & 3));
-                    smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-                    const uint8_t *cb = codes_base + (r.elem0 + off) / 2;
-#pragma unroll
-                    for (int b = 0; b < kChunk / 2; ++b)
-                        if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
-                    // odd element count: the unused high nibble must be 0
-                    if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                    if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
-                }
-                cw[q] = codes;
-                decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
-            }
+            cw[q] = codes;
+            decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
         }
 
-        // ---- escapes of this tile, staged through shared memory
-        for (uint32_t b0 = lo; b0 < hi; b0 += kEscBatch) {
-            const uint32_t nb = umin32(kEscBatch, hi - b0);
-            __syncthreads();
-            for (uint32_t i = tid; i < nb; i += kThreads) {
-                const uint64_t p = load_u32_any(pos + 4 * (uint64_t)(b0 + i));
-                const uint32_t x = raw[b0 + i];
-                bool bad = p < r.elem0 || p >= r.elem0 + r.len;
-                if (b0 + i > lo) bad |= load_u32_any(pos + 4 * (uint64_t)(b0 + i - 1)) >= p;
-                bad |= (s_inset[x >> 5] >> (x & 31)) & 1u;
-                if (bad) set_status(status, SZ_ERR_CORRUPT);
-                s_epos[i] = bad ? 0xFFFFu : (uint16_t)(p - r.elem0);
-                s_eraw[i] = (uint8_t)x;
-            }
-            __syncthreads();
+        // ---- escapes
+        if (m.flags & kDFlagStaged) {
+            const uint16_t *cf = sh.chunk_first[s];
+            const uint16_t *ep = sh.esc_pos[s];
+            const uint8_t *er = sh.esc_raw[s];
 #pragma unroll
             for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                uint32_t a0 = 0, a1 = nb;  // first staged escape at or after off
-                while (a0 < a1) {
-                    const uint32_t mid = (a0 + a1) >> 1;
-                    if (s_epos[mid] < off) a0 = mid + 1; else a1 = mid;
+                const uint32_t ci = q * kThreads + tid;
+                uint32_t i = cf[ci];
+                if (i == kNoEsc) continue;
+                for (; i < m.cnt; ++i) {
+                    const uint32_t l = ep[i];
+                    if ((l >> 4) != ci) break;  // next chunk (or a rejected entry)
+                    const int jj = (int)(l & 15u);
+                    if (((cw[q] >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+                    patch_elem(o[2 * q], o[2 * q + 1], jj, er[i]);
                 }
-                for (uint32_t i = a0; i < nb && s_epos[i] < off + kChunk; ++i) {
-                    const int j = (int)(s_epos[i] - off);
-                    if (((cw[q] >> (4 * j)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                    patch_elem(o[2 * q], o[2 * q + 1], j, s_eraw[i]);
+            }
+        } else {
+            // more escapes than one stage holds: stream them through the
+            // stage's escape area in batches (every consumer takes part)
+            const uint8_t *pos = m.c + kHeader + m.n + (m.n + 1) / 2;
+            const uint8_t *raw = pos + 4 * m.e;
+            uint16_t *ep = sh.esc_pos[s];
+            uint8_t *er = sh.esc_raw[s];
+            for (uint32_t b0 = 0; b0 < m.cnt; b0 += kEscCap) {
+                const uint32_t nb = umin32(kEscCap, m.cnt - b0);
+                consumer_sync();
+                for (uint32_t i = tid; i < nb; i += kThreads) {
+                    const uint64_t g = (uint64_t)m.lo + b0 + i;
+                    const uint64_t p = load_u32_any(pos + 4 * g);
+                    const uint32_t x = raw[g];
+                    bool bad = p < m.elem0 || p - m.elem0 >= m.len;
+                    if (b0 + i > 0) bad |= load_u32_any(pos + 4 * (g - 1)) >= p;
+                    bad |= (sh.inset[x >> 5] >> (x & 31)) & 1u;
+                    if (bad) set_status(status, SZ_ERR_CORRUPT);
+                    ep[i] = bad ? kNoEsc : (uint16_t)(p - m.elem0);
+                    er[i] = (uint8_t)x;
+                }
+                consumer_sync();
+#pragma unroll
+                for (int q = 0; q < kChunks; ++q) {
+                    const uint32_t off = (q * kThreads + tid) * kChunk;
+                    uint32_t a0 = 0, a1 = nb;  // first staged escape at or after off
+                    while (a0 < a1) {
+                        const uint32_t mid = (a0 + a1) >> 1;
+                        if (ep[mid] < off) a0 = mid + 1; else a1 = mid;
+                    }
+                    for (uint32_t i = a0; i < nb && ep[i] < off + kChunk; ++i) {
+                        const int jj = (int)(ep[i] - off);
+                        if (((cw[q] >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+                        patch_elem(o[2 * q], o[2 * q + 1], jj, er[i]);
+                    }
                 }
             }
         }
 
         // ---- store
-        if (fast) {
+        if (m.dst != nullptr) {
 #pragma unroll
             for (int q = 0; q < kChunks; ++q) {
                 const uint32_t off = (q * kThreads + tid) * kChunk;
-                st_stream_v4(dst + off, o[2 * q]);
-                st_stream_v4(dst + off + 8, o[2 * q + 1]);
-            }
-        } else {
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                const uint32_t cnt = off < r.len ? umin32(kChunk, r.len - off) : 0u;
-                if (cnt == (uint32_t)kChunk && dst_aligned) {
-                    st_stream_v4(dst + off, o[2 * q]);
-                    st_stream_v4(dst + off + 8, o[2 * q + 1]);
-                } else if (cnt && dst_aligned) {
+                const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
+                if (cnt == (uint32_t)kChunk) {
+                    st_stream_v4(m.dst + off, o[2 * q]);
+                    st_stream_v4(m.dst + off + 8, o[2 * q + 1]);
+                } else if (cnt) {
                     const uint32_t w[8] = {o[2 * q].x, o[2 * q].y, o[2 * q].z, o[2 * q].w,
                                            o[2 * q + 1].x, o[2 * q + 1].y, o[2 * q + 1].z, o[2 * q + 1].w};
 #pragma unroll
-                    for (int j = 0; j < kChunk; ++j)
-                        if (j < (int)cnt) dst[off + j] = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
+                    for (int jj = 0; jj < kChunk; ++jj)
+                        if (jj < (int)cnt) m.dst[off + jj] = (uint16_t)(w[jj >> 1] >> (16 * (jj & 1)));
                 }
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
     }
 }
 
+template <bool kBatched>
+__global__ void __launch_bounds__(kPipeThreads, 2) decode_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    DecShared &sh = *reinterpret_cast<DecShared *>(smem_raw);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], kWarps);
+        }
+        fence_mbar_init();
+    }
+    seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
+    if (tid >= kThreads)
+        decode_producer<kBatched>(a, sh);
+    else
+        decode_consumers<kBatched>(a, sh);
+}
+
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {
-    const uint64_t entries = a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
+    const uint64_t entries = 4 * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
     const uint64_t grid = div_up(entries, 256);
     if (batched)
         esc_index_kernel<true><<<(unsigned)grid, 256, 0, s>>>(a, entries);
@@ -343,19 +517,31 @@ cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) 
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStream_t s) {
+    DecodeArgs a = a0;
     if (a.batch.n_tiles == 0) return cudaSuccess;
+    const size_t smem = sizeof(DecShared);
     grid = (int)umax64(1, umin64((uint64_t)grid, a.batch.n_tiles));
-    if (batched)
-        decode_kernel<true><<<grid, kThreads, 0, s>>>(a);
-    else
-        decode_kernel<false><<<grid, kThreads, 0, s>>>(a);
+    a.tiles_per_cta = div_up(a.batch.n_tiles, (uint64_t)grid);
+    grid = (int)div_up(a.batch.n_tiles, a.tiles_per_cta);
+    cudaError_t e;
+    if (batched) {
+        e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        decode_kernel<true><<<grid, kPipeThreads, smem, s>>>(a);
+    } else {
+        e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        decode_kernel<false><<<grid, kPipeThreads, smem, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
 int decode_blocks_per_sm() {
+    const size_t smem = sizeof(DecShared);
+    cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<true>, kThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<true>, kPipeThreads, smem);
     return occ > 0 ? occ : 1;
 }
 

@@ -5,17 +5,52 @@
 // 4-bit code of its codebook slot (two codes per byte), and an exponent
 // outside the codebook becomes an escape note (position, raw exponent).
 // Section 4: fixed-length codes make this one straight pass -- every output
-// byte's address is known from the element index, except the escape
-// records, whose place is the number of escapes before them.
+// byte's address follows from the element index, and each tile's first
+// escape index is already known from the per-tile histograms, so tiles are
+// independent.
 //
-// One persistent kernel: CTAs draw tiles from an atomic ticket (so a tile's
-// predecessors are always running or done), write the sm and code streams
-// with coalesced 16-byte / 8-byte stores, count escapes per thread-chunk,
-// scan the counts across the CTA, and find the tile's starting escape index
-// with a decoupled lookback over the tiles before it in the same segment.
+// One persistent CTA per slot, warp-specialised:
+//   producer warp   walks the CTA's tiles, 1-D TMA bulk copy of each
+//                   16,384-element sub-tile (32 KiB) into a 3-stage
+//                   shared-memory ring, signalled by mbarriers;
+//   8 consumer warps read the stage, write the sm stream (16-byte stores)
+//                   and code stream (8-byte stores), scan the escape counts
+//                   across the CTA and write the escape records in element
+//                   order, then release the stage.
+// Every mbarrier wait is bounded (SZ_ERR_DEVICE_TIMEOUT).
 #include "sz_internal.cuh"
 
 namespace sz {
+
+constexpr int kEncStages = 3;
+
+constexpr uint32_t kFlagEnd = 1u;        // no more sub-tiles
+constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
+constexpr uint32_t kFlagLastSub = 4u;    // last sub-tile of its tile
+constexpr uint32_t kFlagHeader = 8u;     // first sub-tile of the segment: write the header
+constexpr uint32_t kFlagLastTile = 16u;  // last tile of the segment: write the size
+
+struct EncMeta {
+    const uint16_t *src;  // global address of the sub-tile's first element
+    uint64_t elem0;       // first element of the sub-tile in the segment stream
+    uint32_t seg;
+    uint32_t len;         // elements of the sub-tile
+    uint32_t flags;
+    uint32_t esc_base;    // first escape index of the tile
+    uint32_t esc_count;   // escapes the tile must produce
+    uint32_t pad;
+};
+
+struct __align__(128) EncShared {
+    uint8_t stage[kEncStages][kSub * 2];
+    EncMeta meta[kEncStages];
+    uint64_t full[kEncStages];
+    uint64_t empty[kEncStages];
+    SegCache segc;
+    uint64_t warp_tot[kWarps];
+    uint8_t lut[256];
+    int go;
+};
 
 // ---------------------------------------------------------- chunk encode
 // 16 consecutive BF16 values (two uint4) -> 16 sm bytes, 8 code bytes and an
@@ -89,38 +124,283 @@ __device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligne
     }
 }
 
-// Warp-wide inclusive scan of a packed u64 (four 16-bit counters).
-__device__ __forceinline__ uint64_t warp_incl_scan(uint64_t v, int lane) {
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, v, d);
-        if (lane >= d) v += y;
-    }
-    return v;
-}
-
 __device__ __forceinline__ uint32_t field16(uint64_t v, int c) { return (uint32_t)(v >> (16 * c)) & 0xFFFFu; }
 
-template <bool kBatched>
-__global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a) {
-    __shared__ SegCache s_segc;
-    __shared__ __align__(16) uint8_t s_lut[256];
-    __shared__ uint64_t s_warp[kWarps];
-    __shared__ unsigned long long s_tile;
-    __shared__ uint32_t s_excl;
-    __shared__ int s_timeout;
+// Read chunk (c, tid) of a stage: 32 bytes at (c*256 + tid)*32.  Lanes with
+// bit 2 set read the upper half first, so each quarter-warp's 16-byte reads
+// cover all 32 banks exactly once.
+__device__ __forceinline__ void read_chunk_smem(const uint8_t *stage, int c, int tid, uint4 &v0, uint4 &v1) {
+    const uint8_t *p = stage + (uint32_t)(c * kThreads + tid) * 32u;
+    const uint32_t h = ((uint32_t)tid >> 2) & 1u;
+    const uint4 a = *reinterpret_cast<const uint4 *>(p + 16 * h);
+    const uint4 b = *reinterpret_cast<const uint4 *>(p + 16 * (1 - h));
+    v0 = h ? b : a;
+    v1 = h ? a : b;
+}
 
+// Chunk from global memory, `cnt` (<= 16) valid elements, the rest zero.
+__device__ __forceinline__ void read_chunk_global(const uint16_t *p, uint32_t cnt, uint4 &v0, uint4 &v1) {
+    uint32_t wv[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint32_t lo = (2 * q < (int)cnt) ? (uint32_t)p[2 * q] : 0u;
+        const uint32_t hi = (2 * q + 1 < (int)cnt) ? (uint32_t)p[2 * q + 1] : 0u;
+        wv[q] = lo | (hi << 16);
+    }
+    v0 = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    v1 = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+}
+
+// ------------------------------------------------------------ producer
+template <bool kBatched>
+__device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
+    if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
+    const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
+    const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
+    uint32_t j = 0;
+    uint32_t cur = 0xFFFFFFFFu;
+    sz_segment seg{};
+    bool seg_ok = false;
+    uint64_t e_total = 0;
+    for (uint64_t t = t_begin; t < t_end; ++t) {
+        const uint32_t k = find_segment(sh.segc, a.batch, t);
+        if (k != cur) {
+            cur = k;
+            seg = load_segment(a.batch, k);
+            const SegMeta &m = a.meta[k];
+            e_total = m.n_escapes;
+            const bool fits = seg.out_offset <= a.out_cap &&
+                              container_size(seg.n_elems, e_total) <= a.out_cap - seg.out_offset;
+            const bool aligned = (reinterpret_cast<uintptr_t>(a.out + seg.out_offset) & 15) == 0;
+            seg_ok = m.valid != 0 && fits && aligned;
+            if (m.valid == 0) set_status(a.status + k, SZ_ERR_INVALID);
+            else if (!fits) set_status(a.status + k, SZ_ERR_CAPACITY);
+            else if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
+        }
+        if (!seg_ok) continue;  // every tile of the segment is skipped
+        const TileRef r = resolve_tile(a.batch, seg, k, t);
+        const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
+        const uint32_t off = a.tile_off[t];
+        const uint64_t next = (r.local + 1 < r.tiles) ? (uint64_t)a.tile_off[t + 1] : e_total;
+        const bool aligned = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+        if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
+        for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
+            const int s = (int)(j % kEncStages);
+            if (j >= (uint32_t)kEncStages && !mbar_wait(&sh.empty[s], ((j / kEncStages) - 1) & 1u, a.wait_limit_ns)) {
+                set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
+                return;
+            }
+            EncMeta &m = sh.meta[s];
+            m.src = src + sub * kSub;
+            m.elem0 = r.elem0 + (uint64_t)sub * kSub;
+            m.seg = k;
+            m.len = aligned ? umin32(kSub, r.len - sub * kSub) : 0u;  // nothing is read from a misaligned page
+            m.esc_base = off;
+            m.esc_count = (uint32_t)(next - off);
+            uint32_t f = 0;
+            if (sub + 1 == r.n_subs) f |= kFlagLastSub;
+            if (r.local == 0 && sub == 0) f |= kFlagHeader;
+            if (r.local + 1 == r.tiles) f |= kFlagLastTile;
+            const bool tma = m.len == kSub;
+            if (tma) f |= kFlagInSmem;
+            m.flags = f;
+            if (tma) {
+                mbar_arrive_expect_tx(&sh.full[s], kSub * 2);
+                tma_load_1d(sh.stage[s], m.src, kSub * 2, &sh.full[s]);
+            } else {
+                mbar_arrive(&sh.full[s]);
+            }
+        }
+    }
+    const int s = (int)(j % kEncStages);
+    if (j >= (uint32_t)kEncStages && !mbar_wait(&sh.empty[s], ((j / kEncStages) - 1) & 1u, a.wait_limit_ns)) return;
+    sh.meta[s].flags = kFlagEnd;
+    mbar_arrive(&sh.full[s]);
+}
+
+// ------------------------------------------------------------ consumers
+template <bool kBatched>
+__device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (kBatched) seg_cache_fill(s_segc, a.batch);
+    uint32_t cur = 0xFFFFFFFFu;
+    uint8_t *out = nullptr;
+    uint64_t n = 0, e_total = 0;
+    bool codes_aligned = false, pos_aligned = false;
+    uint32_t running = 0;  // escapes of the current tile so far
+    for (uint32_t j = 0;; ++j) {
+        const int s = (int)(j % kEncStages);
+        if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kEncStages) & 1u, a.wait_limit_ns) ? 1 : 0;
+        consumer_sync();
+        if (!sh.go) {  // the same decision in every consumer thread
+            if (tid == 0 && a.batch.n_tiles > 0) {
+                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.tiles_per_cta, a.batch.n_tiles - 1);
+                set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
+            }
+            return;
+        }
+        const EncMeta m = sh.meta[s];
+        if (m.flags & kFlagEnd) return;
+        if (m.seg != cur) {  // every consumer finished the previous sub-tile (barrier above)
+            sh.lut[tid] = 0x80;
+            consumer_sync();
+            const SegMeta &g = a.meta[m.seg];
+            if (tid < 16) sh.lut[g.codebook[tid]] = (uint8_t)tid;
+            const sz_segment seg = load_segment(a.batch, m.seg);
+            out = a.out + seg.out_offset;
+            n = seg.n_elems;
+            e_total = g.n_escapes;
+            codes_aligned = (n % 8) == 0;
+            pos_aligned = ((kHeader + n + (n + 1) / 2) & 3) == 0;
+            cur = m.seg;
+            consumer_sync();
+        }
+        int32_t *status = a.status + m.seg;
+        if ((m.flags & kFlagHeader) && tid < 6) {
+            uint64_t v = 0;
+            if (tid == 0) v = 0x00000101564B5A53ull;  // "SZKV", version 1, dtype 1, flags 0
+            if (tid == 1) v = n;
+            if (tid == 2) v = e_total;
+            if (tid == 3 || tid == 4) {
+                const uint8_t *cb = a.meta[m.seg].codebook + 8 * (tid - 3);
+                for (int i = 7; i >= 0; --i) v = (v << 8) | cb[i];
+            }
+            reinterpret_cast<uint64_t *>(out)[tid] = v;
+        }
+        uint8_t *out_sm = out + kHeader + m.elem0;
+        uint8_t *codes_base = out + kHeader + n;  // element i's nibble is in byte i/2
+        const uint8_t *stage = sh.stage[s];
+        const bool in_smem = (m.flags & kFlagInSmem) != 0;
+
+        uint32_t esc[kChunks];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            const uint32_t off = (c * kThreads + tid) * kChunk;
+            esc[c] = 0;
+            if (off >= m.len) continue;
+            uint4 v0, v1, smv;
+            uint64_t cw;
+            if (in_smem && codes_aligned) {
+                read_chunk_smem(stage, c, tid, v0, v1);
+                encode_chunk(v0, v1, sh.lut, smv, cw, esc[c]);
+                st_stream_v4(out_sm + off, smv);
+                st_stream_u64(codes_base + (m.elem0 + off) / 2, cw);
+                continue;
+            }
+            // ragged or unaligned chunk: guarded element loads, encoded as a
+            // full chunk, cnt of it kept
+            const uint32_t cnt = umin32(kChunk, m.len - off);
+            read_chunk_global(m.src + off, cnt, v0, v1);
+            uint32_t e;
+            encode_chunk(v0, v1, sh.lut, smv, cw, e);
+            uint32_t keep = 0;
+#pragma unroll
+            for (int q = 0; q < kChunk; ++q)
+                if (q < (int)cnt) keep |= esc_bit_of_elem(q);
+            esc[c] = e & keep;
+            if (cnt < (uint32_t)kChunk) cw &= (1ull << (4 * cnt)) - 1ull;  // odd tail nibble = 0
+            if (cnt == (uint32_t)kChunk && codes_aligned) {
+                st_stream_v4(out_sm + off, smv);
+                st_stream_u64(codes_base + (m.elem0 + off) / 2, cw);
+            } else {
+#pragma unroll
+                for (int q = 0; q < kChunk; ++q)
+                    if (q < (int)cnt) out_sm[off + q] = (uint8_t)byte_of(smv, q);
+                uint8_t *cb = codes_base + (m.elem0 + off) / 2;
+#pragma unroll
+                for (int b = 0; b < kChunk / 2; ++b)
+                    if (2 * b < (int)cnt) cb[b] = (uint8_t)(cw >> (8 * b));
+            }
+        }
+
+        // ---- escapes: CTA scan of the per-chunk counts, packed 4 x 16 bit
+        uint64_t cnt = 0;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) cnt |= (uint64_t)__popc(esc[c]) << (16 * c);
+        uint64_t incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        if (lane == 31) sh.warp_tot[wid] = incl;
+        consumer_sync();
+        uint64_t warp_excl = 0, tot = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const uint64_t v = sh.warp_tot[w];
+            if (w < wid) warp_excl += v;
+            tot += v;
+        }
+        const uint64_t thr_excl = warp_excl + incl - cnt;
+        const uint32_t sub_total = field16(tot, 0) + field16(tot, 1) + field16(tot, 2) + field16(tot, 3);
+
+        // ---- escape records, in element order
+        const uint64_t pos_off = kHeader + n + (n + 1) / 2;
+        uint8_t *pos_base = out + pos_off;
+        uint8_t *raw_base = pos_base + 4 * e_total;
+        uint32_t chunk_base = running;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            uint32_t msk = esc[c] ? esc_in_element_order(esc[c]) : 0u;
+            uint32_t idx = chunk_base + field16(thr_excl, c);
+            chunk_base += field16(tot, c);
+            if (!msk) continue;
+            const uint32_t off = (c * kThreads + tid) * kChunk;
+            uint4 v0, v1;
+            if (in_smem) read_chunk_smem(stage, c, tid, v0, v1);
+            else read_chunk_global(m.src + off, umin32(kChunk, m.len - off), v0, v1);
+            while (msk) {  // ascending element order
+                const int q = __ffs(msk) - 1;
+                msk &= msk - 1;
+                const uint64_t g = (uint64_t)m.esc_base + idx;
+                if (idx >= m.esc_count || g >= e_total) {  // more escapes than the histograms said
+                    set_status(status, SZ_ERR_CORRUPT);
+                    break;
+                }
+                store_u32_le(pos_base + 4 * g, (uint32_t)(m.elem0 + off + q), pos_aligned);
+                raw_base[g] = (uint8_t)exponent_of_chunk_elem(v0, v1, q);
+                ++idx;
+            }
+        }
+        running += sub_total;
+        if (m.flags & kFlagLastSub) {
+            if (tid == 0) {
+                if (running != m.esc_count) set_status(status, SZ_ERR_CORRUPT);
+                else if (m.flags & kFlagLastTile) a.out_bytes[m.seg] = container_size(n, e_total);
+            }
+            running = 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[s]);
+    }
+}
+
+template <bool kBatched>
+__global__ void __launch_bounds__(kPipeThreads, 2) encode_kernel(const EncodeArgs a) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    EncShared &sh = *reinterpret_cast<EncShared *>(smem_raw);
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kEncStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], kWarps);
+        }
+        fence_mbar_init();
+    }
+    seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
 
     // Segments with no elements have no tiles: CTA 0 writes their header.
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0 && tid < kThreads) {
         const uint32_t ns = kBatched ? a.batch.n_segs : 1;
         for (uint32_t k = tid; k < ns; k += kThreads) {
             const sz_segment s = load_segment(a.batch, k);
             if (s.n_elems != 0) continue;
-            if (a.meta[k].valid == 0) { set_status(a.status ? a.status + k : nullptr, SZ_ERR_INVALID); continue; }
-            if (s.out_offset + kHeader > a.out_cap) { set_status(a.status ? a.status + k : nullptr, SZ_ERR_CAPACITY); continue; }
+            if (a.meta[k].valid == 0) { set_status(a.status + k, SZ_ERR_INVALID); continue; }
+            if (s.out_offset + kHeader > a.out_cap) { set_status(a.status + k, SZ_ERR_CAPACITY); continue; }
+            if ((reinterpret_cast<uintptr_t>(a.out + s.out_offset) & 15) != 0) {
+                set_status(a.status + k, SZ_ERR_ALIGN);
+                continue;
+            }
             uint64_t *h = reinterpret_cast<uint64_t *>(a.out + s.out_offset);
             const uint8_t *cb = a.meta[k].codebook;
             uint64_t c0 = 0, c1 = 0;
@@ -135,246 +415,38 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
         }
     }
 
-    uint32_t cur = 0xFFFFFFFFu;
-    sz_segment seg{};
-    uint64_t e_total = 0;
-    bool seg_ok = false;
-
-    while (true) {
-        __syncthreads();  // every thread is done with the previous tile's shared state
-        if (tid == 0) s_tile = atomicAdd(a.ticket, 1ull);
-        __syncthreads();
-        const uint64_t tile = s_tile;
-        if (tile >= a.batch.n_tiles) break;
-        const uint32_t k = find_segment(s_segc, a.batch, tile);
-        int32_t *status = a.status ? a.status + k : nullptr;
-        if (k != cur) {
-            seg = load_segment(a.batch, k);
-            s_lut[tid] = 0x80;
-            __syncthreads();
-            const SegMeta *m = a.meta + k;
-            if (tid < 16) s_lut[m->codebook[tid]] = (uint8_t)tid;
-            e_total = m->n_escapes;
-            const bool valid = m->valid != 0;
-            const bool fits = seg.out_offset <= a.out_cap &&
-                              container_size(seg.n_elems, e_total) <= a.out_cap - seg.out_offset;
-            seg_ok = valid && fits;
-            if (tid == 0 && !valid) set_status(status, SZ_ERR_INVALID);
-            if (tid == 0 && valid && !fits) set_status(status, SZ_ERR_CAPACITY);
-            __syncthreads();
-            cur = k;
-        }
-        // An invalid segment is skipped by every one of its tiles, so no
-        // tile ever waits on it.
-        if (!seg_ok) continue;
-
-        const TileRef r = resolve_tile(a.batch, seg, k, tile);
-        const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
-        uint8_t *out = a.out + seg.out_offset;
-        uint8_t *out_sm = out + kHeader + r.elem0;
-        uint8_t *codes_base = out + kHeader + r.n;  // element i's nibble is in byte i/2
-        const bool codes_aligned = (r.n % 8) == 0;
-        const bool src_aligned = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-        if (!src_aligned) {  // only batched pages can be misaligned here
-            if (tid == 0) set_status(status, SZ_ERR_ALIGN);
-        }
-
-        // Header of the segment: written once, by its first tile.
-        if (r.local == 0 && tid < 6) {
-            uint64_t v = 0;
-            if (tid == 0) v = 0x00000101564B5A53ull;
-            if (tid == 1) v = r.n;
-            if (tid == 2) v = e_total;
-            if (tid == 3 || tid == 4) {
-                for (int i = 7; i >= 0; --i) v = (v << 8) | a.meta[k].codebook[8 * (tid - 3) + i];
-            }
-            reinterpret_cast<uint64_t *>(out)[tid] = v;
-        }
-
-        uint4 in[2 * kChunks];
-        uint32_t esc[kChunks];
-        if (r.len == kTile && codes_aligned && src_aligned) {
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                const uint16_t *p = src + (c * kThreads + tid) * kChunk;
-                in[2 * c] = ld_stream_v4(p);
-                in[2 * c + 1] = ld_stream_v4(p + 8);
-            }
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                const uint32_t off = (c * kThreads + tid) * kChunk;
-                uint4 smv;
-                uint64_t cw;
-                encode_chunk(in[2 * c], in[2 * c + 1], s_lut, smv, cw, esc[c]);
-                st_stream_v4(out_sm + off, smv);
-                st_stream_u64(codes_base + (r.elem0 + off) / 2, cw);
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                const uint32_t off = (c * kThreads + tid) * kChunk;
-                esc[c] = 0;
-                in[2 * c] = make_uint4(0, 0, 0, 0);
-                in[2 * c + 1] = make_uint4(0, 0, 0, 0);
-                if (!src_aligned || off >= r.len) continue;
-                if (off + kChunk <= r.len && codes_aligned) {
-                    in[2 * c] = ld_stream_v4(src + off);
-                    in[2 * c + 1] = ld_stream_v4(src + off + 8);
-                    uint4 smv;
-                    uint64_t cw;
-                    encode_chunk(in[2 * c], in[2 * c + 1], s_lut, smv, cw, esc[c]);
-                    st_stream_v4(out_sm + off, smv);
-                    st_stream_u64(codes_base + (r.elem0 + off) / 2, cw);
-                } else {
-                    // ragged or unaligned chunk: assemble the cnt values with
-                    // guarded loads, encode as a full chunk, keep cnt of it
-                    const uint32_t cnt = umin32(kChunk, r.len - off);
-                    uint32_t wv[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint32_t lo = (2 * q < (int)cnt) ? (uint32_t)src[off + 2 * q] : 0u;
-                        const uint32_t hi = (2 * q + 1 < (int)cnt) ? (uint32_t)src[off + 2 * q + 1] : 0u;
-                        wv[q] = lo | (hi << 16);
-                    }
-                    in[2 * c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                    in[2 * c + 1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-                    uint4 smv;
-                    uint64_t cw;
-                    uint32_t e;
-                    encode_chunk(in[2 * c], in[2 * c + 1], s_lut, smv, cw, e);
-                    uint32_t keep = 0;
-#pragma unroll
-                    for (int j = 0; j < kChunk; ++j)
-                        if (j < (int)cnt) keep |= esc_bit_of_elem(j);
-                    esc[c] = e & keep;
-                    if (cnt < (uint32_t)kChunk) cw &= (1ull << (4 * cnt)) - 1ull;  // odd tail nibble = 0
-#pragma unroll
-                    for (int j = 0; j < kChunk; ++j)
-                        if (j < (int)cnt) out_sm[off + j] = (uint8_t)byte_of(smv, j);
-                    uint8_t *cb = codes_base + (r.elem0 + off) / 2;
-#pragma unroll
-                    for (int b = 0; b < kChunk / 2; ++b)
-                        if (2 * b < (int)cnt) cb[b] = (uint8_t)(cw >> (8 * b));
-                }
-            }
-        }
-
-        // ---- escapes: CTA scan of the per-chunk counts, packed 4 x 16 bit
-        uint64_t cnt = 0;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) cnt |= (uint64_t)__popc(esc[c]) << (16 * c);
-        const uint64_t incl = warp_incl_scan(cnt, lane);
-        if (lane == 31) s_warp[wid] = incl;
-        __syncthreads();
-        uint64_t warp_excl = 0, tile_tot = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const uint64_t v = s_warp[w];
-            if (w < wid) warp_excl += v;
-            tile_tot += v;
-        }
-        const uint64_t thr_excl = warp_excl + incl - cnt;
-        const uint32_t total = field16(tile_tot, 0) + field16(tile_tot, 1) + field16(tile_tot, 2) +
-                               field16(tile_tot, 3);
-
-        // ---- decoupled lookback (warp 0)
-        if (wid == 0) {
-            const bool publish = (a.debug_flags & kDebugNoPublish) == 0;
-            uint64_t *st = a.tile_status;
-            uint32_t excl = 0;
-            bool timeout = false;
-            if (tile == seg.tile_begin) {
-                if (lane == 0 && publish) st_relaxed_u64(st + tile, kFlagPrefix | total);
-            } else {
-                if (lane == 0 && publish) st_relaxed_u64(st + tile, kFlagAggregate | total);
-                const int64_t first = (int64_t)seg.tile_begin;
-                int64_t pred = (int64_t)tile - 1;
-                const uint64_t t0 = globaltimer_ns();
-                while (true) {
-                    const int64_t idx = pred - lane;
-                    const uint64_t s = idx >= first ? ld_relaxed_u64(st + idx) : kFlagPrefix;
-                    const uint32_t not_ready = __ballot_sync(0xFFFFFFFFu, (s & kFlagMask) == 0);
-                    const uint32_t prefix = __ballot_sync(0xFFFFFFFFu, (s & kFlagMask) == kFlagPrefix);
-                    const int p_lane = prefix ? __ffs(prefix) - 1 : 32;
-                    const uint32_t upto = p_lane >= 31 ? 0xFFFFFFFFu : ((2u << p_lane) - 1u);
-                    if (not_ready & upto) {
-                        const bool expired = globaltimer_ns() - t0 > a.wait_limit_ns;
-                        if (__any_sync(0xFFFFFFFFu, expired)) {
-                            timeout = true;
-                            break;
-                        }
-                        __nanosleep(100);
-                        continue;
-                    }
-                    const uint32_t v = (lane <= p_lane) ? (uint32_t)s : 0u;
-                    excl += __reduce_add_sync(0xFFFFFFFFu, v);
-                    if (p_lane < 32) break;
-                    pred -= 32;
-                }
-                // Publish even after a timeout so later tiles are not stuck.
-                if (lane == 0 && publish) st_relaxed_u64(st + tile, kFlagPrefix | (uint64_t)(excl + total));
-            }
-            if (lane == 0) {
-                s_excl = excl;
-                s_timeout = timeout ? 1 : 0;
-            }
-        }
-        __syncthreads();
-        const uint32_t tile_excl = s_excl;
-        if (s_timeout) {
-            if (tid == 0) set_status(status, SZ_ERR_DEVICE_TIMEOUT);
-            continue;
-        }
-
-        // ---- escape records, in element order
-        const uint64_t pos_off = kHeader + r.n + (r.n + 1) / 2;
-        uint8_t *pos_base = out + pos_off;
-        uint8_t *raw_base = pos_base + 4 * e_total;
-        const bool pos_aligned = (pos_off & 3) == 0;
-        uint32_t chunk_base = 0;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-            uint32_t m = esc[c] ? esc_in_element_order(esc[c]) : 0u;
-            uint64_t idx = (uint64_t)tile_excl + chunk_base + field16(thr_excl, c);
-            chunk_base += field16(tile_tot, c);
-            while (m) {  // ascending element order
-                const int j = __ffs(m) - 1;
-                m &= m - 1;
-                const uint64_t p = r.elem0 + (uint64_t)(c * kThreads + tid) * kChunk + j;
-                if (idx >= e_total) {  // more escapes than the histogram said
-                    set_status(status, SZ_ERR_CORRUPT);
-                    break;
-                }
-                store_u32_le(pos_base + 4 * idx, (uint32_t)p, pos_aligned);
-                raw_base[idx] = (uint8_t)exponent_of_chunk_elem(in[2 * c], in[2 * c + 1], j);
-                ++idx;
-            }
-        }
-
-        // The segment's last tile knows the final escape count.
-        if (tid == 0 && r.local + 1 == segment_tiles(r.n, a.batch.page_elems)) {
-            if ((uint64_t)tile_excl + total == e_total) {
-                a.out_bytes[k] = container_size(r.n, e_total);
-            } else {
-                set_status(status, SZ_ERR_CORRUPT);
-            }
-        }
+    if (tid >= kThreads) {
+        if (tid == kThreads) encode_producer<kBatched>(a, sh);
+    } else {
+        encode_consumers<kBatched>(a, sh);
     }
 }
 
-cudaError_t launch_encode(const EncodeArgs &a, bool batched, int grid, cudaStream_t s) {
-    if (a.batch.n_tiles == 0 && !batched && a.batch.single.n_elems != 0) return cudaSuccess;
-    grid = (int)umax64(1, umin64((uint64_t)grid, umax64(a.batch.n_tiles, 1)));
-    if (batched)
-        encode_kernel<true><<<grid, kThreads, 0, s>>>(a);
-    else
-        encode_kernel<false><<<grid, kThreads, 0, s>>>(a);
+cudaError_t launch_encode(const EncodeArgs &a0, bool batched, int grid, cudaStream_t s) {
+    EncodeArgs a = a0;
+    const size_t smem = sizeof(EncShared);
+    const uint64_t tiles = a.batch.n_tiles;
+    grid = (int)umax64(1, umin64((uint64_t)grid, umax64(tiles, 1)));
+    a.tiles_per_cta = umax64(1, div_up(tiles, (uint64_t)grid));
+    if (tiles > 0) grid = (int)div_up(tiles, a.tiles_per_cta);
+    cudaError_t e;
+    if (batched) {
+        e = cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        encode_kernel<true><<<grid, kPipeThreads, smem, s>>>(a);
+    } else {
+        e = cudaFuncSetAttribute(encode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        encode_kernel<false><<<grid, kPipeThreads, smem, s>>>(a);
+    }
     return cudaGetLastError();
 }
 
 int encode_blocks_per_sm() {
+    const size_t smem = sizeof(EncShared);
+    cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, encode_kernel<true>, kThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, encode_kernel<true>, kPipeThreads, smem);
     return occ > 0 ? occ : 1;
 }
 

@@ -1,6 +1,6 @@
 // sz_internal.cuh -- shared device-side definitions of the SplitZip B200
 // kernels: tile geometry, the tile -> (segment, page, offset) mapping, the
-// per-segment metadata record and small PTX helpers.
+// per-segment record, TMA / mbarrier helpers and small PTX helpers.
 //
 // Method: "SplitZip: Ultra Fast Lossless KV Compression for Disaggregated LLM
 // Serving" (gist.science explainer), sections 1-4; container layout as
@@ -15,15 +15,20 @@
 namespace sz {
 
 // ---------------------------------------------------------------- geometry
-// A tile is the unit of work of one CTA iteration: 256 threads x 4 chunks x
-// 16 elements.  A thread's chunk c covers tile elements
-// [(c*256 + tid)*16, +16), so one warp-wide 16-byte access is 512
-// contiguous bytes of input (two per chunk) or of sm output (one per chunk).
-constexpr int kThreads = 256;
+// Sub-tile: one pass of the 256 consumer threads, 4 chunks x 16 elements
+// each.  Chunk c of thread t covers sub-tile elements [(c*256 + t)*16, +16),
+// so a warp-wide 16-byte access is 512 contiguous bytes.
+// Tile: 4 sub-tiles (65,536 elements) inside one page; the unit of work
+// scheduling and of the per-tile exponent histograms that give every tile
+// its first escape index before the encode runs.
+constexpr int kThreads = 256;                 // consumer threads
 constexpr int kWarps = kThreads / 32;
+constexpr int kPipeThreads = kThreads + 32;   // + one producer warp
 constexpr int kChunk = 16;
 constexpr int kChunks = 4;
-constexpr uint32_t kTile = kThreads * kChunk * kChunks;  // 16384 elements
+constexpr uint32_t kSub = kThreads * kChunk * kChunks;  // 16,384 elements
+constexpr uint32_t kSubsPerTile = 4;
+constexpr uint32_t kTile = kSub * kSubsPerTile;         // 65,536 elements
 constexpr uint64_t kHeader = 48;
 constexpr uint32_t kMaxSmemSegs = 1024;  // segment starts cached in shared memory
 
@@ -31,17 +36,12 @@ constexpr uint32_t kMaxSmemSegs = 1024;  // segment starts cached in shared memo
 struct SegMeta {
     uint8_t codebook[16];
     uint64_t n_escapes;  // e = n - sum of the codebook's counts
-    uint32_t valid;      // 1 when the 16 entries are distinct
+    uint32_t valid;      // 1 when the 16 entries are distinct and the counts fit n
     uint32_t pad;
 };
 static_assert(sizeof(SegMeta) == 32, "SegMeta layout");
 
-// Lookback tile-status word: flag in bits 63..62, count in bits 31..0.
-constexpr uint64_t kFlagAggregate = 1ull << 62;
-constexpr uint64_t kFlagPrefix = 2ull << 62;
-constexpr uint64_t kFlagMask = 3ull << 62;
-
-constexpr uint32_t kDebugNoPublish = 1u;
+constexpr uint32_t kDebugNoSignal = 1u;  // producer never signals its stages
 
 __host__ __device__ inline uint64_t container_size(uint64_t n, uint64_t e) {
     return kHeader + n + (n + 1) / 2 + 5 * e;
@@ -53,9 +53,7 @@ __host__ __device__ inline uint32_t umin32(uint32_t a, uint32_t b) { return a < 
 
 // Tiles of a segment of n elements in pages of page_elems: every page is cut
 // into tiles of kTile elements (its last tile may be short).
-__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems) {
-    return div_up(page_elems, kTile);
-}
+__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems) { return div_up(page_elems, kTile); }
 __host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems) {
     if (n == 0) return 0;
     const uint64_t full = n / page_elems, rem = n % page_elems;
@@ -69,18 +67,21 @@ struct Batch {
     const sz_segment *segs;  // nullptr for a single tensor
     uint32_t n_segs;
     uint64_t page_elems;
+    uint32_t tiles_per_page;  // ceil(page_elems / kTile), precomputed on the host
     uint64_t n_tiles;
-    sz_segment single;       // the implicit segment of a single-tensor call
+    sz_segment single;        // the implicit segment of a single-tensor call
 };
 
 struct TileRef {
     uint32_t seg;
-    uint64_t local;    // tile index within the segment
+    uint32_t local;    // tile index within the segment
     uint64_t n;        // elements of the segment
-    uint64_t page;     // page index within the segment
+    uint32_t page;     // page index within the segment
     uint64_t elem0;    // first element of the tile in the segment's stream
-    uint64_t in_page;  // offset of the tile within its page (elements)
+    uint32_t in_page;  // offset of the tile within its page (elements)
     uint32_t len;      // elements in the tile
+    uint32_t n_subs;   // sub-tiles in the tile
+    uint32_t tiles;    // tiles of the segment
 };
 
 // Segment-start cache: tile_begin of every segment in shared memory when
@@ -89,10 +90,12 @@ struct SegCache {
     uint64_t tile_begin[kMaxSmemSegs + 1];
 };
 
+// Must be reached by every thread of the block.
 __device__ inline void seg_cache_fill(SegCache &c, const Batch &b) {
-    if (b.segs == nullptr || b.n_segs > kMaxSmemSegs) return;
-    for (uint32_t i = threadIdx.x; i < b.n_segs; i += blockDim.x) c.tile_begin[i] = b.segs[i].tile_begin;
-    if (threadIdx.x == 0) c.tile_begin[b.n_segs] = b.n_tiles;
+    if (b.segs != nullptr && b.n_segs <= kMaxSmemSegs) {
+        for (uint32_t i = threadIdx.x; i < b.n_segs; i += blockDim.x) c.tile_begin[i] = b.segs[i].tile_begin;
+        if (threadIdx.x == 0) c.tile_begin[b.n_segs] = b.n_tiles;
+    }
     __syncthreads();
 }
 
@@ -130,23 +133,24 @@ __device__ inline sz_segment load_segment(const Batch &b, uint32_t k) {
     return s;
 }
 
+// Geometry of global tile `tile` of segment k.  Tile and page counts fit in
+// 32 bits (n < 2^32), so the divisions here are 32-bit.
 __device__ inline TileRef resolve_tile(const Batch &b, const sz_segment &s, uint32_t k, uint64_t tile) {
     TileRef r;
     r.seg = k;
-    r.local = tile - s.tile_begin;
+    r.local = (uint32_t)(tile - s.tile_begin);
     r.n = s.n_elems;
-    const uint64_t tpp = tiles_per_page(b.page_elems);
+    const uint32_t tpp = b.tiles_per_page;
     r.page = r.local / tpp;
-    r.in_page = (r.local % tpp) * kTile;
-    r.elem0 = r.page * b.page_elems + r.in_page;
-    const uint64_t page_len = umin64(b.page_elems, r.n - r.page * b.page_elems);
+    r.in_page = (r.local - r.page * tpp) * kTile;
+    r.elem0 = (uint64_t)r.page * b.page_elems + r.in_page;
+    const uint64_t page_len = umin64(b.page_elems, r.n - (uint64_t)r.page * b.page_elems);
     r.len = (uint32_t)umin64(kTile, page_len - r.in_page);
+    r.n_subs = (r.len + kSub - 1) / kSub;
+    const uint64_t full = r.n / b.page_elems;
+    const uint64_t rem = r.n - full * b.page_elems;
+    r.tiles = (uint32_t)(full * tpp + (rem + kTile - 1) / kTile);
     return r;
-}
-
-// Tile (within its segment) that holds element p.
-__device__ inline uint64_t tile_of_element(uint64_t p, uint64_t page_elems) {
-    return (p / page_elems) * tiles_per_page(page_elems) + (p % page_elems) / kTile;
 }
 
 // ------------------------------------------------------------ status words
@@ -161,19 +165,14 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
-    uint64_t v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
 }
 
 // Streaming loads/stores: each byte is touched once by the kernel.
@@ -192,30 +191,78 @@ __device__ __forceinline__ uint32_t load_u32_any(const uint8_t *p) {
     if ((reinterpret_cast<uintptr_t>(p) & 3) == 0) return *reinterpret_cast<const uint32_t *>(p);
     return (uint32_t)p[0] | ((uint32_t)p[1] << 8) | ((uint32_t)p[2] << 16) | ((uint32_t)p[3] << 24);
 }
-__device__ __forceinline__ uint64_t load_u64_le(const uint8_t *p) {
-    uint64_t v = 0;
-    for (int b = 7; b >= 0; --b) v = (v << 8) | p[b];
-    return v;
+
+// Consumer-only barrier (named barrier 1): the 256 consumer threads, never
+// the producer warp.
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+
+// ------------------------------------------------- mbarrier + 1-D TMA copy
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for phase `parity` of `bar` to complete, for at most limit_ns of
+// device time.  Returns false when the wait ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+// One bulk copy global -> shared (16-byte aligned addresses, size a
+// multiple of 16), completing `bytes` of transaction count on `bar`.
+__device__ __forceinline__ void tma_load_1d(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ------------------------------------------------------- launch arguments
 struct HistArgs {
     Batch batch;
-    const uint16_t *const *pages;  // batched: page pointers; single: &base in `base`
+    const uint16_t *const *pages;  // batched: page pointers
     const uint16_t *base;          // single-tensor input
-    uint32_t *hist;                // [n_segs][256]
+    uint32_t *seg_hist;            // [n_segs][256]
+    uint32_t *tile_hist;           // [n_tiles][256]
     uint64_t tiles_per_cta;
     int32_t *status;               // [n_segs] or nullptr
 };
 
 struct SelectArgs {
-    uint32_t n_segs;
-    const sz_segment *segs;  // nullptr: single segment of `single_n` elements
-    uint64_t single_n;
-    const uint32_t *hist;    // [n_segs][256]
-    SegMeta *meta;           // [n_segs]
-    uint8_t *codebooks_out;  // optional [n_segs][16]
-    uint32_t *hist_out;      // optional [256] (single only)
+    Batch batch;
+    const uint32_t *seg_hist;    // [n_segs][256]
+    const uint32_t *tile_hist;   // [n_tiles][256]
+    SegMeta *meta;               // [n_segs]
+    uint32_t *tile_off;          // [n_tiles] first escape index of each tile
+    const uint8_t *codebook_in;  // single-tensor encode with a caller codebook, else nullptr
+    uint8_t *codebooks_out;      // optional [n_segs][16]
+    uint32_t *hist_out;          // optional [256] (single only)
 };
 
 struct EncodeArgs {
@@ -224,11 +271,11 @@ struct EncodeArgs {
     const uint16_t *base;
     uint8_t *out;
     uint64_t out_cap;
-    uint64_t *out_bytes;    // [n_segs]
-    int32_t *status;        // [n_segs] or nullptr
-    const SegMeta *meta;    // [n_segs]
-    uint64_t *tile_status;  // [n_tiles]
-    unsigned long long *ticket;
+    uint64_t *out_bytes;      // [n_segs]
+    int32_t *status;          // [n_segs]
+    const SegMeta *meta;      // [n_segs]
+    const uint32_t *tile_off; // [n_tiles]
+    uint64_t tiles_per_cta;
     uint64_t wait_limit_ns;
     uint32_t debug_flags;
 };
@@ -240,7 +287,10 @@ struct DecodeArgs {
     const uint8_t *in;
     uint64_t in_cap;         // bytes available from d_in (single: in_bytes)
     int32_t *status;         // [n_segs]
-    uint32_t *tile_start;    // per segment: tiles+1 escape start indices
+    uint32_t *sub_start;     // per segment: 4*tiles+1 escape start indices
+    uint64_t tiles_per_cta;
+    uint64_t wait_limit_ns;
+    uint32_t debug_flags;
 };
 
 }  // namespace sz

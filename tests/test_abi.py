@@ -21,7 +21,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert sz.sz_version().startswith("splitzip-b200")
-    assert sz.sz_tile_elems() == 16384
+    assert sz.sz_tile_elems() == 65536
 
 
 def test_library_is_built_for_sm100a():
@@ -29,12 +29,13 @@ def test_library_is_built_for_sm100a():
     assert "sm_100a" in sz.sz_version()
 
 
-@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 16385, 1 << 25, (1 << 32) - 2])
+@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 65536, 65537, 1 << 25, (1 << 32) - 2])
 def test_plan_worst_case_bound(n):
     cap, ws = sz.sz_plan(n)
     assert cap == 48 + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
-    tiles = -(-n // 16384)
-    assert ws >= 1280 + 8 * tiles + 4 * (tiles + 1)
+    tiles = -(-n // 65536)
+    # segment histogram + record, tile histograms, tile offsets, sub-tile starts
+    assert ws >= 1024 + 32 + 1024 * tiles + 4 * tiles + 4 * (4 * tiles + 1)
     assert ws % 256 == 0
 
 
@@ -61,10 +62,12 @@ def test_plan_batched_layout():
 
 
 def test_plan_batched_tiles_inside_pages():
-    # page of 40000 elements: tiles of 16384, 16384, 7232 per page
-    segs, pages, tiles, out, ws = sz.sz_plan_batched([100000], 40000)
+    # pages of 150016 elements: tiles of 65536, 65536, 18944 per page
+    segs, pages, tiles, out, ws = sz.sz_plan_batched([400000], 150016)
     assert pages == 3
-    assert tiles == 3 + 3 + 2  # 2 full pages x 3 tiles, last page of 20000: 2 tiles
+    assert tiles == 3 + 3 + 2  # 2 full pages x 3 tiles, last page of 99968: 2 tiles
+    segs, pages, tiles, out, ws = sz.sz_plan_batched([100000], 40000)
+    assert pages == 3 and tiles == 3  # pages shorter than a tile: one tile each
 
 
 def test_plan_batched_page_alignment():
@@ -86,17 +89,19 @@ def test_encode_argument_errors():
     L = sz.lib()
     cap, ws = sz.sz_plan(1000)
     # null output
-    assert L.sz_encode(A, 1000, A, None, cap, A, None, A, ws, None) == sz.SZ_ERR_NULL
+    assert L.sz_encode(A, 1000, A, None, cap, A, A, A, ws, None) == sz.SZ_ERR_NULL
+    # status word required
+    assert L.sz_encode(A, 1000, A, A, cap, A, None, A, ws, None) == sz.SZ_ERR_NULL
     # misaligned output
-    assert L.sz_encode(A, 1000, A, A + 4, cap, A, None, A, ws, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_encode(A, 1000, A, A + 4, cap, A, A, A, ws, None) == sz.SZ_ERR_ALIGN
     # misaligned input
-    assert L.sz_encode(A + 2, 1000, A, A, cap, A, None, A, ws, None) == sz.SZ_ERR_ALIGN
+    assert L.sz_encode(A + 2, 1000, A, A, cap, A, A, A, ws, None) == sz.SZ_ERR_ALIGN
     # capacity below 48 + n + ceil(n/2)
-    assert L.sz_encode(A, 1000, A, A, 48 + 1000 + 499, A, None, A, ws, None) == sz.SZ_ERR_CAPACITY
+    assert L.sz_encode(A, 1000, A, A, 48 + 1000 + 499, A, A, A, ws, None) == sz.SZ_ERR_CAPACITY
     # workspace too small
-    assert L.sz_encode(A, 1000, A, A, cap, A, None, A, ws - 1, None) == sz.SZ_ERR_WORKSPACE
+    assert L.sz_encode(A, 1000, A, A, cap, A, A, A, ws - 1, None) == sz.SZ_ERR_WORKSPACE
     # too large
-    assert L.sz_encode(A, 1 << 32, A, A, cap, A, None, A, ws, None) == sz.SZ_ERR_TOO_LARGE
+    assert L.sz_encode(A, 1 << 32, A, A, cap, A, A, A, ws, None) == sz.SZ_ERR_TOO_LARGE
 
 
 def test_histogram_and_decode_argument_errors():

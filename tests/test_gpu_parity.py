@@ -70,7 +70,8 @@ def assert_parity(x):
 
 # -------------------------------------------------------------- small cases
 RAGGED = [0, 1, 2, 3, 7, 8, 15, 16, 17, 31, 33, 100, 255, 4095, 4096, 4097, 8191, 16383, 16384, 16385,
-          16400, 32768, 3 * 16384 + 5, 65536, 65537, 100003, 262147]
+          16400, 32768, 3 * 16384 + 5, 65535, 65536, 65537, 65536 + 16384 + 8, 100003, 3 * 65536 + 100,
+          262147]
 
 
 @pytest.mark.parametrize("n", RAGGED)
@@ -383,9 +384,10 @@ def test_paged_full_workload4_adversarial():
         assert host[off: off + int(sizes[r])].tobytes() == oracle.encode(b.request_stream(r))
 
 
-def test_pages_larger_than_tiles_with_partial_last_page():
-    # pages of 40000 elements: tiles 16384 + 16384 + 7232 per page
-    page = 40000 - 40000 % 64  # 39936
+@pytest.mark.parametrize("page", [39936, 150016])
+def test_pages_with_partial_last_page(page):
+    # 39936: pages shorter than a tile (ragged sub-tiles); 150016: three
+    # tiles per page (65536 + 65536 + 18944)
     lens = [page * 2 + 1000, 17, page, 5 * page + 64]
     streams = [kvgen.mixed_small(n, seed=600 + i) for i, n in enumerate(lens)]
     plan = sz.BatchPlan(lens, page, device=DEV)
