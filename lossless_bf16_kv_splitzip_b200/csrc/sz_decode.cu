@@ -273,7 +273,9 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
             }
             const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
             const uint32_t len = umin32(kSub, r.len - sub * kSub);
-            uint32_t lo = ts[sub], hi = ts[sub + 1];
+            // the last sub-tile of a tile ends where the next tile starts (the
+            // segment's last: at e), so the ranges cover every escape record
+            uint32_t lo = ts[sub], hi = ts[sub + 1 == r.n_subs ? kSubsPerTile : sub + 1];
             if (hi < lo || hi > h.e || hi - lo > len) {  // sub-tile starts not monotone
                 if (lane == 0) set_status(a.status + k, SZ_ERR_CORRUPT);
                 hi = lo = 0;
