@@ -219,6 +219,26 @@ struct __align__(128) DecShared {
     int go;
 };
 
+constexpr int kEscPerLane = 8;  // escape records a producer lane loads at once
+
+// Records lo+b0+u*32+lane (u < kEscPerLane, index < cnt) into registers;
+// all loads are issued before any is used.  Past cnt: zeros.
+__device__ __forceinline__ void load_escape_batch(const uint8_t *pos, const uint8_t *raw, uint32_t lo, uint32_t b0,
+                                                  uint32_t cnt, int lane, bool pos_aligned,
+                                                  uint32_t (&pv)[kEscPerLane], uint32_t (&xv)[kEscPerLane]) {
+#pragma unroll
+    for (int u = 0; u < kEscPerLane; ++u) {
+        const uint32_t i = b0 + (uint32_t)u * 32 + lane;
+        pv[u] = 0;
+        xv[u] = 0;
+        if (i < cnt) {
+            const uint64_t g = (uint64_t)lo + i;
+            pv[u] = pos_aligned ? *reinterpret_cast<const uint32_t *>(pos + 4 * g) : load_u32_any(pos + 4 * g);
+            xv[u] = raw[g];
+        }
+    }
+}
+
 // ------------------------------------------------------------ producer
 template <bool kBatched>
 __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
@@ -258,11 +278,35 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
         uint16_t *dst = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
         const bool dst_aligned = (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
         if (!dst_aligned && lane == 0) set_status(a.status + k, SZ_ERR_ALIGN);
+        // the tile's five sub-tile starts in one round trip; the last sub-tile
+        // of a tile ends where the next tile starts (the segment's last: at
+        // e), so the ranges cover every escape record
         const uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k + 4 * (uint64_t)r.local;
+        uint32_t tsv[kSubsPerTile + 1];
+#pragma unroll
+        for (uint32_t q = 0; q <= kSubsPerTile; ++q) tsv[q] = ts[q];
         const uint8_t *pos = c + kHeader + h.n + (h.n + 1) / 2;
         const uint8_t *raw = pos + 4 * h.e;
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
             const int s = (int)(j % kDecStages);
+            const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
+            const uint32_t len = umin32(kSub, r.len - sub * kSub);
+            uint32_t lo = tsv[0], hi = tsv[kSubsPerTile];
+#pragma unroll
+            for (uint32_t q = 0; q < kSubsPerTile; ++q) {
+                if (q == sub) {
+                    lo = tsv[q];
+                    if (sub + 1 < r.n_subs) hi = tsv[q + 1];
+                }
+            }
+            bool bad_range = hi < lo || hi > h.e || hi - lo > len;  // starts not monotone
+            if (bad_range) hi = lo = 0;
+            const uint32_t cnt = hi - lo;
+            const bool staged = cnt <= kEscCap;
+            // first batch of escape records into registers before waiting for
+            // the stage, so their latency overlaps the consumers' work
+            uint32_t pv[kEscPerLane], xv[kEscPerLane];
+            if (staged) load_escape_batch(pos, raw, lo, 0, cnt, lane, pos_aligned, pv, xv);
             bool ok = true;
             if (j >= (uint32_t)kDecStages && lane == 0)
                 ok = mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns);
@@ -271,33 +315,32 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                 if (lane == 0) set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
                 return;
             }
-            const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
-            const uint32_t len = umin32(kSub, r.len - sub * kSub);
-            // the last sub-tile of a tile ends where the next tile starts (the
-            // segment's last: at e), so the ranges cover every escape record
-            uint32_t lo = ts[sub], hi = ts[sub + 1 == r.n_subs ? kSubsPerTile : sub + 1];
-            if (hi < lo || hi > h.e || hi - lo > len) {  // sub-tile starts not monotone
-                if (lane == 0) set_status(a.status + k, SZ_ERR_CORRUPT);
-                hi = lo = 0;
-            }
-            const uint32_t cnt = hi - lo;
-            const bool staged = cnt <= kEscCap;
+            if (bad_range && lane == 0) set_status(a.status + k, SZ_ERR_CORRUPT);
             if (staged) {
-                uint16_t *cf = sh.chunk_first[s];
-                for (uint32_t i = lane; i < (uint32_t)(kThreads * kChunks); i += 32) cf[i] = kNoEsc;
+                uint4 *cf4 = reinterpret_cast<uint4 *>(sh.chunk_first[s]);
+                const uint4 none = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                for (uint32_t i = lane; i < (uint32_t)(kThreads * kChunks) / 8; i += 32) cf4[i] = none;
                 __syncwarp();
-                for (uint32_t i = lane; i < cnt; i += 32) {
-                    const uint64_t p = pos_aligned ? *reinterpret_cast<const uint32_t *>(pos + 4 * (uint64_t)(lo + i))
-                                                   : load_u32_any(pos + 4 * (uint64_t)(lo + i));
-                    const uint32_t x = raw[lo + i];
-                    const uint64_t pp = i == 0 ? 0 : load_u32_any(pos + 4 * (uint64_t)(lo + i - 1));
-                    bool bad = p < elem0 || p - elem0 >= len || in_set8(cbset, x) || (i > 0 && pp >= p);
-                    if (bad) set_status(a.status + k, SZ_ERR_CORRUPT);
-                    const uint32_t local = bad ? kNoEsc : (uint32_t)(p - elem0);
-                    sh.esc_pos[s][i] = (uint16_t)local;
-                    sh.esc_raw[s][i] = (uint8_t)x;
-                    const bool first = i == 0 || pp < elem0 || ((uint32_t)(pp - elem0) >> 4) != (local >> 4);
-                    if (!bad && first) cf[local >> 4] = (uint16_t)i;
+                uint16_t *cf = sh.chunk_first[s];
+                uint32_t carry = 0;  // position of the record before this batch
+                for (uint32_t b0 = 0; b0 < cnt; b0 += 32 * kEscPerLane) {
+                    if (b0 > 0) load_escape_batch(pos, raw, lo, b0, cnt, lane, pos_aligned, pv, xv);
+#pragma unroll
+                    for (int u = 0; u < kEscPerLane; ++u) {
+                        const uint32_t i = b0 + (uint32_t)u * 32 + lane;
+                        const uint32_t p = pv[u], x = xv[u];
+                        uint32_t pp = __shfl_up_sync(0xFFFFFFFFu, p, 1);
+                        if (lane == 0) pp = carry;
+                        carry = __shfl_sync(0xFFFFFFFFu, p, 31);
+                        if (i >= cnt) continue;
+                        const bool bad = p < elem0 || p - elem0 >= len || in_set8(cbset, x) || (i > 0 && pp >= p);
+                        if (bad) set_status(a.status + k, SZ_ERR_CORRUPT);
+                        const uint32_t local = bad ? kNoEsc : (uint32_t)(p - elem0);
+                        sh.esc_pos[s][i] = (uint16_t)local;
+                        sh.esc_raw[s][i] = (uint8_t)x;
+                        const bool first = i == 0 || pp < elem0 || ((uint32_t)(pp - elem0) >> 4) != (local >> 4);
+                        if (!bad && first) cf[local >> 4] = (uint16_t)i;
+                    }
                 }
                 __syncwarp();
             }
