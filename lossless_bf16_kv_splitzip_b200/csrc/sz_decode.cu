@@ -179,22 +179,14 @@ __device__ __forceinline__ void patch_elem(uint4 &o0, uint4 &o1, int j, uint32_t
 #undef SZ_PATCH
 }
 
-// 256-bit codebook membership, 8 words, selected without local memory.
-__device__ __forceinline__ bool in_set8(const uint32_t s[8], uint32_t x) {
-    const uint32_t w = x >> 5;
-    uint32_t v = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v = (w == (uint32_t)i) ? s[i] : v;
-    return (v >> (x & 31)) & 1u;
-}
-
 constexpr int kDecStages = 3;
 constexpr uint32_t kEscCap = 1024;  // escapes staged per sub-tile; more: consumers stream them
 constexpr uint16_t kNoEsc = 0xFFFFu;
 
 constexpr uint32_t kDFlagEnd = 1u;
 constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
-constexpr uint32_t kDFlagStaged = 4u;   // escapes are in the stage (else consumers stream them)
+constexpr uint32_t kDFlagStaged = 4u;   // cnt <= kEscCap: escapes are checked and mapped in the stage
+constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage
 
 struct DecMeta {
     uint16_t *dst;      // global destination of the sub-tile's first element
@@ -202,15 +194,19 @@ struct DecMeta {
     uint64_t elem0;     // first element of the sub-tile in the segment stream
     uint64_t n, e;
     uint64_t cb_lo, cb_hi;
-    uint32_t seg, len, flags, lo, cnt, pad;
+    uint32_t seg, len, flags, lo, cnt;
+    uint32_t pos_skew;  // byte offset of record lo's position inside the staged copy
+    uint32_t raw_skew;  // byte offset of record lo's exponent inside the staged copy
+    uint32_t pad;
 };
 
 struct __align__(128) DecShared {
     uint8_t sm[kDecStages][kSub];
     uint8_t codes[kDecStages][kSub / 2];
-    uint16_t esc_pos[kDecStages][kEscCap];  // sub-tile-local offsets
+    uint8_t pos[kDecStages][4 * kEscCap + 32];  // 16-byte aligned superset of the positions
+    uint8_t raw[kDecStages][kEscCap + 32];      // 16-byte aligned superset of the exponents
+    uint16_t esc_pos[kDecStages][kEscCap];      // checked sub-tile-local offsets
     uint16_t chunk_first[kDecStages][kThreads * kChunks];
-    uint8_t esc_raw[kDecStages][kEscCap];
     DecMeta meta[kDecStages];
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
@@ -219,30 +215,12 @@ struct __align__(128) DecShared {
     int go;
 };
 
-constexpr int kEscPerLane = 8;  // escape records a producer lane loads at once
-
-// Records lo+b0+u*32+lane (u < kEscPerLane, index < cnt) into registers;
-// all loads are issued before any is used.  Past cnt: zeros.
-__device__ __forceinline__ void load_escape_batch(const uint8_t *pos, const uint8_t *raw, uint32_t lo, uint32_t b0,
-                                                  uint32_t cnt, int lane, bool pos_aligned,
-                                                  uint32_t (&pv)[kEscPerLane], uint32_t (&xv)[kEscPerLane]) {
-#pragma unroll
-    for (int u = 0; u < kEscPerLane; ++u) {
-        const uint32_t i = b0 + (uint32_t)u * 32 + lane;
-        pv[u] = 0;
-        xv[u] = 0;
-        if (i < cnt) {
-            const uint64_t g = (uint64_t)lo + i;
-            pv[u] = pos_aligned ? *reinterpret_cast<const uint32_t *>(pos + 4 * g) : load_u32_any(pos + 4 * g);
-            xv[u] = raw[g];
-        }
-    }
-}
-
 // ------------------------------------------------------------ producer
+// One thread: per sub-tile, wait for the stage to be free, then bulk-copy
+// the sm bytes, the codes and (when they fit and stay inside the buffer) a
+// 16-byte aligned superset of the sub-tile's escape positions and exponents.
 template <bool kBatched>
 __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
-    const int lane = threadIdx.x & 31;
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
     const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
     const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
@@ -250,45 +228,40 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     uint32_t cur = 0xFFFFFFFFu;
     sz_segment seg{};
     Header h{};
-    uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const uint8_t *c = nullptr;
-    bool tma_ok = false, pos_aligned = false;
+    uint64_t cap = 0;
+    bool tma_ok = false;
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
             cur = k;
             seg = load_segment(a.batch, k);
-            const uint64_t cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
+            cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
             c = a.in + seg.out_offset;
             h = read_header(c, cap, seg.n_elems);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) cbset[i] = 0;
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const uint32_t x = cb_entry(h.cb_lo, h.cb_hi, q);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) cbset[i] |= ((x >> 5) == (uint32_t)i) ? (1u << (x & 31)) : 0u;
-            }
-            tma_ok = (seg.n_elems % 16) == 0;  // code stream 16-byte aligned (container is)
-            pos_aligned = ((kHeader + h.n + (h.n + 1) / 2) & 3) == 0;
-            if (!h.ok && lane == 0) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
+            tma_ok = (seg.n_elems % 16) == 0;  // code and position streams 16-byte aligned
+            if (!h.ok) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
         }
         if (!h.ok) continue;
         const TileRef r = resolve_tile(a.batch, seg, k, t);
         uint16_t *dst = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
         const bool dst_aligned = (reinterpret_cast<uintptr_t>(dst) & 15) == 0;
-        if (!dst_aligned && lane == 0) set_status(a.status + k, SZ_ERR_ALIGN);
-        // the tile's five sub-tile starts in one round trip; the last sub-tile
-        // of a tile ends where the next tile starts (the segment's last: at
-        // e), so the ranges cover every escape record
+        if (!dst_aligned) set_status(a.status + k, SZ_ERR_ALIGN);
+        // the tile's five sub-tile starts; the last sub-tile of a tile ends
+        // where the next tile starts (the segment's last: at e), so the
+        // ranges cover every escape record
         const uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k + 4 * (uint64_t)r.local;
         uint32_t tsv[kSubsPerTile + 1];
 #pragma unroll
         for (uint32_t q = 0; q <= kSubsPerTile; ++q) tsv[q] = ts[q];
-        const uint8_t *pos = c + kHeader + h.n + (h.n + 1) / 2;
-        const uint8_t *raw = pos + 4 * h.e;
+        const uint64_t pos_off = kHeader + h.n + (h.n + 1) / 2;
+        const uint64_t raw_off = pos_off + 4 * h.e;
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
             const int s = (int)(j % kDecStages);
+            if (j >= (uint32_t)kDecStages && !mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns)) {
+                set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
+                return;
+            }
             const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
             const uint32_t len = umin32(kSub, r.len - sub * kSub);
             uint32_t lo = tsv[0], hi = tsv[kSubsPerTile];
@@ -299,85 +272,63 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                     if (sub + 1 < r.n_subs) hi = tsv[q + 1];
                 }
             }
-            bool bad_range = hi < lo || hi > h.e || hi - lo > len;  // starts not monotone
-            if (bad_range) hi = lo = 0;
+            if (hi < lo || hi > h.e || hi - lo > len) {  // sub-tile starts not monotone
+                set_status(a.status + k, SZ_ERR_CORRUPT);
+                hi = lo = 0;
+            }
             const uint32_t cnt = hi - lo;
             const bool staged = cnt <= kEscCap;
-            // first batch of escape records into registers before waiting for
-            // the stage, so their latency overlaps the consumers' work
-            uint32_t pv[kEscPerLane], xv[kEscPerLane];
-            if (staged) load_escape_batch(pos, raw, lo, 0, cnt, lane, pos_aligned, pv, xv);
-            bool ok = true;
-            if (j >= (uint32_t)kDecStages && lane == 0)
-                ok = mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns);
-            ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-            if (!ok) {
-                if (lane == 0) set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
-                return;
-            }
-            if (bad_range && lane == 0) set_status(a.status + k, SZ_ERR_CORRUPT);
-            if (staged) {
-                uint4 *cf4 = reinterpret_cast<uint4 *>(sh.chunk_first[s]);
-                const uint4 none = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
-                for (uint32_t i = lane; i < (uint32_t)(kThreads * kChunks) / 8; i += 32) cf4[i] = none;
-                __syncwarp();
-                uint16_t *cf = sh.chunk_first[s];
-                uint32_t carry = 0;  // position of the record before this batch
-                for (uint32_t b0 = 0; b0 < cnt; b0 += 32 * kEscPerLane) {
-                    if (b0 > 0) load_escape_batch(pos, raw, lo, b0, cnt, lane, pos_aligned, pv, xv);
-#pragma unroll
-                    for (int u = 0; u < kEscPerLane; ++u) {
-                        const uint32_t i = b0 + (uint32_t)u * 32 + lane;
-                        const uint32_t p = pv[u], x = xv[u];
-                        uint32_t pp = __shfl_up_sync(0xFFFFFFFFu, p, 1);
-                        if (lane == 0) pp = carry;
-                        carry = __shfl_sync(0xFFFFFFFFu, p, 31);
-                        if (i >= cnt) continue;
-                        const bool bad = p < elem0 || p - elem0 >= len || in_set8(cbset, x) || (i > 0 && pp >= p);
-                        if (bad) set_status(a.status + k, SZ_ERR_CORRUPT);
-                        const uint32_t local = bad ? kNoEsc : (uint32_t)(p - elem0);
-                        sh.esc_pos[s][i] = (uint16_t)local;
-                        sh.esc_raw[s][i] = (uint8_t)x;
-                        const bool first = i == 0 || pp < elem0 || ((uint32_t)(pp - elem0) >> 4) != (local >> 4);
-                        if (!bad && first) cf[local >> 4] = (uint16_t)i;
-                    }
-                }
-                __syncwarp();
-            }
-            if (lane == 0) {
-                DecMeta &m = sh.meta[s];
-                m.dst = dst_aligned ? dst + sub * kSub : nullptr;
-                m.c = c;
-                m.elem0 = elem0;
-                m.n = h.n;
-                m.e = h.e;
-                m.cb_lo = h.cb_lo;
-                m.cb_hi = h.cb_hi;
-                m.seg = k;
-                m.len = len;
-                m.lo = lo;
-                m.cnt = cnt;
-                const bool tma = tma_ok && len == kSub;
-                m.flags = (tma ? kDFlagInSmem : 0u) | (staged ? kDFlagStaged : 0u);
-                if (tma) {
-                    mbar_arrive_expect_tx(&sh.full[s], kSub + kSub / 2);
-                    tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
-                    tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
-                } else {
-                    mbar_arrive(&sh.full[s]);
+            DecMeta &m = sh.meta[s];
+            m.dst = dst_aligned ? dst + sub * kSub : nullptr;
+            m.c = c;
+            m.elem0 = elem0;
+            m.n = h.n;
+            m.e = h.e;
+            m.cb_lo = h.cb_lo;
+            m.cb_hi = h.cb_hi;
+            m.seg = k;
+            m.len = len;
+            m.lo = lo;
+            m.cnt = cnt;
+            const bool tma = tma_ok && len == kSub;
+            uint32_t bytes = 0, f = staged ? kDFlagStaged : 0u;
+            // escape records: aligned supersets [ps & ~15, ceil16(pe)) that
+            // must lie inside the caller's buffer
+            uint64_t p0 = 0, p1 = 0, r0 = 0, r1 = 0;
+            if (tma && staged && cnt > 0) {
+                p0 = (pos_off + 4 * (uint64_t)lo) & ~15ull;
+                p1 = (pos_off + 4 * (uint64_t)hi + 15) & ~15ull;
+                r0 = (raw_off + lo) & ~15ull;
+                r1 = (raw_off + hi + 15) & ~15ull;
+                if (p1 <= cap && r1 <= cap) {
+                    f |= kDFlagEscSmem;
+                    m.pos_skew = (uint32_t)(pos_off + 4 * (uint64_t)lo - p0);
+                    m.raw_skew = (uint32_t)(raw_off + lo - r0);
+                    bytes += (uint32_t)(p1 - p0) + (uint32_t)(r1 - r0);
                 }
             }
-            __syncwarp();
+            if (tma) {
+                f |= kDFlagInSmem;
+                bytes += kSub + kSub / 2;
+            }
+            m.flags = f;
+            if (bytes) {
+                mbar_arrive_expect_tx(&sh.full[s], bytes);
+                tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
+                tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
+                if (f & kDFlagEscSmem) {
+                    tma_load_1d(sh.pos[s], c + p0, (uint32_t)(p1 - p0), &sh.full[s]);
+                    tma_load_1d(sh.raw[s], c + r0, (uint32_t)(r1 - r0), &sh.full[s]);
+                }
+            } else {
+                mbar_arrive(&sh.full[s]);
+            }
         }
     }
     const int s = (int)(j % kDecStages);
-    bool ok = true;
-    if (j >= (uint32_t)kDecStages && lane == 0)
-        ok = mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns);
-    if (lane == 0 && ok) {
-        sh.meta[s].flags = kDFlagEnd;
-        mbar_arrive(&sh.full[s]);
-    }
+    if (j >= (uint32_t)kDecStages && !mbar_wait(&sh.empty[s], ((j / kDecStages) - 1) & 1u, a.wait_limit_ns)) return;
+    sh.meta[s].flags = kDFlagEnd;
+    mbar_arrive(&sh.full[s]);
 }
 
 // ------------------------------------------------------------ consumers
@@ -411,13 +362,46 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
                 sh.inset[tid] = w;
             }
             cur = m.seg;
-            consumer_sync();
         }
         int32_t *status = a.status + m.seg;
         const bool in_smem = (m.flags & kDFlagInSmem) != 0;
         const bool codes_aligned = (m.n % 8) == 0;
         const uint8_t *in_sm = m.c + kHeader + m.elem0;
         const uint8_t *codes_base = m.c + kHeader + m.n;
+        const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
+        const uint8_t *graw = gpos + 4 * m.e;
+        uint16_t *ep = sh.esc_pos[s];
+        uint16_t *cf = sh.chunk_first[s];
+
+        // ---- escapes of the sub-tile: check them and map chunk -> first escape
+        if (m.flags & kDFlagStaged) {
+            reinterpret_cast<uint2 *>(cf)[tid] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+            consumer_sync();  // chunk map cleared (and the codebook bitmap written)
+            const bool es = (m.flags & kDFlagEscSmem) != 0;
+            const uint8_t *spos = sh.pos[s] + m.pos_skew;
+            const uint8_t *sraw = sh.raw[s] + m.raw_skew;
+            for (uint32_t i = tid; i < m.cnt; i += kThreads) {
+                const uint64_t g = (uint64_t)m.lo + i;
+                const uint64_t p = es ? *reinterpret_cast<const uint32_t *>(spos + 4 * i) : load_u32_any(gpos + 4 * g);
+                const uint64_t pp = i == 0 ? 0 : (es ? *reinterpret_cast<const uint32_t *>(spos + 4 * (i - 1))
+                                                     : load_u32_any(gpos + 4 * (g - 1)));
+                const uint32_t x = es ? sraw[i] : graw[g];
+                const bool bad = p < m.elem0 || p - m.elem0 >= m.len || ((sh.inset[x >> 5] >> (x & 31)) & 1u) ||
+                                 (i > 0 && pp >= p);
+                if (bad) set_status(status, SZ_ERR_CORRUPT);
+                const uint32_t local = bad ? kNoEsc : (uint32_t)(p - m.elem0);
+                ep[i] = (uint16_t)local;
+                const bool first = i == 0 || pp < m.elem0 || ((uint32_t)(pp - m.elem0) >> 4) != (local >> 4);
+                if (!bad && first) cf[local >> 4] = (uint16_t)i;
+            }
+            if (!es) {
+                // exponents read from global memory: keep them next to the offsets
+                for (uint32_t i = tid; i < m.cnt; i += kThreads) sh.raw[s][i] = graw[(uint64_t)m.lo + i];
+            }
+            consumer_sync();
+        } else {
+            consumer_sync();  // codebook bitmap written
+        }
 
         // ---- decode all chunks into registers
         uint4 o[2 * kChunks];
@@ -453,11 +437,9 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
             decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
         }
 
-        // ---- escapes
+        // ---- patch the escapes in registers
         if (m.flags & kDFlagStaged) {
-            const uint16_t *cf = sh.chunk_first[s];
-            const uint16_t *ep = sh.esc_pos[s];
-            const uint8_t *er = sh.esc_raw[s];
+            const uint8_t *er = (m.flags & kDFlagEscSmem) ? sh.raw[s] + m.raw_skew : sh.raw[s];
 #pragma unroll
             for (int q = 0; q < kChunks; ++q) {
                 const uint32_t ci = q * kThreads + tid;
@@ -474,19 +456,16 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
         } else {
             // more escapes than one stage holds: stream them through the
             // stage's escape area in batches (every consumer takes part)
-            const uint8_t *pos = m.c + kHeader + m.n + (m.n + 1) / 2;
-            const uint8_t *raw = pos + 4 * m.e;
-            uint16_t *ep = sh.esc_pos[s];
-            uint8_t *er = sh.esc_raw[s];
+            uint8_t *er = sh.raw[s];
             for (uint32_t b0 = 0; b0 < m.cnt; b0 += kEscCap) {
                 const uint32_t nb = umin32(kEscCap, m.cnt - b0);
                 consumer_sync();
                 for (uint32_t i = tid; i < nb; i += kThreads) {
                     const uint64_t g = (uint64_t)m.lo + b0 + i;
-                    const uint64_t p = load_u32_any(pos + 4 * g);
-                    const uint32_t x = raw[g];
+                    const uint64_t p = load_u32_any(gpos + 4 * g);
+                    const uint32_t x = graw[g];
                     bool bad = p < m.elem0 || p - m.elem0 >= m.len;
-                    if (b0 + i > 0) bad |= load_u32_any(pos + 4 * (g - 1)) >= p;
+                    if (b0 + i > 0) bad |= load_u32_any(gpos + 4 * (g - 1)) >= p;
                     bad |= (sh.inset[x >> 5] >> (x & 31)) & 1u;
                     if (bad) set_status(status, SZ_ERR_CORRUPT);
                     ep[i] = bad ? kNoEsc : (uint16_t)(p - m.elem0);
@@ -546,10 +525,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2) decode_kernel(const DecodeArg
         fence_mbar_init();
     }
     seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
-    if (tid >= kThreads)
-        decode_producer<kBatched>(a, sh);
-    else
+    if (tid >= kThreads) {
+        if (tid == kThreads) decode_producer<kBatched>(a, sh);
+    } else {
         decode_consumers<kBatched>(a, sh);
+    }
 }
 
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {

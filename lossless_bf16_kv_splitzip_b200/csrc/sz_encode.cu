@@ -60,28 +60,30 @@ struct __align__(128) EncShared {
 __device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, const uint8_t *lut,
                                              uint4 &sm, uint64_t &codes, uint32_t &esc) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t smw[4], B[4];
+    const uint32_t lut_s = smem_u32(lut);
+    uint32_t smw[4], P[4];
+    esc = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint32_t a = w[2 * q], b = w[2 * q + 1];
-        const uint32_t hi = prmt(a, b, 0x7531u);  // high bytes of the 4 values
-        const uint32_t lo = prmt(a, b, 0x6420u);  // low bytes
+        const uint32_t hi = prmt(a, b, 0x7531u);  // high bytes of the 4 values: sign | exp >> 1
+        const uint32_t lo = prmt(a, b, 0x6420u);  // low bytes: exp & 1 | mantissa
         smw[q] = (hi & 0x80808080u) | (lo & 0x7F7F7F7Fu);
-        const uint32_t c0 = lut[(a >> 7) & 0xFFu];
-        const uint32_t c1 = lut[(a >> 23) & 0xFFu];
-        const uint32_t c2 = lut[(b >> 7) & 0xFFu];
-        const uint32_t c3 = lut[(b >> 23) & 0xFFu];
-        B[q] = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+        // the 4 exponents, one per byte: (hi << 1) supplies bits 7..1, lo's
+        // bit 7 supplies bit 0
+        const uint32_t e4 = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
+        uint32_t c[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t ek = prmt(e4, 0u, 0x4440u | (uint32_t)k);  // byte k, zero-extended
+            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(c[k]) : "r"(lut_s + ek));
+        }
+        const uint32_t B = prmt(prmt(c[0], c[1], 0x5140u), prmt(c[2], c[3], 0x5140u), 0x5410u);
+        esc |= (B & 0x80808080u) >> (7 - q);
+        // byte 0 = n0 | n1 << 4, byte 2 = n2 | n3 << 4 (the escape bits drop out)
+        P[q] = (B & 0x0F0F0F0Fu) | ((B >> 4) & 0xF0F0F0F0u);
     }
     sm = make_uint4(smw[0], smw[1], smw[2], smw[3]);
-    esc = ((B[0] & 0x80808080u) >> 7) | ((B[1] & 0x80808080u) >> 6) | ((B[2] & 0x80808080u) >> 5) |
-          ((B[3] & 0x80808080u) >> 4);
-    uint32_t P[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t nib = B[q] & 0x0F0F0F0Fu;
-        P[q] = nib | (nib >> 4);  // byte 0 = n0 | n1<<4, byte 2 = n2 | n3<<4
-    }
     const uint32_t lo32 = prmt(P[0], P[1], 0x6420u);
     const uint32_t hi32 = prmt(P[2], P[3], 0x6420u);
     codes = (uint64_t)lo32 | ((uint64_t)hi32 << 32);
