@@ -211,7 +211,6 @@ struct __align__(128) DecShared {
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
     SegCache segc;
-    uint32_t inset[8];
     int go;
 };
 
@@ -332,11 +331,90 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
 }
 
 // ------------------------------------------------------------ consumers
+// 256-bit codebook membership in 8 registers, selected without local memory.
+__device__ __forceinline__ bool in_set8(const uint32_t (&set)[8], uint32_t x) {
+    const uint32_t w = x >> 5;
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v = (w == (uint32_t)i) ? set[i] : v;
+    return (v >> (x & 31)) & 1u;
+}
+
+// One chunk: 16 sm bytes + 8 code bytes -> 16 BF16 values, escapes patched,
+// stored.  Escape records come from the stage's chunk map.
+template <bool kStaged>
+__device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &sh, int s, const DecTables &T, int q,
+                                                   int tid, int32_t *status) {
+    const uint32_t ci = q * kThreads + tid;
+    const uint32_t off = ci * kChunk;
+    if (off >= m.len) return;
+    const uint32_t cnt = umin32(kChunk, m.len - off);
+    const bool codes_aligned = (m.n % 8) == 0;
+    uint4 smv = make_uint4(0, 0, 0, 0);
+    uint64_t codes = 0;
+    if (m.flags & kDFlagInSmem) {
+        smv = *reinterpret_cast<const uint4 *>(sh.sm[s] + off);
+        codes = *reinterpret_cast<const unsigned long long *>(sh.codes[s] + off / 2);
+    } else {
+        const uint8_t *in_sm = m.c + kHeader + m.elem0;
+        const uint8_t *codes_base = m.c + kHeader + m.n;
+        if (cnt == (uint32_t)kChunk && codes_aligned) {
+            smv = ld_stream_v4(in_sm + off);
+            codes = *reinterpret_cast<const unsigned long long *>(codes_base + (m.elem0 + off) / 2);
+        } else {
+            uint32_t sw[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int jj = 0; jj < kChunk; ++jj)
+                if (jj < (int)cnt) sw[jj >> 2] |= (uint32_t)in_sm[off + jj] << (8 * (jj & 3));
+            smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+            const uint8_t *cb = codes_base + (m.elem0 + off) / 2;
+#pragma unroll
+            for (int b = 0; b < kChunk / 2; ++b)
+                if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
+            // odd element count: the unused high nibble must be 0
+            if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+            if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
+        }
+    }
+    uint4 o0, o1;
+    decode_chunk(smv, codes, T, o0, o1);
+    if (kStaged) {
+        uint32_t i = sh.chunk_first[s][ci];
+        if (i != kNoEsc) {
+            const uint16_t *ep = sh.esc_pos[s];
+            const uint8_t *er = (m.flags & kDFlagEscSmem) ? sh.raw[s] + m.raw_skew : sh.raw[s];
+            for (; i < m.cnt; ++i) {
+                const uint32_t l = ep[i];
+                if ((l >> 4) != ci) break;  // next chunk (or a rejected entry)
+                const int jj = (int)(l & 15u);
+                if (((codes >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+                patch_elem(o0, o1, jj, er[i]);
+            }
+        }
+    }
+    if (m.dst == nullptr) return;
+    if (cnt == (uint32_t)kChunk) {
+        st_stream_v4(m.dst + off, o0);
+        st_stream_v4(m.dst + off + 8, o1);
+    } else {
+        const uint32_t w[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+        for (int jj = 0; jj < kChunk; ++jj)
+            if (jj < (int)cnt) m.dst[off + jj] = (uint16_t)(w[jj >> 1] >> (16 * (jj & 1)));
+    }
+}
+
 template <bool kBatched>
 __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
     const int tid = threadIdx.x, lane = tid & 31;
     uint32_t cur = 0xFFFFFFFFu;
     DecTables T{};
+    uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    // every stage's chunk map starts empty; a thread clears its own entries
+    // again each time it releases a stage
+#pragma unroll
+    for (int st = 0; st < kDecStages; ++st)
+        reinterpret_cast<uint2 *>(sh.chunk_first[st])[tid] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kDecStages);
         if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
@@ -352,31 +430,24 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
         if (m.flags & kDFlagEnd) return;
         if (m.seg != cur) {
             T = make_tables(m.cb_lo, m.cb_hi);
-            if (tid < 8) {
-                uint32_t w = 0;
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const uint32_t x = cb_entry(m.cb_lo, m.cb_hi, q);
-                    if ((x >> 5) == (uint32_t)tid) w |= 1u << (x & 31);
-                }
-                sh.inset[tid] = w;
+            for (int i = 0; i < 8; ++i) cbset[i] = 0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                const uint32_t x = cb_entry(m.cb_lo, m.cb_hi, q);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cbset[i] |= ((x >> 5) == (uint32_t)i) ? (1u << (x & 31)) : 0u;
             }
             cur = m.seg;
         }
         int32_t *status = a.status + m.seg;
-        const bool in_smem = (m.flags & kDFlagInSmem) != 0;
-        const bool codes_aligned = (m.n % 8) == 0;
-        const uint8_t *in_sm = m.c + kHeader + m.elem0;
-        const uint8_t *codes_base = m.c + kHeader + m.n;
         const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
         const uint8_t *graw = gpos + 4 * m.e;
         uint16_t *ep = sh.esc_pos[s];
         uint16_t *cf = sh.chunk_first[s];
 
-        // ---- escapes of the sub-tile: check them and map chunk -> first escape
         if (m.flags & kDFlagStaged) {
-            reinterpret_cast<uint2 *>(cf)[tid] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-            consumer_sync();  // chunk map cleared (and the codebook bitmap written)
+            // ---- check the sub-tile's escapes and map chunk -> first escape
             const bool es = (m.flags & kDFlagEscSmem) != 0;
             const uint8_t *spos = sh.pos[s] + m.pos_skew;
             const uint8_t *sraw = sh.raw[s] + m.raw_skew;
@@ -386,76 +457,51 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
                 const uint64_t pp = i == 0 ? 0 : (es ? *reinterpret_cast<const uint32_t *>(spos + 4 * (i - 1))
                                                      : load_u32_any(gpos + 4 * (g - 1)));
                 const uint32_t x = es ? sraw[i] : graw[g];
-                const bool bad = p < m.elem0 || p - m.elem0 >= m.len || ((sh.inset[x >> 5] >> (x & 31)) & 1u) ||
-                                 (i > 0 && pp >= p);
+                const bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x) || (i > 0 && pp >= p);
                 if (bad) set_status(status, SZ_ERR_CORRUPT);
                 const uint32_t local = bad ? kNoEsc : (uint32_t)(p - m.elem0);
                 ep[i] = (uint16_t)local;
+                if (!es) sh.raw[s][i] = (uint8_t)x;  // exponents read from global: keep them staged
                 const bool first = i == 0 || pp < m.elem0 || ((uint32_t)(pp - m.elem0) >> 4) != (local >> 4);
                 if (!bad && first) cf[local >> 4] = (uint16_t)i;
             }
-            if (!es) {
-                // exponents read from global memory: keep them next to the offsets
-                for (uint32_t i = tid; i < m.cnt; i += kThreads) sh.raw[s][i] = graw[(uint64_t)m.lo + i];
-            }
             consumer_sync();
+#pragma unroll
+            for (int q = 0; q < kChunks; ++q) decode_store_chunk<true>(m, sh, s, T, q, tid, status);
+#pragma unroll
+            for (int q = 0; q < kChunks; ++q) cf[q * kThreads + tid] = kNoEsc;  // this thread's own entries
         } else {
-            consumer_sync();  // codebook bitmap written
-        }
-
-        // ---- decode all chunks into registers
-        uint4 o[2 * kChunks];
-        uint64_t cw[kChunks];
-#pragma unroll
-        for (int q = 0; q < kChunks; ++q) {
-            const uint32_t ci = q * kThreads + tid;
-            const uint32_t off = ci * kChunk;
-            const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
-            uint4 smv = make_uint4(0, 0, 0, 0);
-            uint64_t codes = 0;
-            if (in_smem) {
-                smv = *reinterpret_cast<const uint4 *>(sh.sm[s] + off);
-                codes = *reinterpret_cast<const unsigned long long *>(sh.codes[s] + off / 2);
-            } else if (cnt == (uint32_t)kChunk && codes_aligned) {
-                smv = ld_stream_v4(in_sm + off);
-                codes = *reinterpret_cast<const unsigned long long *>(codes_base + (m.elem0 + off) / 2);
-            } else if (cnt) {
-                uint32_t sw[4] = {0, 0, 0, 0};
-#pragma unroll
-                for (int jj = 0; jj < kChunk; ++jj)
-                    if (jj < (int)cnt) sw[jj >> 2] |= (uint32_t)in_sm[off + jj] << (8 * (jj & 3));
-                smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-                const uint8_t *cb = codes_base + (m.elem0 + off) / 2;
-#pragma unroll
-                for (int b = 0; b < kChunk / 2; ++b)
-                    if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
-                // odd element count: the unused high nibble must be 0
-                if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
-            }
-            cw[q] = codes;
-            decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
-        }
-
-        // ---- patch the escapes in registers
-        if (m.flags & kDFlagStaged) {
-            const uint8_t *er = (m.flags & kDFlagEscSmem) ? sh.raw[s] + m.raw_skew : sh.raw[s];
+            // more escapes than one stage holds: decode all chunks into
+            // registers, then stream the escapes through the stage's escape
+            // area in batches (every consumer takes part)
+            uint4 o[2 * kChunks];
+            uint64_t cw[kChunks];
 #pragma unroll
             for (int q = 0; q < kChunks; ++q) {
-                const uint32_t ci = q * kThreads + tid;
-                uint32_t i = cf[ci];
-                if (i == kNoEsc) continue;
-                for (; i < m.cnt; ++i) {
-                    const uint32_t l = ep[i];
-                    if ((l >> 4) != ci) break;  // next chunk (or a rejected entry)
-                    const int jj = (int)(l & 15u);
-                    if (((cw[q] >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                    patch_elem(o[2 * q], o[2 * q + 1], jj, er[i]);
+                const uint32_t off = (q * kThreads + tid) * kChunk;
+                const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
+                uint4 smv = make_uint4(0, 0, 0, 0);
+                uint64_t codes = 0;
+                if (m.flags & kDFlagInSmem) {
+                    smv = *reinterpret_cast<const uint4 *>(sh.sm[s] + off);
+                    codes = *reinterpret_cast<const unsigned long long *>(sh.codes[s] + off / 2);
+                } else if (cnt) {
+                    const uint8_t *in_sm = m.c + kHeader + m.elem0;
+                    const uint8_t *cb = m.c + kHeader + m.n + (m.elem0 + off) / 2;
+                    uint32_t sw[4] = {0, 0, 0, 0};
+#pragma unroll
+                    for (int jj = 0; jj < kChunk; ++jj)
+                        if (jj < (int)cnt) sw[jj >> 2] |= (uint32_t)in_sm[off + jj] << (8 * (jj & 3));
+                    smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+#pragma unroll
+                    for (int b = 0; b < kChunk / 2; ++b)
+                        if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
+                    if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
+                    if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
                 }
+                cw[q] = codes;
+                decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
             }
-        } else {
-            // more escapes than one stage holds: stream them through the
-            // stage's escape area in batches (every consumer takes part)
             uint8_t *er = sh.raw[s];
             for (uint32_t b0 = 0; b0 < m.cnt; b0 += kEscCap) {
                 const uint32_t nb = umin32(kEscCap, m.cnt - b0);
@@ -464,9 +510,8 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
                     const uint64_t g = (uint64_t)m.lo + b0 + i;
                     const uint64_t p = load_u32_any(gpos + 4 * g);
                     const uint32_t x = graw[g];
-                    bool bad = p < m.elem0 || p - m.elem0 >= m.len;
+                    bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x);
                     if (b0 + i > 0) bad |= load_u32_any(gpos + 4 * (g - 1)) >= p;
-                    bad |= (sh.inset[x >> 5] >> (x & 31)) & 1u;
                     if (bad) set_status(status, SZ_ERR_CORRUPT);
                     ep[i] = bad ? kNoEsc : (uint16_t)(p - m.elem0);
                     er[i] = (uint8_t)x;
@@ -487,23 +532,21 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
                     }
                 }
             }
-        }
-
-        // ---- store
-        if (m.dst != nullptr) {
+            if (m.dst != nullptr) {
 #pragma unroll
-            for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
-                if (cnt == (uint32_t)kChunk) {
-                    st_stream_v4(m.dst + off, o[2 * q]);
-                    st_stream_v4(m.dst + off + 8, o[2 * q + 1]);
-                } else if (cnt) {
-                    const uint32_t w[8] = {o[2 * q].x, o[2 * q].y, o[2 * q].z, o[2 * q].w,
-                                           o[2 * q + 1].x, o[2 * q + 1].y, o[2 * q + 1].z, o[2 * q + 1].w};
+                for (int q = 0; q < kChunks; ++q) {
+                    const uint32_t off = (q * kThreads + tid) * kChunk;
+                    const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
+                    if (cnt == (uint32_t)kChunk) {
+                        st_stream_v4(m.dst + off, o[2 * q]);
+                        st_stream_v4(m.dst + off + 8, o[2 * q + 1]);
+                    } else if (cnt) {
+                        const uint32_t w[8] = {o[2 * q].x, o[2 * q].y, o[2 * q].z, o[2 * q].w,
+                                               o[2 * q + 1].x, o[2 * q + 1].y, o[2 * q + 1].z, o[2 * q + 1].w};
 #pragma unroll
-                    for (int jj = 0; jj < kChunk; ++jj)
-                        if (jj < (int)cnt) m.dst[off + jj] = (uint16_t)(w[jj >> 1] >> (16 * (jj & 1)));
+                        for (int jj = 0; jj < kChunk; ++jj)
+                            if (jj < (int)cnt) m.dst[off + jj] = (uint16_t)(w[jj >> 1] >> (16 * (jj & 1)));
+                    }
                 }
             }
         }

@@ -47,20 +47,22 @@ struct __align__(128) EncShared {
     uint64_t full[kEncStages];
     uint64_t empty[kEncStages];
     SegCache segc;
-    uint64_t warp_tot[kWarps];
-    uint8_t lut[256];
-    int go;
+    uint64_t warp_tot[2][kWarps];  // double-buffered by sub-tile parity
+    int go[2];                     // stage j's data arrived (slot j & 1)
 };
+
+// exponent -> code (0..15) or 0x80 (escape); static so that lookups address
+// it as [index + constant]
+__shared__ __align__(16) uint8_t s_lut[256];
 
 // ---------------------------------------------------------- chunk encode
 // 16 consecutive BF16 values (two uint4) -> 16 sm bytes, 8 code bytes and an
 // escape mask.  The LUT maps exponent -> code (0..15) or 0x80 (escape; its
 // low nibble 0 is the placeholder code).  Escape mask layout: element j of
 // the chunk is bit 8*(j%4) + j/4.
-__device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, const uint8_t *lut,
-                                             uint4 &sm, uint64_t &codes, uint32_t &esc) {
+__device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, uint4 &sm, uint64_t &codes,
+                                             uint32_t &esc) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    const uint32_t lut_s = smem_u32(lut);
     uint32_t smw[4], P[4];
     esc = 0;
 #pragma unroll
@@ -74,12 +76,9 @@ __device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, con
         const uint32_t e4 = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
         uint32_t c[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t ek = prmt(e4, 0u, 0x4440u | (uint32_t)k);  // byte k, zero-extended
-            asm volatile("ld.shared.u8 %0, [%1];" : "=r"(c[k]) : "r"(lut_s + ek));
-        }
+        for (int k = 0; k < 4; ++k) c[k] = s_lut[prmt(e4, 0u, 0x4440u | (uint32_t)k)];  // byte k, zero-extended
         const uint32_t B = prmt(prmt(c[0], c[1], 0x5140u), prmt(c[2], c[3], 0x5140u), 0x5410u);
-        esc |= (B & 0x80808080u) >> (7 - q);
+        esc |= (B >> (7 - q)) & (0x01010101u << q);
         // byte 0 = n0 | n1 << 4, byte 2 = n2 | n3 << 4 (the escape bits drop out)
         P[q] = (B & 0x0F0F0F0Fu) | ((B >> 4) & 0xF0F0F0F0u);
     }
@@ -221,6 +220,44 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
 }
 
 // ------------------------------------------------------------ consumers
+// Escape counts of the thread's 4 chunks -> (exclusive prefix within the
+// warp, warp total), both packed as four 16-bit fields.  When no chunk holds
+// more than one escape -- the usual case -- ballots do it; otherwise a
+// shuffle scan of the packed counts.
+__device__ __forceinline__ void warp_escape_scan(const uint32_t (&esc)[kChunks], int lane, uint64_t &excl,
+                                                 uint64_t &total) {
+    uint32_t cnt[kChunks];
+    uint32_t any_multi = 0;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+        cnt[c] = __popc(esc[c]);
+        any_multi |= cnt[c] > 1u;
+    }
+    excl = 0;
+    total = 0;
+    if (!__any_sync(0xFFFFFFFFu, any_multi)) {
+        const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            const uint32_t b = __ballot_sync(0xFFFFFFFFu, cnt[c] != 0);
+            excl |= (uint64_t)__popc(b & below) << (16 * c);
+            total |= (uint64_t)__popc(b) << (16 * c);
+        }
+        return;
+    }
+    uint64_t v = 0;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) v |= (uint64_t)cnt[c] << (16 * c);
+    uint64_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    excl = incl - v;
+    total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+}
+
 template <bool kBatched>
 __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -229,11 +266,14 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     uint64_t n = 0, e_total = 0;
     bool codes_aligned = false, pos_aligned = false;
     uint32_t running = 0;  // escapes of the current tile so far
+
+    // The wait for stage j+1 is folded into sub-tile j's scan barrier: one
+    // consumer barrier per sub-tile.
+    if (tid == 0) sh.go[0] = mbar_wait(&sh.full[0], 0u, a.wait_limit_ns) ? 1 : 0;
+    consumer_sync();
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kEncStages);
-        if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kEncStages) & 1u, a.wait_limit_ns) ? 1 : 0;
-        consumer_sync();
-        if (!sh.go) {  // the same decision in every consumer thread
+        if (!sh.go[j & 1]) {  // the same decision in every consumer thread
             if (tid == 0 && a.batch.n_tiles > 0) {
                 const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.tiles_per_cta, a.batch.n_tiles - 1);
                 set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
@@ -242,11 +282,11 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         }
         const EncMeta m = sh.meta[s];
         if (m.flags & kFlagEnd) return;
-        if (m.seg != cur) {  // every consumer finished the previous sub-tile (barrier above)
-            sh.lut[tid] = 0x80;
+        if (m.seg != cur) {  // every consumer is past the previous sub-tile's compute
+            s_lut[tid] = 0x80;
             consumer_sync();
             const SegMeta &g = a.meta[m.seg];
-            if (tid < 16) sh.lut[g.codebook[tid]] = (uint8_t)tid;
+            if (tid < 16) s_lut[g.codebook[tid]] = (uint8_t)tid;
             const sz_segment seg = load_segment(a.batch, m.seg);
             out = a.out + seg.out_offset;
             n = seg.n_elems;
@@ -283,7 +323,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             uint64_t cw;
             if (in_smem && codes_aligned) {
                 read_chunk_smem(stage, c, tid, v0, v1);
-                encode_chunk(v0, v1, sh.lut, smv, cw, esc[c]);
+                encode_chunk(v0, v1, smv, cw, esc[c]);
                 st_stream_v4(out_sm + off, smv);
                 st_stream_u64(codes_base + (m.elem0 + off) / 2, cw);
                 continue;
@@ -293,7 +333,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             const uint32_t cnt = umin32(kChunk, m.len - off);
             read_chunk_global(m.src + off, cnt, v0, v1);
             uint32_t e;
-            encode_chunk(v0, v1, sh.lut, smv, cw, e);
+            encode_chunk(v0, v1, smv, cw, e);
             uint32_t keep = 0;
 #pragma unroll
             for (int q = 0; q < kChunk; ++q)
@@ -314,54 +354,52 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             }
         }
 
-        // ---- escapes: CTA scan of the per-chunk counts, packed 4 x 16 bit
-        uint64_t cnt = 0;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) cnt |= (uint64_t)__popc(esc[c]) << (16 * c);
-        uint64_t incl = cnt;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += y;
-        }
-        if (lane == 31) sh.warp_tot[wid] = incl;
+        // ---- escapes: position of every escape in the sub-tile's order
+        uint64_t wexcl, wtot;
+        warp_escape_scan(esc, lane, wexcl, wtot);
+        uint64_t *wt = sh.warp_tot[j & 1];
+        if (lane == 0) wt[wid] = wtot;
+        const int s_next = (int)((j + 1) % kEncStages);
+        if (tid == 0) sh.go[(j + 1) & 1] = mbar_wait(&sh.full[s_next], ((j + 1) / kEncStages) & 1u, a.wait_limit_ns) ? 1 : 0;
         consumer_sync();
         uint64_t warp_excl = 0, tot = 0;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const uint64_t v = sh.warp_tot[w];
+            const uint64_t v = wt[w];
             if (w < wid) warp_excl += v;
             tot += v;
         }
-        const uint64_t thr_excl = warp_excl + incl - cnt;
+        const uint64_t thr_excl = warp_excl + wexcl;
         const uint32_t sub_total = field16(tot, 0) + field16(tot, 1) + field16(tot, 2) + field16(tot, 3);
 
         // ---- escape records, in element order
-        const uint64_t pos_off = kHeader + n + (n + 1) / 2;
-        uint8_t *pos_base = out + pos_off;
-        uint8_t *raw_base = pos_base + 4 * e_total;
-        uint32_t chunk_base = running;
+        if (sub_total) {
+            const uint64_t pos_off = kHeader + n + (n + 1) / 2;
+            uint8_t *pos_base = out + pos_off;
+            uint8_t *raw_base = pos_base + 4 * e_total;
+            uint32_t chunk_base = running;
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-            uint32_t msk = esc[c] ? esc_in_element_order(esc[c]) : 0u;
-            uint32_t idx = chunk_base + field16(thr_excl, c);
-            chunk_base += field16(tot, c);
-            if (!msk) continue;
-            const uint32_t off = (c * kThreads + tid) * kChunk;
-            uint4 v0, v1;
-            if (in_smem) read_chunk_smem(stage, c, tid, v0, v1);
-            else read_chunk_global(m.src + off, umin32(kChunk, m.len - off), v0, v1);
-            while (msk) {  // ascending element order
-                const int q = __ffs(msk) - 1;
-                msk &= msk - 1;
-                const uint64_t g = (uint64_t)m.esc_base + idx;
-                if (idx >= m.esc_count || g >= e_total) {  // more escapes than the histograms said
-                    set_status(status, SZ_ERR_CORRUPT);
-                    break;
+            for (int c = 0; c < kChunks; ++c) {
+                uint32_t msk = esc[c] ? esc_in_element_order(esc[c]) : 0u;
+                uint32_t idx = chunk_base + field16(thr_excl, c);
+                chunk_base += field16(tot, c);
+                if (!msk) continue;
+                const uint32_t off = (c * kThreads + tid) * kChunk;
+                uint4 v0, v1;
+                if (in_smem) read_chunk_smem(stage, c, tid, v0, v1);
+                else read_chunk_global(m.src + off, umin32(kChunk, m.len - off), v0, v1);
+                while (msk) {  // ascending element order
+                    const int q = __ffs(msk) - 1;
+                    msk &= msk - 1;
+                    const uint64_t g = (uint64_t)m.esc_base + idx;
+                    if (idx >= m.esc_count || g >= e_total) {  // more escapes than the histograms said
+                        set_status(status, SZ_ERR_CORRUPT);
+                        break;
+                    }
+                    store_u32_le(pos_base + 4 * g, (uint32_t)(m.elem0 + off + q), pos_aligned);
+                    raw_base[g] = (uint8_t)exponent_of_chunk_elem(v0, v1, q);
+                    ++idx;
                 }
-                store_u32_le(pos_base + 4 * g, (uint32_t)(m.elem0 + off + q), pos_aligned);
-                raw_base[g] = (uint8_t)exponent_of_chunk_elem(v0, v1, q);
-                ++idx;
             }
         }
         running += sub_total;
