@@ -23,6 +23,7 @@
 namespace sz {
 
 constexpr int kEncStages = 3;
+constexpr uint32_t kEscStage = 1024;  // staged escape records per sub-tile; more: written directly
 
 constexpr uint32_t kFlagEnd = 1u;        // no more sub-tiles
 constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
@@ -49,6 +50,10 @@ struct __align__(128) EncShared {
     SegCache segc;
     uint64_t warp_tot[2][kWarps];  // double-buffered by sub-tile parity
     int go[2];                     // stage j's data arrived (slot j & 1)
+    // escape records of a sub-tile, (raw exponent << 16 | offset in the
+    // sub-tile), written in element order and copied out coalesced one
+    // sub-tile later; double-buffered by sub-tile parity
+    uint32_t esc[2][kEscStage];
 };
 
 // exponent -> code (0..15) or 0x80 (escape); static so that lookups address
@@ -86,14 +91,6 @@ __device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, uin
     const uint32_t lo32 = prmt(P[0], P[1], 0x6420u);
     const uint32_t hi32 = prmt(P[2], P[3], 0x6420u);
     codes = (uint64_t)lo32 | ((uint64_t)hi32 << 32);
-}
-
-// Exponent of chunk element j (runtime j; selects, no local-memory array).
-__device__ __forceinline__ uint32_t exponent_of_chunk_elem(const uint4 v0, const uint4 v1, int j) {
-    const int q = j >> 1;
-    const uint4 v = (q & 4) ? v1 : v0;
-    const uint32_t word = (q & 2) ? ((q & 1) ? v.w : v.z) : ((q & 1) ? v.y : v.x);
-    return (j & 1) ? (word >> 23) & 0xFFu : (word >> 7) & 0xFFu;
 }
 
 __device__ __forceinline__ uint32_t byte_of(uint4 v, int b) {  // b is a compile-time constant
@@ -220,6 +217,33 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
 }
 
 // ------------------------------------------------------------ consumers
+// A sub-tile's staged escape records waiting to be copied out.
+struct PendingEsc {
+    uint32_t cnt;           // records staged (0: none)
+    uint64_t first;         // segment index of the first record
+    uint64_t lim;           // records may not reach this index
+    uint64_t elem0;         // first element of the sub-tile
+    uint8_t *pos_base;
+    uint8_t *raw_base;
+    bool pos_aligned;
+    int32_t *status;
+};
+
+// Every consumer thread takes records tid, tid + 256, ...: consecutive
+// threads write consecutive positions and exponents.
+__device__ __forceinline__ void copy_out_escapes(const uint32_t *stg, const PendingEsc &p, int tid) {
+    for (uint32_t i = tid; i < p.cnt; i += kThreads) {
+        const uint64_t g = p.first + i;
+        if (g >= p.lim) {  // more escapes than the histograms said
+            set_status(p.status, SZ_ERR_CORRUPT);
+            break;
+        }
+        const uint32_t rec = stg[i];
+        store_u32_le(p.pos_base + 4 * g, (uint32_t)(p.elem0 + (rec & 0xFFFFu)), p.pos_aligned);
+        p.raw_base[g] = (uint8_t)(rec >> 16);
+    }
+}
+
 // Escape counts of the thread's 4 chunks -> (exclusive prefix within the
 // warp, warp total), both packed as four 16-bit fields.  When no chunk holds
 // more than one escape -- the usual case -- ballots do it; otherwise a
@@ -266,6 +290,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     uint64_t n = 0, e_total = 0;
     bool codes_aligned = false, pos_aligned = false;
     uint32_t running = 0;  // escapes of the current tile so far
+    PendingEsc pend{};
 
     // The wait for stage j+1 is folded into sub-tile j's scan barrier: one
     // consumer barrier per sub-tile.
@@ -281,7 +306,11 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             return;
         }
         const EncMeta m = sh.meta[s];
-        if (m.flags & kFlagEnd) return;
+        if (m.flags & kFlagEnd) {
+            consumer_sync();  // the last sub-tile's staged records are complete
+            copy_out_escapes(sh.esc[(j + 1) & 1], pend, tid);
+            return;
+        }
         if (m.seg != cur) {  // every consumer is past the previous sub-tile's compute
             s_lut[tid] = 0x80;
             consumer_sync();
@@ -372,34 +401,57 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const uint64_t thr_excl = warp_excl + wexcl;
         const uint32_t sub_total = field16(tot, 0) + field16(tot, 1) + field16(tot, 2) + field16(tot, 3);
 
-        // ---- escape records, in element order
+        // ---- the previous sub-tile's staged records, coalesced
+        copy_out_escapes(sh.esc[(j + 1) & 1], pend, tid);
+        pend.cnt = 0;
+
+        // ---- this sub-tile's records, in element order
         if (sub_total) {
             const uint64_t pos_off = kHeader + n + (n + 1) / 2;
             uint8_t *pos_base = out + pos_off;
             uint8_t *raw_base = pos_base + 4 * e_total;
-            uint32_t chunk_base = running;
+            // the records this sub-tile may write: [first, last) of the segment
+            const uint64_t first = (uint64_t)m.esc_base + running;
+            const uint64_t lim = umin64(e_total, (uint64_t)m.esc_base + m.esc_count);
+            const bool staged = sub_total <= kEscStage;
+            uint32_t *stg = sh.esc[j & 1];
+            uint32_t chunk_base = 0;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
                 uint32_t msk = esc[c] ? esc_in_element_order(esc[c]) : 0u;
-                uint32_t idx = chunk_base + field16(thr_excl, c);
+                uint32_t idx = chunk_base + field16(thr_excl, c);  // index within the sub-tile
                 chunk_base += field16(tot, c);
                 if (!msk) continue;
                 const uint32_t off = (c * kThreads + tid) * kChunk;
-                uint4 v0, v1;
-                if (in_smem) read_chunk_smem(stage, c, tid, v0, v1);
-                else read_chunk_global(m.src + off, umin32(kChunk, m.len - off), v0, v1);
                 while (msk) {  // ascending element order
                     const int q = __ffs(msk) - 1;
                     msk &= msk - 1;
-                    const uint64_t g = (uint64_t)m.esc_base + idx;
-                    if (idx >= m.esc_count || g >= e_total) {  // more escapes than the histograms said
-                        set_status(status, SZ_ERR_CORRUPT);
-                        break;
+                    const uint32_t x = in_smem ? (uint32_t)reinterpret_cast<const uint16_t *>(stage)[off + q]
+                                               : (uint32_t)m.src[off + q];
+                    const uint32_t raw = (x >> 7) & 0xFFu;
+                    if (staged) {
+                        stg[idx] = (raw << 16) | (off + q);
+                    } else {
+                        const uint64_t g = first + idx;
+                        if (g >= lim) {  // more escapes than the histograms said
+                            set_status(status, SZ_ERR_CORRUPT);
+                            break;
+                        }
+                        store_u32_le(pos_base + 4 * g, (uint32_t)(m.elem0 + off + q), pos_aligned);
+                        raw_base[g] = (uint8_t)raw;
                     }
-                    store_u32_le(pos_base + 4 * g, (uint32_t)(m.elem0 + off + q), pos_aligned);
-                    raw_base[g] = (uint8_t)exponent_of_chunk_elem(v0, v1, q);
                     ++idx;
                 }
+            }
+            if (staged) {
+                pend.cnt = sub_total;
+                pend.first = first;
+                pend.lim = lim;
+                pend.elem0 = m.elem0;
+                pend.pos_base = pos_base;
+                pend.raw_base = raw_base;
+                pend.pos_aligned = pos_aligned;
+                pend.status = status;
             }
         }
         running += sub_total;

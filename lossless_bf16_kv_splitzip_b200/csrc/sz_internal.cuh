@@ -30,7 +30,7 @@ constexpr uint32_t kSub = kThreads * kChunk * kChunks;  // 16,384 elements
 constexpr uint32_t kSubsPerTile = 4;
 constexpr uint32_t kTile = kSub * kSubsPerTile;         // 65,536 elements
 constexpr uint64_t kHeader = 48;
-constexpr uint32_t kMaxSmemSegs = 1024;  // segment starts cached in shared memory
+constexpr uint32_t kMaxSmemSegs = 256;  // segment starts cached in shared memory
 
 // Per-segment record kept in the workspace between kernels (32 bytes).
 struct SegMeta {
