@@ -180,12 +180,10 @@ __device__ __forceinline__ void patch_elem(uint4 &o0, uint4 &o1, int j, uint32_t
 }
 
 constexpr int kDecStages = 3;
-constexpr uint32_t kEscCap = 1024;  // escapes staged per sub-tile; more: consumers stream them
-constexpr uint16_t kNoEsc = 0xFFFFu;
+constexpr uint32_t kEscCap = 1024;  // escape records bulk-copied per sub-tile; more: read directly
 
 constexpr uint32_t kDFlagEnd = 1u;
 constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
-constexpr uint32_t kDFlagStaged = 4u;   // cnt <= kEscCap: escapes are checked and mapped in the stage
 constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage
 
 struct DecMeta {
@@ -205,8 +203,6 @@ struct __align__(128) DecShared {
     uint8_t codes[kDecStages][kSub / 2];
     uint8_t pos[kDecStages][4 * kEscCap + 32];  // 16-byte aligned superset of the positions
     uint8_t raw[kDecStages][kEscCap + 32];      // 16-byte aligned superset of the exponents
-    uint16_t esc_pos[kDecStages][kEscCap];      // checked sub-tile-local offsets
-    uint16_t chunk_first[kDecStages][kThreads * kChunks];
     DecMeta meta[kDecStages];
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
@@ -276,7 +272,6 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                 hi = lo = 0;
             }
             const uint32_t cnt = hi - lo;
-            const bool staged = cnt <= kEscCap;
             DecMeta &m = sh.meta[s];
             m.dst = dst_aligned ? dst + sub * kSub : nullptr;
             m.c = c;
@@ -290,11 +285,11 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
             m.lo = lo;
             m.cnt = cnt;
             const bool tma = tma_ok && len == kSub;
-            uint32_t bytes = 0, f = staged ? kDFlagStaged : 0u;
+            uint32_t bytes = 0, f = 0;
             // escape records: aligned supersets [ps & ~15, ceil16(pe)) that
             // must lie inside the caller's buffer
             uint64_t p0 = 0, p1 = 0, r0 = 0, r1 = 0;
-            if (tma && staged && cnt > 0) {
+            if (tma && cnt > 0 && cnt <= kEscCap) {
                 p0 = (pos_off + 4 * (uint64_t)lo) & ~15ull;
                 p1 = (pos_off + 4 * (uint64_t)hi + 15) & ~15ull;
                 r0 = (raw_off + lo) & ~15ull;
@@ -340,16 +335,13 @@ __device__ __forceinline__ bool in_set8(const uint32_t (&set)[8], uint32_t x) {
     return (v >> (x & 31)) & 1u;
 }
 
-// One chunk: 16 sm bytes + 8 code bytes -> 16 BF16 values, escapes patched,
-// stored.  Escape records come from the stage's chunk map.
-template <bool kStaged>
+// One chunk: 16 sm bytes + 8 code bytes -> 16 BF16 values, stored.  The
+// escaped places get codebook[0] here and are overwritten afterwards.
 __device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &sh, int s, const DecTables &T, int q,
                                                    int tid, int32_t *status) {
-    const uint32_t ci = q * kThreads + tid;
-    const uint32_t off = ci * kChunk;
+    const uint32_t off = (q * kThreads + tid) * kChunk;
     if (off >= m.len) return;
     const uint32_t cnt = umin32(kChunk, m.len - off);
-    const bool codes_aligned = (m.n % 8) == 0;
     uint4 smv = make_uint4(0, 0, 0, 0);
     uint64_t codes = 0;
     if (m.flags & kDFlagInSmem) {
@@ -358,7 +350,7 @@ __device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &
     } else {
         const uint8_t *in_sm = m.c + kHeader + m.elem0;
         const uint8_t *codes_base = m.c + kHeader + m.n;
-        if (cnt == (uint32_t)kChunk && codes_aligned) {
+        if (cnt == (uint32_t)kChunk && (m.n % 8) == 0) {
             smv = ld_stream_v4(in_sm + off);
             codes = *reinterpret_cast<const unsigned long long *>(codes_base + (m.elem0 + off) / 2);
         } else {
@@ -378,20 +370,6 @@ __device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &
     }
     uint4 o0, o1;
     decode_chunk(smv, codes, T, o0, o1);
-    if (kStaged) {
-        uint32_t i = sh.chunk_first[s][ci];
-        if (i != kNoEsc) {
-            const uint16_t *ep = sh.esc_pos[s];
-            const uint8_t *er = (m.flags & kDFlagEscSmem) ? sh.raw[s] + m.raw_skew : sh.raw[s];
-            for (; i < m.cnt; ++i) {
-                const uint32_t l = ep[i];
-                if ((l >> 4) != ci) break;  // next chunk (or a rejected entry)
-                const int jj = (int)(l & 15u);
-                if (((codes >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                patch_elem(o0, o1, jj, er[i]);
-            }
-        }
-    }
     if (m.dst == nullptr) return;
     if (cnt == (uint32_t)kChunk) {
         st_stream_v4(m.dst + off, o0);
@@ -410,11 +388,6 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
     uint32_t cur = 0xFFFFFFFFu;
     DecTables T{};
     uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    // every stage's chunk map starts empty; a thread clears its own entries
-    // again each time it releases a stage
-#pragma unroll
-    for (int st = 0; st < kDecStages; ++st)
-        reinterpret_cast<uint2 *>(sh.chunk_first[st])[tid] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kDecStages);
         if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
@@ -441,113 +414,43 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
             cur = m.seg;
         }
         int32_t *status = a.status + m.seg;
-        const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
-        const uint8_t *graw = gpos + 4 * m.e;
-        uint16_t *ep = sh.esc_pos[s];
-        uint16_t *cf = sh.chunk_first[s];
 
-        if (m.flags & kDFlagStaged) {
-            // ---- check the sub-tile's escapes and map chunk -> first escape
+        // ---- every chunk: codes -> exponents, joined with sign and mantissa
+#pragma unroll
+        for (int q = 0; q < kChunks; ++q) decode_store_chunk(m, sh, s, T, q, tid, status);
+
+        // ---- escapes, one per thread, after every chunk store of the
+        // sub-tile (the barrier orders the two writes of an escaped place):
+        // check the record and overwrite its value's exponent
+        if (m.cnt) {
+            consumer_sync();
             const bool es = (m.flags & kDFlagEscSmem) != 0;
+            const bool ss = (m.flags & kDFlagInSmem) != 0;
+            const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
+            const uint8_t *graw = gpos + 4 * m.e;
             const uint8_t *spos = sh.pos[s] + m.pos_skew;
             const uint8_t *sraw = sh.raw[s] + m.raw_skew;
+            const uint8_t *gsm = m.c + kHeader + m.elem0;
+            const uint8_t *gcodes = m.c + kHeader + m.n;
             for (uint32_t i = tid; i < m.cnt; i += kThreads) {
                 const uint64_t g = (uint64_t)m.lo + i;
                 const uint64_t p = es ? *reinterpret_cast<const uint32_t *>(spos + 4 * i) : load_u32_any(gpos + 4 * g);
-                const uint64_t pp = i == 0 ? 0 : (es ? *reinterpret_cast<const uint32_t *>(spos + 4 * (i - 1))
-                                                     : load_u32_any(gpos + 4 * (g - 1)));
                 const uint32_t x = es ? sraw[i] : graw[g];
-                const bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x) || (i > 0 && pp >= p);
+                bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x);
+                if (i > 0) {
+                    const uint64_t pp = es ? *reinterpret_cast<const uint32_t *>(spos + 4 * (i - 1))
+                                           : load_u32_any(gpos + 4 * (g - 1));
+                    bad |= pp >= p;
+                }
+                if (!bad) {
+                    const uint32_t l = (uint32_t)(p - m.elem0);
+                    const uint32_t cbyte = ss ? sh.codes[s][l >> 1] : gcodes[(p >> 1)];
+                    if (((cbyte >> (4 * (l & 1))) & 0xFu) != 0) bad = true;  // placeholder must be 0
+                    const uint32_t smb = ss ? sh.sm[s][l] : gsm[l];
+                    if (!bad && m.dst != nullptr)
+                        m.dst[l] = (uint16_t)(((smb & 0x80u) << 8) | (x << 7) | (smb & 0x7Fu));
+                }
                 if (bad) set_status(status, SZ_ERR_CORRUPT);
-                const uint32_t local = bad ? kNoEsc : (uint32_t)(p - m.elem0);
-                ep[i] = (uint16_t)local;
-                if (!es) sh.raw[s][i] = (uint8_t)x;  // exponents read from global: keep them staged
-                const bool first = i == 0 || pp < m.elem0 || ((uint32_t)(pp - m.elem0) >> 4) != (local >> 4);
-                if (!bad && first) cf[local >> 4] = (uint16_t)i;
-            }
-            consumer_sync();
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) decode_store_chunk<true>(m, sh, s, T, q, tid, status);
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) cf[q * kThreads + tid] = kNoEsc;  // this thread's own entries
-        } else {
-            // more escapes than one stage holds: decode all chunks into
-            // registers, then stream the escapes through the stage's escape
-            // area in batches (every consumer takes part)
-            uint4 o[2 * kChunks];
-            uint64_t cw[kChunks];
-#pragma unroll
-            for (int q = 0; q < kChunks; ++q) {
-                const uint32_t off = (q * kThreads + tid) * kChunk;
-                const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
-                uint4 smv = make_uint4(0, 0, 0, 0);
-                uint64_t codes = 0;
-                if (m.flags & kDFlagInSmem) {
-                    smv = *reinterpret_cast<const uint4 *>(sh.sm[s] + off);
-                    codes = *reinterpret_cast<const unsigned long long *>(sh.codes[s] + off / 2);
-                } else if (cnt) {
-                    const uint8_t *in_sm = m.c + kHeader + m.elem0;
-                    const uint8_t *cb = m.c + kHeader + m.n + (m.elem0 + off) / 2;
-                    uint32_t sw[4] = {0, 0, 0, 0};
-#pragma unroll
-                    for (int jj = 0; jj < kChunk; ++jj)
-                        if (jj < (int)cnt) sw[jj >> 2] |= (uint32_t)in_sm[off + jj] << (8 * (jj & 3));
-                    smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-#pragma unroll
-                    for (int b = 0; b < kChunk / 2; ++b)
-                        if (2 * b < (int)cnt) codes |= (uint64_t)cb[b] << (8 * b);
-                    if ((cnt & 1) && ((codes >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                    if (cnt < (uint32_t)kChunk) codes &= (1ull << (4 * cnt)) - 1ull;
-                }
-                cw[q] = codes;
-                decode_chunk(smv, codes, T, o[2 * q], o[2 * q + 1]);
-            }
-            uint8_t *er = sh.raw[s];
-            for (uint32_t b0 = 0; b0 < m.cnt; b0 += kEscCap) {
-                const uint32_t nb = umin32(kEscCap, m.cnt - b0);
-                consumer_sync();
-                for (uint32_t i = tid; i < nb; i += kThreads) {
-                    const uint64_t g = (uint64_t)m.lo + b0 + i;
-                    const uint64_t p = load_u32_any(gpos + 4 * g);
-                    const uint32_t x = graw[g];
-                    bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x);
-                    if (b0 + i > 0) bad |= load_u32_any(gpos + 4 * (g - 1)) >= p;
-                    if (bad) set_status(status, SZ_ERR_CORRUPT);
-                    ep[i] = bad ? kNoEsc : (uint16_t)(p - m.elem0);
-                    er[i] = (uint8_t)x;
-                }
-                consumer_sync();
-#pragma unroll
-                for (int q = 0; q < kChunks; ++q) {
-                    const uint32_t off = (q * kThreads + tid) * kChunk;
-                    uint32_t a0 = 0, a1 = nb;  // first staged escape at or after off
-                    while (a0 < a1) {
-                        const uint32_t mid = (a0 + a1) >> 1;
-                        if (ep[mid] < off) a0 = mid + 1; else a1 = mid;
-                    }
-                    for (uint32_t i = a0; i < nb && ep[i] < off + kChunk; ++i) {
-                        const int jj = (int)(ep[i] - off);
-                        if (((cw[q] >> (4 * jj)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);
-                        patch_elem(o[2 * q], o[2 * q + 1], jj, er[i]);
-                    }
-                }
-            }
-            if (m.dst != nullptr) {
-#pragma unroll
-                for (int q = 0; q < kChunks; ++q) {
-                    const uint32_t off = (q * kThreads + tid) * kChunk;
-                    const uint32_t cnt = off < m.len ? umin32(kChunk, m.len - off) : 0u;
-                    if (cnt == (uint32_t)kChunk) {
-                        st_stream_v4(m.dst + off, o[2 * q]);
-                        st_stream_v4(m.dst + off + 8, o[2 * q + 1]);
-                    } else if (cnt) {
-                        const uint32_t w[8] = {o[2 * q].x, o[2 * q].y, o[2 * q].z, o[2 * q].w,
-                                               o[2 * q + 1].x, o[2 * q + 1].y, o[2 * q + 1].z, o[2 * q + 1].w};
-#pragma unroll
-                        for (int jj = 0; jj < kChunk; ++jj)
-                            if (jj < (int)cnt) m.dst[off + jj] = (uint16_t)(w[jj >> 1] >> (16 * (jj & 1)));
-                    }
-                }
             }
         }
         __syncwarp();

@@ -248,7 +248,7 @@ __device__ __forceinline__ void copy_out_escapes(const uint32_t *stg, const Pend
 // warp, warp total), both packed as four 16-bit fields.  When no chunk holds
 // more than one escape -- the usual case -- ballots do it; otherwise a
 // shuffle scan of the packed counts.
-__device__ __forceinline__ void warp_escape_scan(const uint32_t (&esc)[kChunks], int lane, uint64_t &excl,
+__device__ __forceinline__ bool warp_escape_scan(const uint32_t (&esc)[kChunks], int lane, uint64_t &excl,
                                                  uint64_t &total) {
     uint32_t cnt[kChunks];
     uint32_t any_multi = 0;
@@ -267,7 +267,7 @@ __device__ __forceinline__ void warp_escape_scan(const uint32_t (&esc)[kChunks],
             excl |= (uint64_t)__popc(b & below) << (16 * c);
             total |= (uint64_t)__popc(b) << (16 * c);
         }
-        return;
+        return false;
     }
     uint64_t v = 0;
 #pragma unroll
@@ -280,6 +280,7 @@ __device__ __forceinline__ void warp_escape_scan(const uint32_t (&esc)[kChunks],
     }
     excl = incl - v;
     total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    return true;  // some chunk of the warp has several escapes
 }
 
 template <bool kBatched>
@@ -385,7 +386,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
 
         // ---- escapes: position of every escape in the sub-tile's order
         uint64_t wexcl, wtot;
-        warp_escape_scan(esc, lane, wexcl, wtot);
+        const bool multi = warp_escape_scan(esc, lane, wexcl, wtot);
         uint64_t *wt = sh.warp_tot[j & 1];
         if (lane == 0) wt[wid] = wtot;
         const int s_next = (int)((j + 1) % kEncStages);
@@ -418,14 +419,21 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             uint32_t chunk_base = 0;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
-                uint32_t msk = esc[c] ? esc_in_element_order(esc[c]) : 0u;
                 uint32_t idx = chunk_base + field16(thr_excl, c);  // index within the sub-tile
                 chunk_base += field16(tot, c);
-                if (!msk) continue;
+                if (!esc[c]) continue;
                 const uint32_t off = (c * kThreads + tid) * kChunk;
-                while (msk) {  // ascending element order
-                    const int q = __ffs(msk) - 1;
+                // the usual case, one escape in the chunk: no ordering loop
+                uint32_t msk = multi ? esc_in_element_order(esc[c]) : 0u;
+                int q = 0;
+                if (!multi) {
+                    const int bit = __ffs(esc[c]) - 1;
+                    q = 4 * (bit & 7) + (bit >> 3);
+                } else {
+                    q = __ffs(msk) - 1;
                     msk &= msk - 1;
+                }
+                for (;;) {  // ascending element order
                     const uint32_t x = in_smem ? (uint32_t)reinterpret_cast<const uint16_t *>(stage)[off + q]
                                                : (uint32_t)m.src[off + q];
                     const uint32_t raw = (x >> 7) & 0xFFu;
@@ -441,6 +449,9 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
                         raw_base[g] = (uint8_t)raw;
                     }
                     ++idx;
+                    if (!msk) break;
+                    q = __ffs(msk) - 1;
+                    msk &= msk - 1;
                 }
             }
             if (staged) {
