@@ -124,16 +124,13 @@ __device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligne
 
 __device__ __forceinline__ uint32_t field16(uint64_t v, int c) { return (uint32_t)(v >> (16 * c)) & 0xFFFFu; }
 
-// Read chunk (c, tid) of a stage: 32 bytes at (c*256 + tid)*32.  Lanes with
-// bit 2 set read the upper half first, so each quarter-warp's 16-byte reads
-// cover all 32 banks exactly once.
+// Read chunk (c, tid) of a stage: 32 bytes at (c*256 + tid)*32 (two 16-byte
+// reads; a quarter-warp's reads meet each bank twice, cheaper here than the
+// selects that would avoid it).
 __device__ __forceinline__ void read_chunk_smem(const uint8_t *stage, int c, int tid, uint4 &v0, uint4 &v1) {
-    const uint8_t *p = stage + (uint32_t)(c * kThreads + tid) * 32u;
-    const uint32_t h = ((uint32_t)tid >> 2) & 1u;
-    const uint4 a = *reinterpret_cast<const uint4 *>(p + 16 * h);
-    const uint4 b = *reinterpret_cast<const uint4 *>(p + 16 * (1 - h));
-    v0 = h ? b : a;
-    v1 = h ? a : b;
+    const uint4 *p = reinterpret_cast<const uint4 *>(stage + (uint32_t)(c * kThreads + tid) * 32u);
+    v0 = p[0];
+    v1 = p[1];
 }
 
 // Chunk from global memory, `cnt` (<= 16) valid elements, the rest zero.
@@ -344,6 +341,19 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const bool in_smem = (m.flags & kFlagInSmem) != 0;
 
         uint32_t esc[kChunks];
+        if (in_smem && codes_aligned) {  // a full sub-tile in shared memory
+            uint8_t *psm = out_sm + tid * kChunk;
+            uint8_t *pcw = codes_base + (m.elem0 + tid * kChunk) / 2;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                uint4 v0, v1, smv;
+                uint64_t cw;
+                read_chunk_smem(stage, c, tid, v0, v1);
+                encode_chunk(v0, v1, smv, cw, esc[c]);
+                st_stream_v4(psm + c * kThreads * kChunk, smv);
+                st_stream_u64(pcw + c * kThreads * kChunk / 2, cw);
+            }
+        } else {
 #pragma unroll
         for (int c = 0; c < kChunks; ++c) {
             const uint32_t off = (c * kThreads + tid) * kChunk;
@@ -351,13 +361,6 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             if (off >= m.len) continue;
             uint4 v0, v1, smv;
             uint64_t cw;
-            if (in_smem && codes_aligned) {
-                read_chunk_smem(stage, c, tid, v0, v1);
-                encode_chunk(v0, v1, smv, cw, esc[c]);
-                st_stream_v4(out_sm + off, smv);
-                st_stream_u64(codes_base + (m.elem0 + off) / 2, cw);
-                continue;
-            }
             // ragged or unaligned chunk: guarded element loads, encoded as a
             // full chunk, cnt of it kept
             const uint32_t cnt = umin32(kChunk, m.len - off);
@@ -383,6 +386,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
                     if (2 * b < (int)cnt) cb[b] = (uint8_t)(cw >> (8 * b));
             }
         }
+        }
 
         // ---- escapes: position of every escape in the sub-tile's order
         uint64_t wexcl, wtot;
@@ -392,13 +396,17 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const int s_next = (int)((j + 1) % kEncStages);
         if (tid == 0) sh.go[(j + 1) & 1] = mbar_wait(&sh.full[s_next], ((j + 1) / kEncStages) & 1u, a.wait_limit_ns) ? 1 : 0;
         consumer_sync();
-        uint64_t warp_excl = 0, tot = 0;
+        // warp totals -> this warp's exclusive prefix and the sub-tile total
+        // (packed fields): an 8-lane shuffle scan instead of 8 sums per thread
+        uint64_t wv = lane < kWarps ? wt[lane] : 0ull;
+        uint64_t wi = wv;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const uint64_t v = wt[w];
-            if (w < wid) warp_excl += v;
-            tot += v;
+        for (int d = 1; d < kWarps; d <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xFFFFFFFFu, wi, d);
+            if (lane >= d) wi += y;
         }
+        const uint64_t tot = __shfl_sync(0xFFFFFFFFu, wi, kWarps - 1);
+        const uint64_t warp_excl = __shfl_sync(0xFFFFFFFFu, wi - wv, wid);
         const uint64_t thr_excl = warp_excl + wexcl;
         const uint32_t sub_total = field16(tot, 0) + field16(tot, 1) + field16(tot, 2) + field16(tot, 3);
 
