@@ -241,6 +241,34 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
                             uint64_t page_elems, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
                             void *stream);
 
+/* ------------------------------------------------------- no-allocation path */
+/*
+ * sz_encode_static -- the whole compression of one tensor (histogram,
+ * codebook, container) without any workspace from the caller and without
+ * allocating: for callers that cannot allocate device memory at the moment
+ * they compress -- code running inside an allocator or memory-pool callback,
+ * or an engine that reserved all device memory up front.  The explainer has
+ * no counterpart; it is an interface of this library only.
+ *
+ * Its scratch is one file-scope device array of SZ_STATIC_SCRATCH_BYTES,
+ * present on every GPU that loads the library until the process exits.
+ *   d_in, n         n <= SZ_STATIC_MAX_ELEMS (2^28 elements, 512 MiB of
+ *                   BF16); larger n returns SZ_ERR_TOO_LARGE
+ *   d_out, out_cap, d_out_bytes, d_status  as for sz_encode
+ *   d_codebook16_or_null  optional out: the 16-entry codebook
+ * The container is byte for byte the one sz_histogram_codebook + sz_encode
+ * write.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls on a device share the one array: calls that overlap on the GPU
+ * (other streams, other host threads) race and must be serialised by the
+ * caller.
+ */
+#define SZ_STATIC_MAX_ELEMS (1ull << 28)
+#define SZ_STATIC_SCRATCH_BYTES (1280ull + 1028ull * 4096ull)
+sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap,
+                           uint64_t *d_out_bytes, uint8_t *d_codebook16_or_null, int32_t *d_status,
+                           void *stream);
+
 /* ------------------------------------------------------------ diagnostics */
 /*
  * sz_set_wait_limit_ns -- upper bound, in nanoseconds of device time, of

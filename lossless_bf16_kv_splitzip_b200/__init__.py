@@ -24,7 +24,7 @@ from ._build import LIB_PATH, build, is_stale
 
 __all__ = [
     "SzError", "sz_plan", "sz_histogram_codebook", "sz_encode", "sz_decode", "sz_plan_batched",
-    "sz_histogram_codebook_batched", "sz_encode_batched", "sz_decode_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags",
+    "sz_histogram_codebook_batched", "sz_encode_batched", "sz_encode_static", "sz_decode_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags",
     "sz_tile_elems", "sz_version", "encode", "decode", "BatchPlan", "lib", "HEADER_BYTES",
     "max_bytes", "STATUS",
 ]
@@ -71,6 +71,7 @@ def lib():
             "sz_histogram_codebook_batched": [u32, vp, u64, vp, u64, vp, vp, vp, u64, vp],
             "sz_encode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, vp, u64, vp],
             "sz_decode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, u64, vp],
+            "sz_encode_static": [vp, u64, vp, u64, vp, vp, vp, vp],
             "sz_set_wait_limit_ns": [u64],
             "sz_debug_set_flags": [u32],
         }
@@ -172,6 +173,13 @@ def sz_decode_batched(n_segs, d_segs, n_tiles, d_in, in_cap, d_pages, page_elems
                       stream=None):
     _check(lib().sz_decode_batched(n_segs, _p(d_segs), n_tiles, _p(d_in), in_cap, _p(d_pages), page_elems,
                                    _p(d_status), _p(d_ws), ws_bytes, _s(stream)), "sz_decode_batched")
+
+
+def sz_encode_static(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16, d_status, stream=None):
+    """Compress one tensor using the library's own device scratch array (no
+    workspace argument, nothing allocated); n <= 2^28."""
+    _check(lib().sz_encode_static(_p(d_in), n, _p(d_out), out_cap, _p(d_out_bytes), _p(d_codebook16),
+                                  _p(d_status), _s(stream)), "sz_encode_static")
 
 
 def sz_set_wait_limit_ns(limit_ns: int):
