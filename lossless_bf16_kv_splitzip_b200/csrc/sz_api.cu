@@ -58,7 +58,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 //   meta       SegMeta[S]      codebook and escape count per segment
 //   tile_hist  u32[T][256]     exponent counts per tile
 //   tile_off   u32[T]          first escape index of each tile
-//   sub_start  u32[4T + S]     first escape index of each sub-tile (decode)
+//   sub_start  u32[4T + S]     first escape index of each sub-tile (decode; 4 = sub-tiles per tile)
 struct Ws {
     uint64_t seg_hist, meta, tile_hist, tile_off, sub_start, total;
 };
@@ -69,7 +69,7 @@ Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
     w.tile_hist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
     w.tile_off = round_up(w.tile_hist + 1024 * n_tiles, kAlign);
     w.sub_start = round_up(w.tile_off + 4 * n_tiles, kAlign);
-    w.total = round_up(w.sub_start + 4 * (4 * n_tiles + n_segs), kAlign);
+    w.total = round_up(w.sub_start + 4 * (kSubsPerTile * n_tiles + n_segs), kAlign);
     return w;
 }
 

@@ -10,7 +10,7 @@
 // binary search per sub-tile, all in parallel); it also checks each
 // segment's header.  (2) decode_kernel, warp-specialised like the encode:
 //   producer warp   TMA bulk copies of the sub-tile's sm bytes (16 KiB) and
-//                   codes (8 KiB) into a 3-stage ring; its 32 lanes also
+//                   codes (8 KiB) into a 2-stage ring (3 CTAs per SM); its 32 lanes also
 //                   load the sub-tile's escape records, check them (inside
 //                   the sub-tile, strictly ascending, raw exponent outside
 //                   the codebook) and store them in the stage together with
@@ -61,10 +61,10 @@ __device__ inline Header read_header(const uint8_t *c, uint64_t cap, uint64_t n)
 }
 
 // ------------------------------------------------- per-sub-tile escape index
-// Entry j of segment k (j = 4*tile + sub, j = 0..4*tiles_k) = index of the
-// first escape whose position is >= the first element of that sub-tile
-// (sub-tiles past a short tile's end start at the tile's end); entry
-// 4*tiles_k = e.  Entries of segment k start at 4*tile_begin_k + k.
+// Entry j of segment k (j = S*tile + sub, S = kSubsPerTile, j = 0..S*tiles_k)
+// = index of the first escape whose position is >= the first element of that
+// sub-tile (sub-tiles past a short tile's end start at the tile's end); entry
+// S*tiles_k = e.  Entries of segment k start at S*tile_begin_k + k.
 template <bool kBatched>
 __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint64_t n_entries) {
     __shared__ uint64_t s_entry_begin[kMaxSmemSegs + 1];
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
     const bool cached = kBatched && ns <= kMaxSmemSegs;
     if (cached) {
         for (uint32_t i = threadIdx.x; i < ns; i += blockDim.x)
-            s_entry_begin[i] = 4 * a.batch.segs[i].tile_begin + i;
+            s_entry_begin[i] = kSubsPerTile * a.batch.segs[i].tile_begin + i;
     }
     __syncthreads();
     const uint64_t j_glob = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -82,20 +82,20 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
         uint32_t lo = 0, hi = ns;
         while (hi - lo > 1) {
             const uint32_t mid = (lo + hi) >> 1;
-            const uint64_t b = cached ? s_entry_begin[mid] : 4 * a.batch.segs[mid].tile_begin + mid;
+            const uint64_t b = cached ? s_entry_begin[mid] : kSubsPerTile * a.batch.segs[mid].tile_begin + mid;
             if (b <= j_glob) lo = mid; else hi = mid;
         }
         k = lo;
     }
     const sz_segment seg = load_segment(a.batch, k);
-    const uint64_t j = j_glob - (4 * seg.tile_begin + k);
+    const uint64_t j = j_glob - (kSubsPerTile * seg.tile_begin + k);
     const uint64_t tiles = segment_tiles(seg.n_elems, a.batch.page_elems);
-    uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k;
-    if (j > 4 * tiles) return;
+    uint32_t *ts = a.sub_start + kSubsPerTile * seg.tile_begin + k;
+    if (j > kSubsPerTile * tiles) return;
     const uint64_t cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
     const uint8_t *c = a.in + seg.out_offset;
     const Header h = read_header(c, cap, seg.n_elems);
-    if (j == 4 * tiles) {  // the sentinel thread reports the header of its segment
+    if (j == kSubsPerTile * tiles) {  // the sentinel thread reports the header of its segment
         if (!h.ok) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
         ts[j] = h.ok ? (uint32_t)h.e : 0u;
         return;
@@ -104,8 +104,8 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
         ts[j] = 0;
         return;
     }
-    const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / 4);
-    const uint64_t first = r.elem0 + umin32((uint32_t)(j % 4) * kSub, r.len);
+    const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / kSubsPerTile);
+    const uint64_t first = r.elem0 + umin32((uint32_t)(j % kSubsPerTile) * kSub, r.len);
     const uint64_t n = h.n, e = h.e;
     const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
     uint64_t lo = 0, hi = e;  // first index with pos >= first
@@ -179,7 +179,7 @@ __device__ __forceinline__ void patch_elem(uint4 &o0, uint4 &o1, int j, uint32_t
 #undef SZ_PATCH
 }
 
-constexpr int kDecStages = 3;
+constexpr int kDecStages = 2;  // 3 CTAs per SM
 constexpr uint32_t kEscCap = 1024;  // escape records bulk-copied per sub-tile; more: read directly
 
 constexpr uint32_t kDFlagEnd = 1u;
@@ -245,7 +245,7 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
         // the tile's five sub-tile starts; the last sub-tile of a tile ends
         // where the next tile starts (the segment's last: at e), so the
         // ranges cover every escape record
-        const uint32_t *ts = a.sub_start + 4 * seg.tile_begin + k + 4 * (uint64_t)r.local;
+        const uint32_t *ts = a.sub_start + kSubsPerTile * (seg.tile_begin + r.local) + k;
         uint32_t tsv[kSubsPerTile + 1];
 #pragma unroll
         for (uint32_t q = 0; q <= kSubsPerTile; ++q) tsv[q] = ts[q];
@@ -459,7 +459,7 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
 }
 
 template <bool kBatched>
-__global__ void __launch_bounds__(kPipeThreads, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     DecShared &sh = *reinterpret_cast<DecShared *>(smem_raw);
     const int tid = threadIdx.x;
@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) decode_kernel(const DecodeArg
 }
 
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {
-    const uint64_t entries = 4 * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
+    const uint64_t entries = kSubsPerTile * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
     const uint64_t grid = div_up(entries, 256);
     if (batched)
         esc_index_kernel<true><<<(unsigned)grid, 256, 0, s>>>(a, entries);

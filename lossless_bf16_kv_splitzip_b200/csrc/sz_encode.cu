@@ -11,8 +11,9 @@
 //
 // One persistent CTA per slot, warp-specialised:
 //   producer warp   walks the CTA's tiles, 1-D TMA bulk copy of each
-//                   16,384-element sub-tile (32 KiB) into a 3-stage
-//                   shared-memory ring, signalled by mbarriers;
+//                   16,384-element sub-tile (32 KiB) into a 2-stage
+//                   shared-memory ring (3 CTAs per SM), signalled by
+//                   mbarriers;
 //   8 consumer warps read the stage, write the sm stream (16-byte stores)
 //                   and code stream (8-byte stores), scan the escape counts
 //                   across the CTA and write the escape records in element
@@ -22,8 +23,8 @@
 
 namespace sz {
 
-constexpr int kEncStages = 3;
-constexpr uint32_t kEscStage = 1024;  // staged escape records per sub-tile; more: written directly
+constexpr int kEncStages = 2;  // x 32 KiB; 3 CTAs per SM
+constexpr uint32_t kEscStage = 512;  // staged escape records per sub-tile; more: written directly
 
 constexpr uint32_t kFlagEnd = 1u;        // no more sub-tiles
 constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
@@ -487,7 +488,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
 }
 
 template <bool kBatched>
-__global__ void __launch_bounds__(kPipeThreads, 2) encode_kernel(const EncodeArgs a) {
+__global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     EncShared &sh = *reinterpret_cast<EncShared *>(smem_raw);
     const int tid = threadIdx.x;

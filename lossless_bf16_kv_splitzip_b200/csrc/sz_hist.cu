@@ -74,6 +74,11 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const HistArgs a) {
         for (uint32_t sub = 0; ok && sub < r.n_subs; ++sub) {
             const uint16_t *p = src + sub * kSub;
             const uint32_t len = umin32(kSub, r.len - sub * kSub);
+            // bulk prefetch of the next sub-tile into L2 while this one is counted
+            if (tid == 0 && sub + 1 < r.n_subs) {
+                const uint32_t next = (umin32(kSub, r.len - (sub + 1) * kSub) * 2u) & ~15u;
+                if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + kSub), "r"(next) : "memory");
+            }
             if (len == kSub) {
                 uint4 v[2 * kChunks];
 #pragma unroll
