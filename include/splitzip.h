@@ -53,8 +53,8 @@
  *   - Errors the host can see (null pointer, size, alignment, workspace or
  *     capacity too small, launch failure) are returned at once and nothing
  *     is enqueued.  Errors only the device can see (corrupt container,
- *     workspace histogram that does not describe the input, a lookback wait
- *     that ran out) are written as an sz_status to the caller's d_status
+ *     workspace histogram that does not describe the input, a device-side
+ *     wait that ran out) are written as an sz_status to the caller's d_status
  *     word(s), which the call first sets to SZ_OK.  A container whose status
  *     is not SZ_OK must not be used.
  *   - Vector path: device buffers must be 16-byte aligned (SZ_ERR_ALIGN
@@ -135,8 +135,11 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
  *                   SZ_ERR_CAPACITY, SZ_ERR_INVALID, SZ_ERR_DEVICE_TIMEOUT)
  *   d_ws, ws_bytes  the workspace passed to sz_histogram_codebook for this
  *                   same input (its histogram gives the escape count).
- * The escape stream is compacted in element order across tiles by a
- * decoupled lookback whose waits are bounded (SZ_ERR_DEVICE_TIMEOUT).
+ * The escape stream is compacted in element order across tiles: every
+ * tile's first escape index comes from the workspace's per-tile histograms
+ * (an exclusive scan of the tiles' escape counts under this codebook), so
+ * no tile waits on another; a pipeline wait that runs out gives
+ * SZ_ERR_DEVICE_TIMEOUT.
  */
 sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
                     uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status_or_null, void *d_ws,
@@ -185,7 +188,10 @@ typedef struct sz_segment {
  *   h_segs          out: the segment table (pages numbered consecutively,
  *                   containers at 256-byte aligned offsets, each slot
  *                   SZ_MAX_BYTES(n_elems) long); copy it to the device for
- *                   the batched calls
+ *                   the batched calls.  The container offsets depend only
+ *                   on the segment lengths: a plan of the same lengths with
+ *                   another page_elems finds the same containers, so a
+ *                   batch can be decoded into pages of another size.
  *   *total_pages    out: page pointers the page array must hold
  *   *n_tiles        out: tiles of the whole batch (pass to the calls below)
  *   *out_bytes      out: container buffer size
@@ -264,7 +270,7 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
  * caller.
  */
 #define SZ_STATIC_MAX_ELEMS (1ull << 28)
-#define SZ_STATIC_SCRATCH_BYTES (1280ull + 1028ull * 4096ull)
+#define SZ_STATIC_SCRATCH_BYTES (1536ull + 2064ull * 1024ull)
 sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap,
                            uint64_t *d_out_bytes, uint8_t *d_codebook16_or_null, int32_t *d_status,
                            void *stream);
@@ -272,7 +278,8 @@ sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uin
 /* ------------------------------------------------------------ diagnostics */
 /*
  * sz_set_wait_limit_ns -- upper bound, in nanoseconds of device time, of
- * every device-side wait (the encode's lookback on a predecessor tile).
+ * every device-side wait (a pipeline stage of the encode or decode kernel
+ * waiting for its bulk copy).
  * Default 1e9 (one second).  A wait that runs out sets
  * SZ_ERR_DEVICE_TIMEOUT in the segment's status and the kernel returns.
  * Applies to calls made after it, process-wide.
@@ -280,13 +287,15 @@ sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uin
 sz_status sz_set_wait_limit_ns(uint64_t limit_ns);
 
 /*
- * sz_debug_set_flags -- test hook.  Bit 0: tiles never publish their
- * escape counts, so every lookback wait runs out (exercises the timeout
- * path without faulting anything).  0 restores normal operation.
+ * sz_debug_set_flags -- test hook.  Bit 0: the encode and decode kernels'
+ * copy threads issue no bulk copy, so every stage wait of their consumer
+ * threads runs out (exercises the timeout path without faulting
+ * anything).  0 restores normal operation.
  */
 sz_status sz_debug_set_flags(uint32_t flags);
 
-/* Tile size in elements used by every kernel (16384). */
+/* Tile size in elements used by every kernel (65536; a tile never crosses
+ * a page, so the last tile of a page may be shorter). */
 uint64_t sz_tile_elems(void);
 
 /* Library version string, e.g. "splitzip-b200 1.0 sm_100a". */

@@ -286,8 +286,12 @@ class BatchPlan:
         self.histogram(d_page_ptrs, stream)
         self.encode_only(d_page_ptrs, stream)
 
-    def decode(self, d_page_ptrs, stream=None):
-        sz_decode_batched(self.n_segs, self.d_segs, self.n_tiles, self.container, self.container.numel(),
+    def decode(self, d_page_ptrs, stream=None, container=None):
+        """Decode every segment into the pages d_page_ptrs lists.  container:
+        another plan's container buffer for the same segment lengths (its
+        offsets are the same), e.g. to decode into another page size."""
+        c = self.container if container is None else container
+        sz_decode_batched(self.n_segs, self.d_segs, self.n_tiles, c, c.numel(),
                           d_page_ptrs, self.page_elems, self.dec_status, self.ws, self.ws.numel(), stream)
 
     def container_bytes(self, k: int, size: int) -> "np.ndarray":

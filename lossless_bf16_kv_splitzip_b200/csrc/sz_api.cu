@@ -7,13 +7,11 @@
 #include "sz_internal.cuh"
 
 namespace sz {
-cudaError_t launch_hist(const HistArgs &a, bool batched, int grid, cudaStream_t s);
-cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
-cudaError_t launch_encode(const EncodeArgs &a, bool batched, int grid, cudaStream_t s);
+cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s);
+cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s);
+cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
-int hist_blocks_per_sm();
-int encode_blocks_per_sm();
 int decode_blocks_per_sm();
 }  // namespace sz
 
@@ -29,7 +27,7 @@ std::atomic<uint32_t> g_debug_flags{0};
 
 struct DeviceInfo {
     bool ready = false;
-    int sms = 0, hist_occ = 1, enc_occ = 1, dec_occ = 1;
+    int sms = 0, dec_occ = 1;
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[64];
@@ -41,8 +39,6 @@ bool device_info(DeviceInfo &out) {
     DeviceInfo &d = g_dev[dev];
     if (!d.ready) {
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-        d.hist_occ = hist_blocks_per_sm();
-        d.enc_occ = encode_blocks_per_sm();
         d.dec_occ = decode_blocks_per_sm();
         d.ready = true;
     }
@@ -53,22 +49,26 @@ bool device_info(DeviceInfo &out) {
 uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// ---- workspace layout for S segments and T tiles (256-byte aligned parts)
-//   seg_hist   u32[S][256]     exponent counts per segment
+// ---- workspace layout for S segments, T tiles and G = min(T, kMaxRanges)
+// ranges (256-byte aligned parts)
+//   seg_hist   u32[S][256]     exponent counts per segment      } zeroed together
+//   seg_done   u32[S]          tiles counted so far per segment } by the histogram call
 //   meta       SegMeta[S]      codebook and escape count per segment
-//   tile_hist  u32[T][256]     exponent counts per tile
-//   tile_off   u32[T]          first escape index of each tile
+//   rhist      u32[G][2][256]  counts of each range's first and last piece
+//   rrec       RangeRec[G]     escape placement of each range's pieces
 //   sub_start  u32[4T + S]     first escape index of each sub-tile (decode; 4 = sub-tiles per tile)
 struct Ws {
-    uint64_t seg_hist, meta, tile_hist, tile_off, sub_start, total;
+    uint64_t seg_hist, seg_done, meta, rhist, rrec, sub_start, total;
 };
 Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
+    const uint64_t g = umin64(n_tiles, kMaxRanges);
     Ws w;
     w.seg_hist = 0;
-    w.meta = round_up(w.seg_hist + 1024 * n_segs, kAlign);
-    w.tile_hist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
-    w.tile_off = round_up(w.tile_hist + 1024 * n_tiles, kAlign);
-    w.sub_start = round_up(w.tile_off + 4 * n_tiles, kAlign);
+    w.seg_done = 1024 * n_segs;
+    w.meta = round_up(w.seg_done + 4 * n_segs, kAlign);
+    w.rhist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
+    w.rrec = round_up(w.rhist + 2048 * g, kAlign);
+    w.sub_start = round_up(w.rrec + sizeof(RangeRec) * g, kAlign);
     w.total = round_up(w.sub_start + 4 * (kSubsPerTile * n_tiles + n_segs), kAlign);
     return w;
 }
@@ -104,6 +104,28 @@ T *at(void *ws, uint64_t off) {
     return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
 }
 
+// The select's view of the workspace, with the range partition of this
+// device (the histogram and encode calls of one batch derive the same one).
+SelectCtx select_ctx(const Batch &b, void *ws, const Ws &w, const DeviceInfo &dev) {
+    SelectCtx c{};
+    c.batch = b;
+    c.seg_hist = at<uint32_t>(ws, w.seg_hist);
+    c.rhist = at<uint32_t>(ws, w.rhist);
+    c.meta = at<SegMeta>(ws, w.meta);
+    c.rrec = at<RangeRec>(ws, w.rrec);
+    c.range_tiles = plan_ranges(b.n_tiles, (uint64_t)dev.sms).tiles;
+    return c;
+}
+
+HistArgs hist_args(const SelectCtx &c, void *ws, const Ws &w) {
+    HistArgs h{};
+    h.sel = c;
+    h.seg_hist = at<uint32_t>(ws, w.seg_hist);
+    h.seg_done = at<uint32_t>(ws, w.seg_done);
+    h.rhist = at<uint32_t>(ws, w.rhist);
+    return h;
+}
+
 sz_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SZ_OK : SZ_ERR_CUDA; }
 
 #define SZ_TRY_CUDA(call)                          \
@@ -134,24 +156,13 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024, s));
-    HistArgs h{};
-    h.batch = single_batch(n);
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 + 4, s));  // seg_hist, seg_done
+    SelectCtx c = select_ctx(single_batch(n), d_ws, w, dev);
+    c.codebooks_out = d_codebook16;
+    c.hist_out = d_hist256_or_null;
+    HistArgs h = hist_args(c, d_ws, w);
     h.base = d_in;
-    h.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
-    h.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
-    h.status = nullptr;
-    SZ_TRY_CUDA(launch_hist(h, false, dev.sms * dev.hist_occ, s));
-    SelectArgs sa{};
-    sa.batch = h.batch;
-    sa.seg_hist = h.seg_hist;
-    sa.tile_hist = h.tile_hist;
-    sa.meta = at<SegMeta>(d_ws, w.meta);
-    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
-    sa.codebook_in = nullptr;
-    sa.codebooks_out = d_codebook16;
-    sa.hist_out = d_hist256_or_null;
-    return cuda_status(launch_select(sa, s));
+    return cuda_status(launch_hist(h, false, s));
 }
 
 sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
@@ -166,30 +177,28 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
-    // escape count and per-tile escape offsets for this codebook, from the
-    // histograms sz_histogram_codebook left in the workspace
-    SelectArgs sa{};
-    sa.batch = single_batch(n);
-    sa.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
-    sa.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
-    sa.meta = at<SegMeta>(d_ws, w.meta);
-    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
-    sa.codebook_in = d_codebook16;
-    SZ_TRY_CUDA(launch_select(sa, s));
+    // escape count and range records for this codebook, from the piece
+    // counts sz_histogram_codebook left in the workspace (nothing to do when
+    // it is the codebook chosen there); also resets *d_status, *d_out_bytes
+    ReselectArgs ra{};
+    ra.sel = select_ctx(single_batch(n), d_ws, w, dev);
+    ra.codebook_in = d_codebook16;
+    ra.status = d_status;
+    ra.out_bytes = d_out_bytes;
+    SZ_TRY_CUDA(launch_reselect(ra, s));
     EncodeArgs a{};
-    a.batch = sa.batch;
+    a.batch = ra.sel.batch;
     a.base = d_in;
     a.out = d_out;
     a.out_cap = out_cap;
     a.out_bytes = d_out_bytes;
     a.status = d_status;
-    a.meta = sa.meta;
-    a.tile_off = sa.tile_off;
+    a.meta = ra.sel.meta;
+    a.rrec = ra.sel.rrec;
+    a.range_tiles = ra.sel.range_tiles;
     a.wait_limit_ns = g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
-    return cuda_status(launch_encode(a, false, dev.sms * dev.enc_occ, s));
+    return cuda_status(launch_encode(a, false, s));
 }
 
 sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uint64_t n, int32_t *d_status,
@@ -258,23 +267,14 @@ sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_seg
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 * (uint64_t)n_segs, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1028 * (uint64_t)n_segs, s));  // seg_hist, seg_done
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
-    HistArgs h{};
-    h.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
+    SelectCtx c = select_ctx(make_batch(n_segs, d_segs, n_tiles, page_elems), d_ws, w, dev);
+    c.codebooks_out = d_codebooks_or_null;
+    HistArgs h = hist_args(c, d_ws, w);
     h.pages = d_pages;
-    h.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
-    h.tile_hist = at<uint32_t>(d_ws, w.tile_hist);
     h.status = d_status;
-    SZ_TRY_CUDA(launch_hist(h, true, dev.sms * dev.hist_occ, s));
-    SelectArgs sa{};
-    sa.batch = h.batch;
-    sa.seg_hist = h.seg_hist;
-    sa.tile_hist = h.tile_hist;
-    sa.meta = at<SegMeta>(d_ws, w.meta);
-    sa.tile_off = at<uint32_t>(d_ws, w.tile_off);
-    sa.codebooks_out = d_codebooks_or_null;
-    return cuda_status(launch_select(sa, s));
+    return cuda_status(launch_hist(h, true, s));
 }
 
 sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
@@ -291,18 +291,20 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     if (!device_info(dev)) return SZ_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, 8 * (uint64_t)n_segs, s));
+    const SelectCtx c = select_ctx(make_batch(n_segs, d_segs, n_tiles, page_elems), d_ws, w, dev);
     EncodeArgs a{};
-    a.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
+    a.batch = c.batch;
     a.pages = d_pages;
     a.out = d_out;
     a.out_cap = out_cap;
     a.out_bytes = d_out_bytes;
     a.status = d_status;
-    a.meta = at<SegMeta>(d_ws, w.meta);
-    a.tile_off = at<uint32_t>(d_ws, w.tile_off);
+    a.meta = c.meta;
+    a.rrec = c.rrec;
+    a.range_tiles = c.range_tiles;
     a.wait_limit_ns = g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
-    return cuda_status(launch_encode(a, true, dev.sms * dev.enc_occ, s));
+    return cuda_status(launch_encode(a, true, s));
 }
 
 sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, const uint8_t *d_in,

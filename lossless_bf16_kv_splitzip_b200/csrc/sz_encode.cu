@@ -5,9 +5,9 @@
 // 4-bit code of its codebook slot (two codes per byte), and an exponent
 // outside the codebook becomes an escape note (position, raw exponent).
 // Section 4: fixed-length codes make this one straight pass -- every output
-// byte's address follows from the element index, and each tile's first
-// escape index is already known from the per-tile histograms, so tiles are
-// independent.
+// byte's address follows from the element index, and the first escape
+// index of each CTA's share of tiles is already known from the histogram
+// pass's range records, so CTAs are independent.
 //
 // One persistent CTA per slot, warp-specialised:
 //   producer warp   walks the CTA's tiles, 1-D TMA bulk copy of each
@@ -28,7 +28,7 @@ constexpr uint32_t kEscStage = 512;  // staged escape records per sub-tile; more
 
 constexpr uint32_t kFlagEnd = 1u;        // no more sub-tiles
 constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
-constexpr uint32_t kFlagLastSub = 4u;    // last sub-tile of its tile
+constexpr uint32_t kFlagLastSub = 4u;    // last sub-tile of its piece (the range's tiles of one segment)
 constexpr uint32_t kFlagHeader = 8u;     // first sub-tile of the segment: write the header
 constexpr uint32_t kFlagLastTile = 16u;  // last tile of the segment: write the size
 
@@ -38,8 +38,8 @@ struct EncMeta {
     uint32_t seg;
     uint32_t len;         // elements of the sub-tile
     uint32_t flags;
-    uint32_t esc_base;    // first escape index of the tile
-    uint32_t esc_count;   // escapes the tile must produce
+    uint32_t esc_base;    // first escape index of the piece
+    uint32_t esc_count;   // escapes the piece must produce
     uint32_t pad;
 };
 
@@ -151,16 +151,20 @@ __device__ __forceinline__ void read_chunk_global(const uint16_t *p, uint32_t cn
 template <bool kBatched>
 __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
-    const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
-    const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
+    const uint64_t t_begin = (uint64_t)blockIdx.x * a.range_tiles;
+    const uint64_t t_end = umin64(t_begin + a.range_tiles, a.batch.n_tiles);
+    RangeRec rr{};
+    if (t_begin < t_end) rr = a.rrec[blockIdx.x];
     uint32_t j = 0;
     uint32_t cur = 0xFFFFFFFFu;
     sz_segment seg{};
     bool seg_ok = false;
     uint64_t e_total = 0;
+    uint32_t p_base = 0, p_count = 0;  // the piece's first escape index and escape count
+    uint64_t p_last = 0;               // the piece's last tile
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
-        if (k != cur) {
+        if (k != cur) {  // a new piece: the range's tiles of segment k
             cur = k;
             seg = load_segment(a.batch, k);
             const SegMeta &m = a.meta[k];
@@ -172,12 +176,22 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             if (m.valid == 0) set_status(a.status + k, SZ_ERR_INVALID);
             else if (!fits) set_status(a.status + k, SZ_ERR_CAPACITY);
             else if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
+            const uint64_t seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
+            p_last = umin64(seg_end, t_end) - 1;
+            if (t == t_begin) {  // opens the range
+                p_base = rr.first_off;
+                p_count = rr.first_cnt;
+            } else if (seg_end > t_end) {  // closes the range, the segment goes on
+                p_base = 0;
+                p_count = rr.last_cnt;
+            } else {  // the whole segment
+                p_base = 0;
+                p_count = (uint32_t)e_total;
+            }
         }
         if (!seg_ok) continue;  // every tile of the segment is skipped
         const TileRef r = resolve_tile(a.batch, seg, k, t);
         const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
-        const uint32_t off = a.tile_off[t];
-        const uint64_t next = (r.local + 1 < r.tiles) ? (uint64_t)a.tile_off[t + 1] : e_total;
         const bool aligned = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
         if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
@@ -191,10 +205,10 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             m.elem0 = r.elem0 + (uint64_t)sub * kSub;
             m.seg = k;
             m.len = aligned ? umin32(kSub, r.len - sub * kSub) : 0u;  // nothing is read from a misaligned page
-            m.esc_base = off;
-            m.esc_count = (uint32_t)(next - off);
+            m.esc_base = p_base;
+            m.esc_count = p_count;
             uint32_t f = 0;
-            if (sub + 1 == r.n_subs) f |= kFlagLastSub;
+            if (t == p_last && sub + 1 == r.n_subs) f |= kFlagLastSub;
             if (r.local == 0 && sub == 0) f |= kFlagHeader;
             if (r.local + 1 == r.tiles) f |= kFlagLastTile;
             const bool tma = m.len == kSub;
@@ -288,7 +302,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     uint8_t *out = nullptr;
     uint64_t n = 0, e_total = 0;
     bool codes_aligned = false, pos_aligned = false;
-    uint32_t running = 0;  // escapes of the current tile so far
+    uint32_t running = 0;  // escapes of the current piece so far
     PendingEsc pend{};
 
     // The wait for stage j+1 is folded into sub-tile j's scan barrier: one
@@ -299,7 +313,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const int s = (int)(j % kEncStages);
         if (!sh.go[j & 1]) {  // the same decision in every consumer thread
             if (tid == 0 && a.batch.n_tiles > 0) {
-                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.tiles_per_cta, a.batch.n_tiles - 1);
+                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.range_tiles, a.batch.n_tiles - 1);
                 set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
             }
             return;
@@ -534,13 +548,10 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
     }
 }
 
-cudaError_t launch_encode(const EncodeArgs &a0, bool batched, int grid, cudaStream_t s) {
-    EncodeArgs a = a0;
+// One CTA per range of the partition the histogram kernel used.
+cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s) {
     const size_t smem = sizeof(EncShared);
-    const uint64_t tiles = a.batch.n_tiles;
-    grid = (int)umax64(1, umin64((uint64_t)grid, umax64(tiles, 1)));
-    a.tiles_per_cta = umax64(1, div_up(tiles, (uint64_t)grid));
-    if (tiles > 0) grid = (int)div_up(tiles, a.tiles_per_cta);
+    const int grid = (int)umax64(1, div_up(a.batch.n_tiles, a.range_tiles));
     cudaError_t e;
     if (batched) {
         e = cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -3,12 +3,15 @@
 // SplitZip explainer (gist.science), section 2 "La decouverte secrete": the
 // exponents repeat; section 3 "La strategie SplitZip": the 16 most common
 // exponents get the 4-bit codes.  The histogram pass reads the input once
-// and keeps, besides each segment's 256 counts, the 256 counts of every
-// 65,536-element tile.  The select step orders the 256 exponents by (count
-// descending, exponent ascending), keeps the first 16, and turns the tile
-// histograms into the number of escapes of every tile -- an exclusive scan
-// of those gives each tile the index of its first escape record, so the
-// encode needs no cross-tile communication.
+// and keeps, besides each segment's 256 counts, the 256 counts of the first
+// and last segment piece of every range (the encode's per-CTA share of
+// tiles).  The block that completes a segment orders its 256 exponents by
+// (count descending, exponent ascending), keeps the first 16, and turns the
+// piece counts into the escape count of each of the segment's pieces -- an
+// exclusive scan of those gives every encode CTA the index of its first
+// escape record, so the encode needs no cross-CTA communication.  There is
+// no wait anywhere: the last block of a segment is found with one atomic
+// completion count per segment.
 #include "sz_internal.cuh"
 
 namespace sz {
@@ -41,62 +44,230 @@ __device__ __forceinline__ void count_v4(uint4 v, uint32_t col) {
     count_word(v.w, col);
 }
 
+// ---------------------------------------------------------- top-16 select
+// Shared state of one segment's select (256 threads).
+struct SelShared {
+    uint32_t cnt[256];
+    uint32_t warp[kWarps];
+    unsigned long long top;
+    uint32_t carry;
+    int valid;
+    int flag;
+    uint8_t cb[16];
+};
+
+// Codebook, escape count and range records of segment k, by the kThreads
+// threads of one block (every one of them must call it).  Thread t holds
+// exponent t: its rank is the number of exponents before it in (count
+// descending, exponent ascending); ranks 0..15 form the codebook and
+// e = n - (sum of their counts).  With a caller's codebook, that codebook is
+// used instead (repeated entries: invalid).  Then, for every range the
+// segment reaches, the escapes of the segment's piece in it = the piece's
+// length - its counts of the 16 codebook exponents; an exclusive scan over
+// the ranges places each piece.  Counts written by other blocks are read
+// from L2 (__ldcg): they were published before the completion count that
+// made this block the segment's last.
+__device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *codebook_in, SelShared &ss) {
+    const uint32_t tid = threadIdx.x;
+    const int lane = tid & 31, wid = tid >> 5;
+    const sz_segment seg = load_segment(a.batch, k);
+    const uint64_t n = seg.n_elems;
+    const uint32_t c = __ldcg(a.seg_hist + (size_t)k * 256 + tid);
+    ss.cnt[tid] = c;
+    __syncthreads();
+    if (codebook_in == nullptr) {
+        uint32_t rank = 0;
+#pragma unroll 8
+        for (uint32_t u = 0; u < 256; ++u) {
+            const uint32_t cu = ss.cnt[u];
+            rank += (cu > c) || (cu == c && u < tid);
+        }
+        if (rank < 16) ss.cb[rank] = (uint8_t)tid;
+    } else if (tid < 16) {
+        ss.cb[tid] = codebook_in[tid];
+    }
+    __syncthreads();
+    if (wid == 0) {
+        unsigned long long v = 0;
+        bool dup = false;
+        if (lane < 16) {
+            const uint32_t x = ss.cb[lane];
+            v = ss.cnt[x];
+            for (int j = 0; j < 16; ++j) dup |= (j != lane) && ss.cb[j] == x;
+        }
+#pragma unroll
+        for (int d = 8; d >= 1; d >>= 1) v += __shfl_down_sync(0xFFFFFFFFu, v, d);
+        const bool any_dup = __any_sync(0xFFFFFFFFu, dup) != 0;
+        if (lane == 0) {
+            ss.top = v;
+            ss.valid = (!any_dup && v <= n) ? 1 : 0;
+            ss.carry = 0;
+        }
+    }
+    __syncthreads();
+    const bool valid = ss.valid != 0;
+    const uint64_t e = valid ? n - ss.top : 0;
+    if (tid < 16) {
+        a.meta[k].codebook[tid] = ss.cb[tid];
+        if (a.codebooks_out) a.codebooks_out[(size_t)k * 16 + tid] = ss.cb[tid];
+    }
+    if (a.hist_out) a.hist_out[tid] = c;
+    if (tid == 0) {
+        a.meta[k].n_escapes = e;
+        a.meta[k].valid = valid ? 1u : 0u;
+        a.meta[k].pad = 0;
+    }
+    if (n == 0) return;
+
+    // ---- the segment's pieces: one per range it reaches
+    const uint64_t R = a.range_tiles;
+    const uint64_t t_first = seg.tile_begin;
+    const uint64_t t_last = t_first + segment_tiles(n, a.batch.page_elems) - 1;
+    const uint64_t b_first = t_first / R, b_last = t_last / R;
+    if (b_first == b_last) {  // inside one range: only a range-opening segment has a record
+        if (tid == 0 && t_first == b_first * R) {
+            a.rrec[b_first].first_off = 0;
+            a.rrec[b_first].first_cnt = (uint32_t)e;
+        }
+        return;
+    }
+    uint32_t cbq[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) cbq[q] = ss.cb[q];
+    for (uint64_t base = b_first; base <= b_last; base += kThreads) {
+        const uint64_t b = base + tid;
+        uint32_t cnt = 0;
+        bool opens = false;  // the piece opens its range (else it closes it)
+        if (b <= b_last) {
+            const uint64_t ps = umax64(t_first, b * R), pe = umin64(t_last + 1, (b + 1) * R);
+            opens = ps == b * R;
+            const uint32_t *H = a.rhist + (b * 2 + (opens ? 0 : 1)) * 256;
+            uint64_t in = 0;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) in += __ldcg(H + cbq[q]);
+            const TileRef r0 = resolve_tile(a.batch, seg, k, ps);
+            const TileRef r1 = resolve_tile(a.batch, seg, k, pe - 1);
+            const uint64_t len = r1.elem0 + r1.len - r0.elem0;
+            cnt = in <= len ? (uint32_t)(len - in) : 0u;
+        }
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        if (lane == 31) ss.warp[wid] = incl;
+        __syncthreads();
+        if (wid == 0) {
+            uint32_t w = lane < kWarps ? ss.warp[lane] : 0u;
+#pragma unroll
+            for (int d = 1; d < kWarps; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, d);
+                if (lane >= d) w += y;
+            }
+            if (lane < kWarps) ss.warp[lane] = w;  // inclusive over warps
+        }
+        __syncthreads();
+        const uint32_t carry = ss.carry;
+        const uint32_t excl = carry + (wid ? ss.warp[wid - 1] : 0u) + incl - cnt;
+        if (b <= b_last) {
+            RangeRec &rr = a.rrec[b];
+            if (opens) {
+                rr.first_off = excl;
+                rr.first_cnt = cnt;
+            } else {
+                rr.last_cnt = cnt;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) ss.carry = carry + ss.warp[kWarps - 1];
+        __syncthreads();
+    }
+}
+
+// Segments with no elements have no tiles, so no range completes them:
+// their codebook is exponents 0..15 (all counts zero) and e = 0.
+__device__ void empty_segments(const HistArgs &h) {
+    const SelectCtx &a = h.sel;
+    const uint32_t ns = a.batch.segs ? a.batch.n_segs : 1u;
+    for (uint32_t k = threadIdx.x; k < ns; k += blockDim.x) {
+        if (load_segment(a.batch, k).n_elems != 0) continue;
+        SegMeta &m = a.meta[k];
+        for (int q = 0; q < 16; ++q) {
+            m.codebook[q] = (uint8_t)q;
+            if (a.codebooks_out) a.codebooks_out[(size_t)k * 16 + q] = (uint8_t)q;
+        }
+        m.n_escapes = 0;
+        m.valid = 1;
+        m.pad = 0;
+    }
+    if (a.hist_out && a.batch.segs == nullptr && a.batch.single.n_elems == 0)
+        for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) a.hist_out[i] = 0;
+}
+
+// ------------------------------------------------------------- histogram
+// One block per range.  The tiles of a range are counted piece by piece (a
+// piece = the range's tiles of one segment); at the end of a piece its 256
+// counts are the difference of the column sums, added to the segment's
+// counts, and kept when the piece opens or closes the range.  The block
+// that completes a segment's tile count runs that segment's select.
 template <bool kBatched>
 __global__ void __launch_bounds__(kThreads) hist_kernel(const HistArgs a) {
     extern __shared__ __align__(128) uint32_t s_hist[];  // kHistWords
     __shared__ SegCache s_segc;
+    __shared__ SelShared s_sel;
     static_assert(kThreads == 256, "one thread per bin");
+    const Batch &batch = a.sel.batch;
 
     for (uint32_t i = threadIdx.x; i < kHistWords; i += kThreads) s_hist[i] = 0;
-    seg_cache_fill(s_segc, a.batch);  // ends with __syncthreads
+    seg_cache_fill(s_segc, batch);  // ends with __syncthreads
+    if (blockIdx.x == 0) empty_segments(a);
 
     const uint32_t tid = threadIdx.x;
     const uint32_t col = smem_u32(s_hist) + (tid & 31) * 4;
-    const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
-    const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
+    const uint64_t R = a.sel.range_tiles;
+    const uint64_t t_begin = (uint64_t)blockIdx.x * R;
+    const uint64_t t_end = umin64(t_begin + R, batch.n_tiles);
 
-    uint32_t prev = 0;     // column sum of bin `tid` at the last tile boundary
-    uint32_t seg_acc = 0;  // bin `tid` count of the current segment in this CTA
-    uint32_t cur = 0xFFFFFFFFu;
-    sz_segment seg{};
-    for (uint64_t t = t_begin; t < t_end; ++t) {
-        const uint32_t k = find_segment(s_segc, a.batch, t);
-        if (k != cur) {
-            if (cur != 0xFFFFFFFFu && seg_acc) atomicAdd(&a.seg_hist[(size_t)cur * 256 + tid], seg_acc);
-            seg_acc = 0;
-            cur = k;
-            seg = load_segment(a.batch, k);
-        }
-        const TileRef r = resolve_tile(a.batch, seg, k, t);
-        const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
-        const bool ok = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-        if (!ok && tid == 0) set_status(a.status ? a.status + k : nullptr, SZ_ERR_ALIGN);
-        for (uint32_t sub = 0; ok && sub < r.n_subs; ++sub) {
-            const uint16_t *p = src + sub * kSub;
-            const uint32_t len = umin32(kSub, r.len - sub * kSub);
-            // bulk prefetch of the next sub-tile into L2 while this one is counted
-            if (tid == 0 && sub + 1 < r.n_subs) {
-                const uint32_t next = (umin32(kSub, r.len - (sub + 1) * kSub) * 2u) & ~15u;
-                if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + kSub), "r"(next) : "memory");
-            }
-            if (len == kSub) {
-                uint4 v[2 * kChunks];
-#pragma unroll
-                for (int c = 0; c < kChunks; ++c) {
-                    const uint16_t *q = p + (c * kThreads + tid) * kChunk;
-                    v[2 * c] = ld_stream_v4(q);
-                    v[2 * c + 1] = ld_stream_v4(q + 8);
+    uint32_t prev = 0;  // column sum of bin `tid` at the last piece boundary
+    uint64_t t = t_begin;
+    while (t < t_end) {
+        const uint32_t k = find_segment(s_segc, batch, t);
+        const sz_segment seg = load_segment(batch, k);
+        const uint64_t seg_tiles = segment_tiles(seg.n_elems, batch.page_elems);
+        const uint64_t ps = t, pe = umin64(seg.tile_begin + seg_tiles, t_end);  // the piece [ps, pe)
+        for (; t < pe; ++t) {
+            const TileRef r = resolve_tile(batch, seg, k, t);
+            const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
+            const bool ok = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+            if (!ok && tid == 0) set_status(a.status ? a.status + k : nullptr, SZ_ERR_ALIGN);
+            for (uint32_t sub = 0; ok && sub < r.n_subs; ++sub) {
+                const uint16_t *p = src + sub * kSub;
+                const uint32_t len = umin32(kSub, r.len - sub * kSub);
+                // bulk prefetch of the next sub-tile into L2 while this one is counted
+                if (tid == 0 && sub + 1 < r.n_subs) {
+                    const uint32_t next = (umin32(kSub, r.len - (sub + 1) * kSub) * 2u) & ~15u;
+                    if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + kSub), "r"(next) : "memory");
                 }
+                if (len == kSub) {
+                    uint4 v[2 * kChunks];
 #pragma unroll
-                for (int i = 0; i < 2 * kChunks; ++i) count_v4(v[i], col);
-            } else {
-                for (int c = 0; c < kChunks; ++c) {
-                    const uint32_t off = (c * kThreads + tid) * kChunk;
-                    if (off + kChunk <= len) {
-                        count_v4(ld_stream_v4(p + off), col);
-                        count_v4(ld_stream_v4(p + off + 8), col);
-                    } else {
-                        for (uint32_t j = off; j < len; ++j) red_add1(col + (p[j] & 0x7F80u));
+                    for (int c = 0; c < kChunks; ++c) {
+                        const uint16_t *q = p + (c * kThreads + tid) * kChunk;
+                        v[2 * c] = ld_stream_v4(q);
+                        v[2 * c + 1] = ld_stream_v4(q + 8);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2 * kChunks; ++i) count_v4(v[i], col);
+                } else {
+                    for (int c = 0; c < kChunks; ++c) {
+                        const uint32_t off = (c * kThreads + tid) * kChunk;
+                        if (off + kChunk <= len) {
+                            count_v4(ld_stream_v4(p + off), col);
+                            count_v4(ld_stream_v4(p + off + 8), col);
+                        } else {
+                            for (uint32_t j = off; j < len; ++j) red_add1(col + (p[j] & 0x7F80u));
+                        }
                     }
                 }
             }
@@ -107,132 +278,46 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const HistArgs a) {
         uint32_t sum = 0;
 #pragma unroll 8
         for (uint32_t i = 0; i < 32; ++i) sum += s_hist[tid * 32 + ((i + tid) & 31)];
-        const uint32_t cnt = sum - prev;
+        const uint32_t acc = sum - prev;
         prev = sum;
-        a.tile_hist[t * 256 + tid] = cnt;
-        seg_acc += cnt;
-        __syncthreads();  // folds done before the next tile's counts land
+        if (ps == t_begin) a.rhist[(blockIdx.x * 2ull) * 256 + tid] = acc;
+        else if (pe == t_end) a.rhist[(blockIdx.x * 2ull + 1) * 256 + tid] = acc;
+        if (acc) atomicAdd(&a.seg_hist[(size_t)k * 256 + tid], acc);
+        __threadfence();
+        __syncthreads();  // folds done before the next piece's counts land
+        if (tid == 0) {
+            const uint32_t add = (uint32_t)(pe - ps);
+            s_sel.flag = atomicAdd(&a.seg_done[k], add) + add == (uint32_t)seg_tiles;
+        }
+        __syncthreads();
+        if (s_sel.flag) {  // every other piece of segment k is counted and published
+            __threadfence();
+            select_segment(a.sel, k, nullptr, s_sel);
+        }
     }
-    if (cur != 0xFFFFFFFFu && seg_acc) atomicAdd(&a.seg_hist[(size_t)cur * 256 + tid], seg_acc);
 }
 
-// ---------------------------------------------------------- top-16 select
-// One block per segment.  Threads 0..255: the rank of exponent t is the
-// number of exponents before it in (count desc, exponent asc); ranks 0..15
-// form the codebook and e = n - (sum of their counts).  With a caller's
-// codebook, that codebook is used instead (repeated entries: invalid).
-// Then all threads: escapes of tile j = its length - (its counts of the 16
-// codebook exponents), and an exclusive scan over the segment's tiles gives
-// every tile the index of its first escape record.
-constexpr int kSelThreads = 1024;
-
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelectArgs a) {
-    __shared__ uint32_t s_cnt[256];
-    __shared__ uint8_t s_cb[16];
-    __shared__ unsigned long long s_sum;
-    __shared__ int s_valid;
-    __shared__ uint32_t s_warp[kSelThreads / 32];
-    __shared__ uint32_t s_carry;
-    const uint32_t k = blockIdx.x;
-    const uint32_t t = threadIdx.x;
-    const sz_segment seg = load_segment(a.batch, k);
-    const uint64_t n = seg.n_elems;
-    if (t < 256) s_cnt[t] = a.seg_hist[(size_t)k * 256 + t];
-    if (t == 0) {
-        s_sum = 0;
-        s_valid = 1;
-        s_carry = 0;
+// Caller codebook for a single tensor: the select again with that codebook,
+// unless it is the one the workspace already holds.  Also resets the
+// encode's status and size words.
+__global__ void __launch_bounds__(kThreads) reselect_kernel(const ReselectArgs a) {
+    __shared__ SelShared s_sel;
+    __shared__ int s_same;
+    if (threadIdx.x == 0) {
+        *a.status = SZ_OK;
+        *a.out_bytes = 0;
+        s_same = a.sel.meta[0].valid != 0;
     }
     __syncthreads();
-    if (a.codebook_in == nullptr) {
-        if (t < 256) {
-            const uint32_t c = s_cnt[t];
-            uint32_t rank = 0;
-#pragma unroll 8
-            for (uint32_t u = 0; u < 256; ++u) {
-                const uint32_t cu = s_cnt[u];
-                rank += (cu > c) || (cu == c && u < t);
-            }
-            if (rank < 16) {
-                s_cb[rank] = (uint8_t)t;
-                atomicAdd(&s_sum, (unsigned long long)c);
-            }
-        }
-    } else {
-        if (t < 16) s_cb[t] = a.codebook_in[t];
-        __syncthreads();
-        if (t < 16) {
-            for (int j = 0; j < 16; ++j)
-                if (j != (int)t && s_cb[j] == s_cb[t]) s_valid = 0;
-            atomicAdd(&s_sum, (unsigned long long)s_cnt[s_cb[t]]);
-        }
-    }
+    if (threadIdx.x < 16 && a.sel.meta[0].codebook[threadIdx.x] != a.codebook_in[threadIdx.x]) s_same = 0;
     __syncthreads();
-    const uint64_t top = s_sum;
-    const bool valid = s_valid != 0 && top <= n;
-    const uint64_t e = valid ? n - top : 0;
-    if (t < 16) {
-        a.meta[k].codebook[t] = s_cb[t];
-        if (a.codebooks_out) a.codebooks_out[(size_t)k * 16 + t] = s_cb[t];
-    }
-    if (a.hist_out && t < 256) a.hist_out[t] = s_cnt[t];
-    if (t == 0) {
-        a.meta[k].n_escapes = e;
-        a.meta[k].valid = valid ? 1u : 0u;
-        a.meta[k].pad = 0;
-    }
-
-    // per-tile first escape index
-    uint32_t cb[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) cb[q] = s_cb[q];
-    const uint32_t tiles = (uint32_t)segment_tiles(n, a.batch.page_elems);
-    const int lane = t & 31, wid = t >> 5;
-    for (uint32_t base = 0; base < tiles; base += kSelThreads) {
-        const uint32_t j = base + t;
-        uint32_t cnt = 0;
-        if (j < tiles) {
-            const uint32_t *h = a.tile_hist + (size_t)(seg.tile_begin + j) * 256;
-            uint32_t in_cb = 0;
-#pragma unroll
-            for (int q = 0; q < 16; ++q) in_cb += h[cb[q]];
-            const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j);
-            cnt = r.len - in_cb;
-        }
-        uint32_t incl = cnt;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += y;
-        }
-        if (lane == 31) s_warp[wid] = incl;
-        __syncthreads();
-        if (wid == 0) {
-            uint32_t w = s_warp[lane];
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, d);
-                if (lane >= d) w += y;
-            }
-            s_warp[lane] = w;  // inclusive over warps
-        }
-        __syncthreads();
-        const uint32_t carry = s_carry;
-        const uint32_t excl = carry + (wid ? s_warp[wid - 1] : 0u) + incl - cnt;
-        if (j < tiles) a.tile_off[seg.tile_begin + j] = excl;
-        __syncthreads();
-        if (t == kSelThreads - 1) s_carry = carry + s_warp[kSelThreads / 32 - 1];
-        __syncthreads();
-    }
+    if (s_same) return;
+    select_segment(a.sel, 0, a.codebook_in, s_sel);
 }
 
 // ------------------------------------------------------------ launchers
-cudaError_t launch_hist(const HistArgs &a0, bool batched, int grid, cudaStream_t s) {
-    HistArgs a = a0;
-    if (a.batch.n_tiles == 0) return cudaSuccess;
-    grid = (int)umin64((uint64_t)grid, a.batch.n_tiles);
-    a.tiles_per_cta = div_up(a.batch.n_tiles, (uint64_t)grid);
-    grid = (int)div_up(a.batch.n_tiles, a.tiles_per_cta);
+cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s) {
+    const int grid = (int)umax64(1, div_up(a.sel.batch.n_tiles, a.sel.range_tiles));
     const size_t smem = kHistWords * sizeof(uint32_t);
     if (batched)
         hist_kernel<true><<<grid, kThreads, smem, s>>>(a);
@@ -241,10 +326,8 @@ cudaError_t launch_hist(const HistArgs &a0, bool batched, int grid, cudaStream_t
     return cudaGetLastError();
 }
 
-cudaError_t launch_select(const SelectArgs &a, cudaStream_t s) {
-    const uint32_t segs = a.batch.segs ? a.batch.n_segs : 1u;
-    if (segs == 0) return cudaSuccess;
-    select_kernel<<<segs, kSelThreads, 0, s>>>(a);
+cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s) {
+    reselect_kernel<<<1, kThreads, 0, s>>>(a);
     return cudaGetLastError();
 }
 

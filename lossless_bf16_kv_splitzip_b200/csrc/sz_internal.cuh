@@ -19,8 +19,12 @@ namespace sz {
 // each.  Chunk c of thread t covers sub-tile elements [(c*256 + t)*16, +16),
 // so a warp-wide 16-byte access is 512 contiguous bytes.
 // Tile: 4 sub-tiles (65,536 elements) inside one page; the unit of work
-// scheduling and of the per-tile exponent histograms that give every tile
-// its first escape index before the encode runs.
+// scheduling.
+// Range: a run of consecutive tiles of the batch, one CTA's share in both
+// the histogram and the encode kernel (the two use the same partition).  A
+// range cut by segment boundaries holds several pieces; the histogram kernel
+// keeps the exponent counts of its first and last piece, which is all the
+// encode needs to place each CTA's escape records.
 constexpr int kThreads = 256;                 // consumer threads
 constexpr int kWarps = kThreads / 32;
 constexpr int kPipeThreads = kThreads + 32;   // + one producer warp
@@ -31,6 +35,8 @@ constexpr uint32_t kSubsPerTile = 4;
 constexpr uint32_t kTile = kSub * kSubsPerTile;         // 65,536 elements
 constexpr uint64_t kHeader = 48;
 constexpr uint32_t kMaxSmemSegs = 256;  // segment starts cached in shared memory
+constexpr uint64_t kMaxRanges = 1024;   // ranges of one call (workspace bound)
+constexpr uint64_t kRangesPerSM = 3;    // encode CTAs resident per SM
 
 // Per-segment record kept in the workspace between kernels (32 bytes).
 struct SegMeta {
@@ -47,6 +53,35 @@ __host__ __device__ inline uint64_t container_size(uint64_t n, uint64_t e) {
     return kHeader + n + (n + 1) / 2 + 5 * e;
 }
 __host__ __device__ inline uint64_t div_up(uint64_t a, uint64_t b) { return (a + b - 1) / b; }
+
+// The range partition of n_tiles tiles: `tiles` tiles per range, `count`
+// ranges (the last may be shorter); at most kMaxRanges ranges.
+struct RangePlan {
+    uint64_t tiles;
+    uint64_t count;
+};
+__host__ __device__ inline RangePlan plan_ranges(uint64_t n_tiles, uint64_t sms) {
+    RangePlan p;
+    uint64_t want = sms * kRangesPerSM;
+    if (want > kMaxRanges) want = kMaxRanges;
+    if (want == 0) want = 1;
+    p.tiles = n_tiles ? div_up(n_tiles, want) : 1;
+    p.count = div_up(n_tiles, p.tiles);
+    return p;
+}
+
+// Escape bookkeeping of one range, written by the select of the segments
+// that own its first and last pieces (u32: escapes < n < 2^32).
+//   first_off  escapes of the first piece's segment before the range
+//   first_cnt  escapes in the first piece
+//   last_cnt   escapes in the last piece, when it is another piece whose
+//              segment continues past the range
+struct RangeRec {
+    uint32_t first_off;
+    uint32_t first_cnt;
+    uint32_t last_cnt;
+    uint32_t pad;
+};
 __host__ __device__ inline uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
 __host__ __device__ inline uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
 __host__ __device__ inline uint32_t umin32(uint32_t a, uint32_t b) { return a < b ? a : b; }
@@ -244,25 +279,34 @@ __device__ __forceinline__ void tma_load_1d(void *smem_dst, const void *gmem_src
 }
 
 // ------------------------------------------------------- launch arguments
-struct HistArgs {
+// What the select of a segment reads and writes.
+struct SelectCtx {
     Batch batch;
+    const uint32_t *seg_hist;  // [n_segs][256]
+    const uint32_t *rhist;     // [ranges][2][256]: first, last piece of each range
+    SegMeta *meta;             // [n_segs]
+    RangeRec *rrec;            // [ranges]
+    uint64_t range_tiles;      // tiles per range
+    uint8_t *codebooks_out;    // optional [n_segs][16]
+    uint32_t *hist_out;        // optional [256] (single only)
+};
+
+struct HistArgs {
+    SelectCtx sel;
     const uint16_t *const *pages;  // batched: page pointers
     const uint16_t *base;          // single-tensor input
-    uint32_t *seg_hist;            // [n_segs][256]
-    uint32_t *tile_hist;           // [n_tiles][256]
-    uint64_t tiles_per_cta;
+    uint32_t *seg_hist;            // [n_segs][256], zero on entry
+    uint32_t *seg_done;            // [n_segs] tiles counted so far, zero on entry
+    uint32_t *rhist;               // [ranges][2][256]
     int32_t *status;               // [n_segs] or nullptr
 };
 
-struct SelectArgs {
-    Batch batch;
-    const uint32_t *seg_hist;    // [n_segs][256]
-    const uint32_t *tile_hist;   // [n_tiles][256]
-    SegMeta *meta;               // [n_segs]
-    uint32_t *tile_off;          // [n_tiles] first escape index of each tile
-    const uint8_t *codebook_in;  // single-tensor encode with a caller codebook, else nullptr
-    uint8_t *codebooks_out;      // optional [n_segs][16]
-    uint32_t *hist_out;          // optional [256] (single only)
+// Select with a caller codebook (single tensor), ahead of the encode.
+struct ReselectArgs {
+    SelectCtx sel;
+    const uint8_t *codebook_in;
+    int32_t *status;      // set to SZ_OK here
+    uint64_t *out_bytes;  // set to 0 here
 };
 
 struct EncodeArgs {
@@ -274,8 +318,8 @@ struct EncodeArgs {
     uint64_t *out_bytes;      // [n_segs]
     int32_t *status;          // [n_segs]
     const SegMeta *meta;      // [n_segs]
-    const uint32_t *tile_off; // [n_tiles]
-    uint64_t tiles_per_cta;
+    const RangeRec *rrec;     // [ranges]
+    uint64_t range_tiles;     // tiles per range = per CTA
     uint64_t wait_limit_ns;
     uint32_t debug_flags;
 };

@@ -14,28 +14,29 @@
 #include "sz_internal.cuh"
 
 namespace sz {
-cudaError_t launch_hist(const HistArgs &a, bool batched, int grid, cudaStream_t s);
-cudaError_t launch_select(const SelectArgs &a, cudaStream_t s);
-cudaError_t launch_encode(const EncodeArgs &a, bool batched, int grid, cudaStream_t s);
-int hist_blocks_per_sm();
-int encode_blocks_per_sm();
+cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s);
+cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
 }  // namespace sz
 
 using namespace sz;
 
 namespace {
 
-// Scratch layout for one tensor of at most SZ_STATIC_MAX_ELEMS elements:
+// Scratch layout for one tensor of at most SZ_STATIC_MAX_ELEMS elements
+// (4096 tiles, so at most kMaxRanges = 1024 ranges):
 //   [0, 1024)      exponent counts of the tensor, u32[256]
-//   [1024, 1056)   SegMeta (codebook, escape count)
-//   [1280, ...)    exponent counts of every 65,536-element tile, u32[T][256]
-//   then           first escape index of every tile, u32[T]
+//   [1024, 1028)   tiles counted so far
+//   [1280, 1312)   SegMeta (codebook, escape count)
+//   [1536, ...)    counts of each range's first and last piece, u32[1024][2][256]
+//   then           escape placement of each range, RangeRec[1024]
 constexpr uint64_t kMaxTiles = (SZ_STATIC_MAX_ELEMS + kTile - 1) / kTile;
+constexpr uint64_t kRanges = kMaxTiles < kMaxRanges ? kMaxTiles : kMaxRanges;
 constexpr uint64_t kOffSegHist = 0;
-constexpr uint64_t kOffMeta = 1024;
-constexpr uint64_t kOffTileHist = 1280;
-constexpr uint64_t kOffTileOff = kOffTileHist + 1024 * kMaxTiles;
-constexpr uint64_t kStaticScratchBytes = kOffTileOff + 4 * kMaxTiles;
+constexpr uint64_t kOffSegDone = 1024;
+constexpr uint64_t kOffMeta = 1280;
+constexpr uint64_t kOffRhist = 1536;
+constexpr uint64_t kOffRrec = kOffRhist + 2048 * kRanges;
+constexpr uint64_t kStaticScratchBytes = kOffRrec + sizeof(RangeRec) * kRanges;
 static_assert(kStaticScratchBytes == SZ_STATIC_SCRATCH_BYTES, "header and layout agree");
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
@@ -43,7 +44,7 @@ static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 struct StaticDevice {
     bool ready = false;
     uint8_t *scratch = nullptr;  // device address of g_static_scratch on that device
-    int sms = 0, hist_occ = 1, enc_occ = 1;
+    int sms = 0;
 };
 std::mutex g_static_mu;
 StaticDevice g_static_dev[64];
@@ -60,8 +61,6 @@ bool static_device(StaticDevice &out) {
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return false;
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
         d.scratch = static_cast<uint8_t *>(p);
-        d.hist_occ = hist_blocks_per_sm();
-        d.enc_occ = encode_blocks_per_sm();
         d.ready = true;
     }
     out = d;
@@ -83,10 +82,10 @@ extern "C" sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = dev.scratch;
 
-    // The array keeps the previous call's contents: the tensor counts are
-    // accumulated with atomics and must start at zero; everything else is
-    // overwritten before it is read.
-    if (cudaMemsetAsync(ws + kOffSegHist, 0, 1024, s) != cudaSuccess) return SZ_ERR_CUDA;
+    // The array keeps the previous call's contents: the tensor counts and
+    // the tile count are accumulated with atomics and must start at zero;
+    // everything else is overwritten before it is read.
+    if (cudaMemsetAsync(ws + kOffSegHist, 0, 1028, s) != cudaSuccess) return SZ_ERR_CUDA;
     if (cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s) != cudaSuccess) return SZ_ERR_CUDA;
     if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), s) != cudaSuccess) return SZ_ERR_CUDA;
 
@@ -99,20 +98,18 @@ extern "C" sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t 
     b.single.n_elems = n;
 
     HistArgs h{};
-    h.batch = b;
+    h.sel.batch = b;
+    h.sel.seg_hist = reinterpret_cast<uint32_t *>(ws + kOffSegHist);
+    h.sel.rhist = reinterpret_cast<uint32_t *>(ws + kOffRhist);
+    h.sel.meta = reinterpret_cast<SegMeta *>(ws + kOffMeta);
+    h.sel.rrec = reinterpret_cast<RangeRec *>(ws + kOffRrec);
+    h.sel.range_tiles = plan_ranges(b.n_tiles, (uint64_t)dev.sms).tiles;
+    h.sel.codebooks_out = d_codebook16_or_null;
     h.base = d_in;
     h.seg_hist = reinterpret_cast<uint32_t *>(ws + kOffSegHist);
-    h.tile_hist = reinterpret_cast<uint32_t *>(ws + kOffTileHist);
-    if (launch_hist(h, false, dev.sms * dev.hist_occ, s) != cudaSuccess) return SZ_ERR_CUDA;
-
-    SelectArgs sa{};
-    sa.batch = b;
-    sa.seg_hist = h.seg_hist;
-    sa.tile_hist = h.tile_hist;
-    sa.meta = reinterpret_cast<SegMeta *>(ws + kOffMeta);
-    sa.tile_off = reinterpret_cast<uint32_t *>(ws + kOffTileOff);
-    sa.codebooks_out = d_codebook16_or_null;
-    if (launch_select(sa, s) != cudaSuccess) return SZ_ERR_CUDA;
+    h.seg_done = reinterpret_cast<uint32_t *>(ws + kOffSegDone);
+    h.rhist = reinterpret_cast<uint32_t *>(ws + kOffRhist);
+    if (launch_hist(h, false, s) != cudaSuccess) return SZ_ERR_CUDA;
 
     EncodeArgs a{};
     a.batch = b;
@@ -121,9 +118,10 @@ extern "C" sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t 
     a.out_cap = out_cap;
     a.out_bytes = d_out_bytes;
     a.status = d_status;
-    a.meta = sa.meta;
-    a.tile_off = sa.tile_off;
+    a.meta = h.sel.meta;
+    a.rrec = h.sel.rrec;
+    a.range_tiles = h.sel.range_tiles;
     a.wait_limit_ns = 1000000000ull;
     a.debug_flags = 0;
-    return launch_encode(a, false, dev.sms * dev.enc_occ, s) == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+    return launch_encode(a, false, s) == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
 }

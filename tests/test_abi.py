@@ -34,8 +34,11 @@ def test_plan_worst_case_bound(n):
     cap, ws = sz.sz_plan(n)
     assert cap == 48 + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
     tiles = -(-n // 65536)
-    # segment histogram + record, tile histograms, tile offsets, sub-tile starts
-    assert ws >= 1024 + 32 + 1024 * tiles + 4 * tiles + 4 * (4 * tiles + 1)
+    ranges = min(tiles, 1024)
+    # segment histogram, tile count and record; the first- and last-piece
+    # histograms and the record of every range; sub-tile escape starts
+    need = 1024 + 4 + 32 + 2048 * ranges + 16 * ranges + 4 * (4 * tiles + 1)
+    assert need <= ws <= need + 6 * 256
     assert ws % 256 == 0
 
 

@@ -2,8 +2,9 @@
 
 Integer/byte work, so the bar is bit-exactness: every byte of every
 container and every bit of every decoded value must equal the oracle's on
-the same seeded inputs.  Covered: ragged sizes around the tile (16384) and
-chunk (16) boundaries, the exhaustive 65,536-pattern tensor, the golden
+the same seeded inputs.  Covered: ragged sizes around the tile (65536),
+sub-tile (16384) and chunk (16) boundaries, single streams at the sizes of
+the bench's latency sweep, the exhaustive 65,536-pattern tensor, the golden
 containers, every workload at full size in the batched launch the bench
 times, scattered paged KV, incompressible input, a caller-chosen codebook,
 cross decoding, determinism, corrupt containers and the bounded-wait
@@ -119,6 +120,33 @@ def test_single_exponent_and_seventeen_equal():
     assert_parity(x)
     x = ((np.repeat(np.arange(100, 117), 2000).astype(np.uint16) << 7) | np.uint16(3))
     assert_parity(np.random.default_rng(4).permutation(x))
+
+
+_SWEEP_SRC = {}
+
+
+def sweep_prefix(nbytes):
+    """The first nbytes of the 32K-token workload's buffer, as the bench's
+    latency sweep codes them: one stream, one codebook."""
+    n = nbytes // 2
+    nt = kvgen.HEADS * 32768 * kvgen.HEAD_DIM
+    parts = []
+    for k in range(-(-n // nt)):
+        if k not in _SWEEP_SRC:
+            _SWEEP_SRC[k] = kvgen.contiguous_tensor(2, k // 2, k % 2)
+        parts.append(_SWEEP_SRC[k])
+    return np.concatenate(parts)[:n] if len(parts) > 1 else parts[0][:n]
+
+
+@pytest.mark.parametrize("nbytes", [1 << 16, 1 << 18, 1 << 20, 1 << 22, 1 << 24, 1 << 26])
+def test_sweep_prefix_single_stream(nbytes):
+    assert_parity(sweep_prefix(nbytes))
+
+
+@pytest.mark.slow
+def test_sweep_prefix_spanning_tensors():
+    # 256 MiB: layer 0-1 K and V as one stream under one codebook
+    assert_parity(sweep_prefix(1 << 28))
 
 
 def test_cross_decode():
@@ -260,8 +288,8 @@ def test_odd_tail_nibble_rejected():
 
 
 # -------------------------------------------------------- bounded waits
-def test_lookback_wait_times_out_cleanly():
-    """Tiles never publish their counts, so every lookback wait runs out:
+def test_stage_wait_times_out_cleanly():
+    """The copy thread issues no bulk copy, so every stage wait runs out:
     the kernel reports SZ_ERR_DEVICE_TIMEOUT and returns; the context stays
     usable and the next normal call is bit-exact."""
     x = kvgen.mixed_small(4 * 16384, seed=31)
@@ -276,6 +304,25 @@ def test_lookback_wait_times_out_cleanly():
         sz.sz_debug_set_flags(0)
         sz.sz_set_wait_limit_ns(1_000_000_000)
     assert gpu_encode(x) == oracle.encode(x)
+
+
+def test_decode_stage_wait_times_out_cleanly():
+    x = kvgen.mixed_small(4 * 16384 + 5, seed=32)
+    blob = oracle.encode(x)
+    c = torch.from_numpy(np.frombuffer(blob, np.uint8).copy()).to(DEV)
+    try:
+        sz.sz_set_wait_limit_ns(2_000_000)
+        sz.sz_debug_set_flags(1)
+        _, status = sz.decode(c, x.size)
+        torch.cuda.synchronize()
+        assert int(status.item()) == sz.SZ_ERR_DEVICE_TIMEOUT
+    finally:
+        sz.sz_debug_set_flags(0)
+        sz.sz_set_wait_limit_ns(1_000_000_000)
+    out, status = sz.decode(c, x.size)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), x)
 
 
 # ----------------------------------------------------- batched / paged
@@ -417,3 +464,68 @@ def test_pages_with_partial_last_page(page):
             seg = x[p: p + page]
             assert np.array_equal(got[i, : seg.size], seg)
             i += 1
+
+
+@pytest.mark.parametrize("dst_page", [8192, 32768, 24576])
+def test_decode_into_other_page_size(dst_page):
+    """Requests encoded from 16-token pages are decoded straight into a pool
+    of another page size under another page table; a request whose length
+    is not a multiple of the new page size ends in a partial page.  The
+    container of a segment does not depend on paging, and a plan places it
+    at an offset that depends only on the segment lengths."""
+    b = kvgen.paged_batch(n_requests=10, min_tokens=16, max_tokens=900, pool_pages=4096)
+    lens = [int(l) * kvgen.HEADS * kvgen.HEAD_DIM for l in b.lengths]
+    src = sz.BatchPlan(lens, kvgen.PAGE_ELEMS, device=DEV)
+    pool = torch.zeros((b.pool_pages, kvgen.PAGE_ELEMS), dtype=torch.int16, device=DEV)
+    src_slots = np.concatenate(b.page_table)
+    pool[torch.from_numpy(src_slots).to(DEV)] = torch.from_numpy(np.concatenate(b.pages).view(np.int16)).to(DEV)
+    src.encode(torch.from_numpy(src_slots * (2 * kvgen.PAGE_ELEMS) + pool.data_ptr()).to(DEV))
+    dst = sz.BatchPlan(lens, dst_page, device=DEV)
+    assert np.array_equal(dst.out_offset, src.out_offset)
+    dst_pool = torch.zeros((dst.total_pages + 7, dst_page), dtype=torch.int16, device=DEV)
+    slots = np.random.default_rng(77).permutation(dst.total_pages + 7)[: dst.total_pages]
+    dst.decode(torch.from_numpy(slots * (2 * dst_page) + dst_pool.data_ptr()).to(DEV), container=src.container)
+    torch.cuda.synchronize()
+    assert src.enc_status.abs().sum().item() == 0 and dst.dec_status.abs().sum().item() == 0
+    got = dst_pool.cpu().numpy().view(np.uint16)
+    for r in range(b.n_requests):
+        x = b.request_stream(r)
+        pages = slots[int(dst.page_begin[r]): int(dst.page_begin[r]) + -(-x.size // dst_page)]
+        flat = got[pages].reshape(-1)[: x.size]
+        assert np.array_equal(flat, x), "request %d" % r
+    check_batch_against_oracle(src, [b.request_stream(r) for r in range(b.n_requests)])
+
+
+@pytest.mark.parametrize("page,seed", [(64, 1), (64, 2), (192, 3)])
+def test_batched_small_pages_cut_ranges_everywhere(page, seed):
+    """Hundreds of segments over thousands of small pages (one tile per
+    page), so every CTA's range of tiles is cut by segment boundaries at
+    every position: segments opening, closing or inside a range, spanning
+    many ranges, empty ones, and more segments than the shared-memory
+    segment cache holds."""
+    rng = np.random.default_rng(seed)
+    lens = [int(v) for v in rng.integers(0, 3000, size=300)]
+    lens[5] = 0
+    lens[17] = page
+    lens[18] = 5 * page
+    streams = [kvgen.mixed_small(n, seed=1000 * seed + i) for i, n in enumerate(lens)]
+    plan = sz.BatchPlan(lens, page, device=DEV)
+    pages_src = []
+    for x in streams:
+        for p in range(0, x.size, page):
+            chunk = np.zeros(page, np.uint16)
+            seg = x[p: p + page]
+            chunk[: seg.size] = seg
+            pages_src.append(chunk)
+    assert len(pages_src) == plan.total_pages and plan.n_tiles == plan.total_pages
+    pool = torch.from_numpy(np.stack(pages_src).view(np.int16)).to(DEV)
+    perm = rng.permutation(len(pages_src))
+    pool_perm = pool[torch.from_numpy(perm).to(DEV)].contiguous()
+    ptrs = torch.from_numpy(np.argsort(perm) * (2 * page) + pool_perm.data_ptr()).to(DEV)
+    plan.encode(ptrs)
+    out = torch.zeros_like(pool)
+    plan.decode(torch.from_numpy(np.arange(len(pages_src)) * (2 * page) + out.data_ptr()).to(DEV))
+    torch.cuda.synchronize()
+    assert plan.enc_status.abs().sum().item() == 0 and plan.dec_status.abs().sum().item() == 0
+    check_batch_against_oracle(plan, streams)
+    assert torch.equal(out, pool)
