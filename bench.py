@@ -511,7 +511,7 @@ def main():
             "decode_roofline_frac": roof["decode"]["frac"],
             "ratio": round(U / comp, 5), "escape_frac": round(esc / (S * n), 6),
             "roofline": roofline, "roofline_phases": roof,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * args.steps,  # hist, encode, esc_index, decode
             "clocks": clock_info, "parity": parity,
         }
         print(json.dumps(line), flush=True)
