@@ -247,6 +247,67 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
                             uint64_t page_elems, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
                             void *stream);
 
+/* ------------------------------------------- one pass, caller's codebook(s) */
+/*
+ * Encoding with a codebook chosen beforehand -- one kept from an earlier
+ * request or chunk, or shared across layers -- needs no histogram pass: the
+ * input is read once.  The explainer's method picks each tensor's own top
+ * 16 (section 3); a codebook that is not the tensor's own stays lossless but
+ * may leave more escapes.  The container is byte for byte the one the
+ * two-call path (sz_histogram_codebook + sz_encode) writes with the same
+ * codebook.
+ *
+ * Two kernels: the encode writes the sign+mantissa and code streams in place
+ * and parks each 65,536-element tile's escape records (up to 4,096 per tile,
+ * 6.25 %) in the workspace; a placement kernel then counts each segment's
+ * escapes, writes the header and the size, and moves the records into place
+ * (a tile with more than 4,096 escapes has its input read again, by a third
+ * kernel that spreads such tiles over the GPU).
+ *
+ * sz_plan_one_pass -- worst-case container (every element an escape:
+ * 48 + n + ceil(n/2) + 5n) and workspace bytes (16,420 bytes per tile,
+ * about 1/8 of the input's bytes, plus 16 bytes per range).  Host only.
+ */
+sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes);
+
+/*
+ * sz_encode_one_pass -- the container of d_in[0..n) with d_codebook16.
+ *   d_codebook16    16 distinct exponents (device memory); repeats give
+ *                   SZ_ERR_INVALID in *d_status
+ *   d_out, out_cap  container buffer, 16-byte aligned; out_cap must be at
+ *                   least 48 + n + ceil(n/2) (host check); the device checks
+ *                   the exact size (SZ_ERR_CAPACITY, *d_out_bytes = 0)
+ *   d_out_bytes, d_status  out, as for sz_encode (both set first)
+ *   d_ws, ws_bytes  workspace of sz_plan_one_pass's size, 16-byte aligned
+ */
+sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
+                             uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
+                             uint64_t ws_bytes, void *stream);
+
+/*
+ * sz_workspace_one_pass_batched -- workspace bytes of
+ * sz_encode_one_pass_batched for a batch of n_tiles tiles (from
+ * sz_plan_batched).  Host only.
+ */
+sz_status sz_workspace_one_pass_batched(uint32_t n_segs, uint64_t n_tiles, uint64_t *workspace_bytes);
+
+/*
+ * sz_encode_one_pass_batched -- every segment's container with its own
+ * caller codebook, in one read of the input.
+ *   d_codebooks     uint8[n_segs][16] device array (row k: segment k)
+ *   d_segs, n_tiles, d_pages, page_elems, d_out, out_cap  as for
+ *                   sz_encode_batched; a plan's container slots hold any
+ *                   codebook's container up to 48 + n + ceil(n/2) + 5(n -
+ *                   ceil(n/16)) bytes, more escapes than that give
+ *                   SZ_ERR_CAPACITY
+ *   d_out_bytes, d_status  out: uint64[n_segs], int32[n_segs] (set first)
+ */
+sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                                     const uint16_t *const *d_pages, uint64_t page_elems,
+                                     const uint8_t *d_codebooks, uint8_t *d_out, uint64_t out_cap,
+                                     uint64_t *d_out_bytes, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
+                                     void *stream);
+
 /* ------------------------------------------------------- no-allocation path */
 /*
  * sz_encode_static -- the whole compression of one tensor (histogram,

@@ -72,6 +72,10 @@ def lib():
             "sz_encode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, vp, u64, vp],
             "sz_decode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, u64, vp],
             "sz_encode_static": [vp, u64, vp, u64, vp, vp, vp, vp],
+            "sz_plan_one_pass": [u64, pu64, pu64],
+            "sz_encode_one_pass": [vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
+            "sz_workspace_one_pass_batched": [u32, u64, pu64],
+            "sz_encode_one_pass_batched": [u32, vp, u64, vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
             "sz_set_wait_limit_ns": [u64],
             "sz_debug_set_flags": [u32],
         }
@@ -182,6 +186,31 @@ def sz_encode_static(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16, d_statu
                                   _p(d_status), _s(stream)), "sz_encode_static")
 
 
+def sz_plan_one_pass(n: int):
+    """-> (max_compressed_bytes for any codebook, workspace_bytes) of sz_encode_one_pass"""
+    a, b = ctypes.c_uint64(), ctypes.c_uint64()
+    _check(lib().sz_plan_one_pass(n, ctypes.byref(a), ctypes.byref(b)), "sz_plan_one_pass")
+    return a.value, b.value
+
+
+def sz_encode_one_pass(d_in, n, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, ws_bytes, stream=None):
+    _check(lib().sz_encode_one_pass(_p(d_in), n, _p(d_codebook16), _p(d_out), out_cap, _p(d_out_bytes),
+                                    _p(d_status), _p(d_ws), ws_bytes, _s(stream)), "sz_encode_one_pass")
+
+
+def sz_workspace_one_pass_batched(n_segs: int, n_tiles: int) -> int:
+    w = ctypes.c_uint64()
+    _check(lib().sz_workspace_one_pass_batched(n_segs, n_tiles, ctypes.byref(w)), "sz_workspace_one_pass_batched")
+    return w.value
+
+
+def sz_encode_one_pass_batched(n_segs, d_segs, n_tiles, d_pages, page_elems, d_codebooks, d_out, out_cap,
+                               d_out_bytes, d_status, d_ws, ws_bytes, stream=None):
+    _check(lib().sz_encode_one_pass_batched(n_segs, _p(d_segs), n_tiles, _p(d_pages), page_elems, _p(d_codebooks),
+                                            _p(d_out), out_cap, _p(d_out_bytes), _p(d_status), _p(d_ws), ws_bytes,
+                                            _s(stream)), "sz_encode_one_pass_batched")
+
+
 def sz_set_wait_limit_ns(limit_ns: int):
     _check(lib().sz_set_wait_limit_ns(limit_ns), "sz_set_wait_limit_ns")
 
@@ -236,6 +265,24 @@ def encode(x, stream=None, workspace=None):
     return out, size, status
 
 
+def encode_one_pass(x, codebook, stream=None, workspace=None):
+    """Encode a contiguous 16-bit CUDA tensor with a given codebook (16
+    distinct exponents, uint8 CUDA tensor), reading it once.  Returns
+    (container uint8 tensor sized for any codebook, size int64 tensor [1],
+    status int32 tensor [1])."""
+    torch = _torch()
+    x = _u16_view(x.contiguous())
+    n = x.numel()
+    cap, wsb = sz_plan_one_pass(n)
+    dev = x.device
+    ws = workspace if workspace is not None else torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    size = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sz_encode_one_pass(x, n, codebook, out, cap, size, status, ws, ws.numel(), stream)
+    return out, size, status
+
+
 def decode(container, n, out=None, stream=None, workspace=None):
     """Decode a container (uint8 CUDA tensor) of n elements into an int16
     tensor (bit patterns).  Returns (out, status int32 tensor [1])."""
@@ -285,6 +332,18 @@ class BatchPlan:
     def encode(self, d_page_ptrs, stream=None):
         self.histogram(d_page_ptrs, stream)
         self.encode_only(d_page_ptrs, stream)
+
+    def encode_one_pass(self, d_page_ptrs, d_codebooks, stream=None):
+        """Every segment's container with the caller's codebooks (uint8
+        [n_segs][16] on the device), reading the input once; the one-pass
+        workspace is allocated on first use."""
+        torch = _torch()
+        if getattr(self, "ws1", None) is None:
+            wb = sz_workspace_one_pass_batched(self.n_segs, self.n_tiles)
+            self.ws1 = torch.empty(max(wb, 256), dtype=torch.uint8, device=self.container.device)
+        sz_encode_one_pass_batched(self.n_segs, self.d_segs, self.n_tiles, d_page_ptrs, self.page_elems, d_codebooks,
+                                   self.container, self.container.numel(), self.sizes, self.enc_status, self.ws1,
+                                   self.ws1.numel(), stream)
 
     def decode(self, d_page_ptrs, stream=None, container=None):
         """Decode every segment into the pages d_page_ptrs lists.  container:

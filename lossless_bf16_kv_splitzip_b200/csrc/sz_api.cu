@@ -10,6 +10,8 @@ namespace sz {
 cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
+cudaError_t launch_encode_one_pass(const EncodeArgs &a, bool batched, cudaStream_t s);
+cudaError_t launch_place(const PlaceArgs &a, bool batched, int sms, cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
@@ -73,6 +75,27 @@ Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
     return w;
 }
 
+// ---- one-pass workspace for T tiles and G = min(T, kMaxRanges) ranges
+//   ovf_count u32                 tiles listed for the rescan (zeroed per call)
+//   rcnt      RangeRec[G]         escapes of each range's first and last piece
+//   tile_cnt  u32[T]              escapes of each tile
+//   ovf       OvfItem[T]          tiles whose records overflowed their slot
+//   slots     u32[T][kSlotCap]    each tile's first kSlotCap escape records
+struct Ws1 {
+    uint64_t ovf_count, rcnt, tile_cnt, ovf, slots, total;
+};
+Ws1 ws1_layout(uint64_t n_tiles) {
+    const uint64_t g = umin64(n_tiles, kMaxRanges);
+    Ws1 w;
+    w.ovf_count = 0;
+    w.rcnt = kAlign;
+    w.tile_cnt = round_up(w.rcnt + sizeof(RangeRec) * g, kAlign);
+    w.ovf = round_up(w.tile_cnt + 4 * n_tiles, kAlign);
+    w.slots = round_up(w.ovf + sizeof(OvfItem) * n_tiles, kAlign);
+    w.total = round_up(w.slots + 4ull * kSlotCap * n_tiles, kAlign);
+    return w;
+}
+
 Batch single_batch(uint64_t n) {
     Batch b{};
     b.segs = nullptr;
@@ -133,6 +156,50 @@ sz_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SZ_OK : SZ_ERR_
         cudaError_t _e = (call);                   \
         if (_e != cudaSuccess) return SZ_ERR_CUDA; \
     } while (0)
+
+// ---- one pass with the caller's codebook(s): encode, then escape placement
+sz_status one_pass(const Batch &b, const uint16_t *const *d_pages, const uint16_t *d_in,
+                          const uint8_t *d_codebooks, uint8_t *d_out, uint64_t out_cap, uint64_t *d_out_bytes,
+                          int32_t *d_status, void *d_ws, const Ws1 &w, cudaStream_t s) {
+    DeviceInfo dev;
+    if (!device_info(dev)) return SZ_ERR_CUDA;
+    const uint64_t ns = b.segs ? b.n_segs : 1;
+    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, 8 * ns, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * ns, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.ovf_count), 0, 4, s));
+    EncodeArgs a{};
+    a.batch = b;
+    a.pages = d_pages;
+    a.base = d_in;
+    a.out = d_out;
+    a.out_cap = out_cap;
+    a.out_bytes = d_out_bytes;
+    a.status = d_status;
+    a.range_tiles = plan_ranges(b.n_tiles, (uint64_t)dev.sms).tiles;
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    a.codebooks_in = d_codebooks;
+    a.tile_cnt = at<uint32_t>(d_ws, w.tile_cnt);
+    a.slots = at<uint32_t>(d_ws, w.slots);
+    a.rcnt = at<RangeRec>(d_ws, w.rcnt);
+    if (b.n_tiles > 0) SZ_TRY_CUDA(launch_encode_one_pass(a, b.segs != nullptr, s));
+    PlaceArgs p{};
+    p.batch = b;
+    p.pages = d_pages;
+    p.base = d_in;
+    p.codebooks_in = d_codebooks;
+    p.out = d_out;
+    p.out_cap = out_cap;
+    p.out_bytes = d_out_bytes;
+    p.status = d_status;
+    p.tile_cnt = a.tile_cnt;
+    p.slots = a.slots;
+    p.rcnt = a.rcnt;
+    p.range_tiles = a.range_tiles;
+    p.ovf_count = at<uint32_t>(d_ws, w.ovf_count);
+    p.ovf = at<OvfItem>(d_ws, w.ovf);
+    return cuda_status(launch_place(p, b.segs != nullptr, dev.sms, s));
+}
 
 }  // namespace
 
@@ -331,6 +398,53 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.debug_flags = g_debug_flags.load();
     SZ_TRY_CUDA(launch_esc_index(a, true, s));
     return cuda_status(launch_decode(a, true, dev.sms * dev.dec_occ, s));
+}
+
+sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes) {
+    if (!max_compressed_bytes || !workspace_bytes) return SZ_ERR_NULL;
+    if (n_elems > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    *max_compressed_bytes = container_size(n_elems, n_elems);
+    *workspace_bytes = ws1_layout(single_batch(n_elems).n_tiles).total;
+    return SZ_OK;
+}
+
+sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
+                             uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
+                             uint64_t ws_bytes, void *stream) {
+    if (!d_codebook16 || !d_out || !d_out_bytes || !d_status || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
+    if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
+    if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
+    const Batch b = single_batch(n);
+    const Ws1 w = ws1_layout(b.n_tiles);
+    if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
+    return one_pass(b, nullptr, d_in, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, w,
+                    static_cast<cudaStream_t>(stream));
+}
+
+sz_status sz_workspace_one_pass_batched(uint32_t n_segs, uint64_t n_tiles, uint64_t *workspace_bytes) {
+    (void)n_segs;
+    if (!workspace_bytes) return SZ_ERR_NULL;
+    if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
+    *workspace_bytes = ws1_layout(n_tiles).total;
+    return SZ_OK;
+}
+
+sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                                     const uint16_t *const *d_pages, uint64_t page_elems,
+                                     const uint8_t *d_codebooks, uint8_t *d_out, uint64_t out_cap,
+                                     uint64_t *d_out_bytes, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
+                                     void *stream) {
+    if (n_segs == 0) return SZ_OK;
+    if (!d_segs || !d_codebooks || !d_out || !d_out_bytes || !d_status || !d_ws || (n_tiles > 0 && !d_pages))
+        return SZ_ERR_NULL;
+    if (page_elems == 0) return SZ_ERR_INVALID;
+    if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
+    if (!aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
+    const Ws1 w = ws1_layout(n_tiles);
+    if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
+    return one_pass(make_batch(n_segs, d_segs, n_tiles, page_elems), d_pages, nullptr, d_codebooks, d_out, out_cap,
+                    d_out_bytes, d_status, d_ws, w, static_cast<cudaStream_t>(stream));
 }
 
 sz_status sz_set_wait_limit_ns(uint64_t limit_ns) {

@@ -326,15 +326,6 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
 }
 
 // ------------------------------------------------------------ consumers
-// 256-bit codebook membership in 8 registers, selected without local memory.
-__device__ __forceinline__ bool in_set8(const uint32_t (&set)[8], uint32_t x) {
-    const uint32_t w = x >> 5;
-    uint32_t v = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v = (w == (uint32_t)i) ? set[i] : v;
-    return (v >> (x & 31)) & 1u;
-}
-
 // One chunk: 16 sm bytes + 8 code bytes -> 16 BF16 values, stored.  The
 // escaped places get codebook[0] here and are overwritten afterwards.
 __device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &sh, int s, const DecTables &T, int q,

@@ -31,6 +31,10 @@ constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
 constexpr uint32_t kFlagLastSub = 4u;    // last sub-tile of its piece (the range's tiles of one segment)
 constexpr uint32_t kFlagHeader = 8u;     // first sub-tile of the segment: write the header
 constexpr uint32_t kFlagLastTile = 16u;  // last tile of the segment: write the size
+// one-pass mode (kFlagLastSub then marks the last sub-tile of a tile)
+constexpr uint32_t kFlagPieceEnd = 32u;     // last sub-tile of the piece
+constexpr uint32_t kFlagPieceOpens = 64u;   // the piece opens the range
+constexpr uint32_t kFlagPieceCloses = 128u; // the piece closes the range
 
 struct EncMeta {
     const uint16_t *src;  // global address of the sub-tile's first element
@@ -38,9 +42,9 @@ struct EncMeta {
     uint32_t seg;
     uint32_t len;         // elements of the sub-tile
     uint32_t flags;
-    uint32_t esc_base;    // first escape index of the piece
-    uint32_t esc_count;   // escapes the piece must produce
-    uint32_t pad;
+    uint32_t esc_base;    // first escape index of the piece (one-pass: the global tile)
+    uint32_t esc_count;   // escapes the piece must produce (one-pass: unused)
+    uint32_t sub_in_tile; // sub-tile index within its tile
 };
 
 struct __align__(128) EncShared {
@@ -112,17 +116,6 @@ __device__ __forceinline__ uint32_t esc_in_element_order(uint32_t m) {
 
 __device__ __forceinline__ uint32_t esc_bit_of_elem(int j) { return 1u << (8 * (j & 3) + (j >> 2)); }
 
-__device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligned) {
-    if (aligned) {
-        *reinterpret_cast<uint32_t *>(p) = v;
-    } else {
-        p[0] = (uint8_t)v;
-        p[1] = (uint8_t)(v >> 8);
-        p[2] = (uint8_t)(v >> 16);
-        p[3] = (uint8_t)(v >> 24);
-    }
-}
-
 __device__ __forceinline__ uint32_t field16(uint64_t v, int c) { return (uint32_t)(v >> (16 * c)) & 0xFFFFu; }
 
 // Read chunk (c, tid) of a stage: 32 bytes at (c*256 + tid)*32 (two 16-byte
@@ -148,7 +141,7 @@ __device__ __forceinline__ void read_chunk_global(const uint16_t *p, uint32_t cn
 }
 
 // ------------------------------------------------------------ producer
-template <bool kBatched>
+template <bool kBatched, bool kOnePass>
 __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
     const uint64_t t_begin = (uint64_t)blockIdx.x * a.range_tiles;
@@ -161,22 +154,29 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
     bool seg_ok = false;
     uint64_t e_total = 0;
     uint32_t p_base = 0, p_count = 0;  // the piece's first escape index and escape count
-    uint64_t p_last = 0;               // the piece's last tile
+    uint64_t p_first = 0, p_last = 0;  // the piece's first and last tile
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {  // a new piece: the range's tiles of segment k
             cur = k;
             seg = load_segment(a.batch, k);
-            const SegMeta &m = a.meta[k];
-            e_total = m.n_escapes;
+            bool valid;
+            if (kOnePass) {  // the caller's codebook; the container size is known only later
+                valid = codebook16_distinct(a.codebooks_in + 16 * (size_t)k);
+                e_total = 0;
+            } else {
+                valid = a.meta[k].valid != 0;
+                e_total = a.meta[k].n_escapes;
+            }
             const bool fits = seg.out_offset <= a.out_cap &&
                               container_size(seg.n_elems, e_total) <= a.out_cap - seg.out_offset;
             const bool aligned = (reinterpret_cast<uintptr_t>(a.out + seg.out_offset) & 15) == 0;
-            seg_ok = m.valid != 0 && fits && aligned;
-            if (m.valid == 0) set_status(a.status + k, SZ_ERR_INVALID);
+            seg_ok = valid && fits && aligned;
+            if (!valid) set_status(a.status + k, SZ_ERR_INVALID);
             else if (!fits) set_status(a.status + k, SZ_ERR_CAPACITY);
             else if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
             const uint64_t seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
+            p_first = t;
             p_last = umin64(seg_end, t_end) - 1;
             if (t == t_begin) {  // opens the range
                 p_base = rr.first_off;
@@ -205,12 +205,24 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             m.elem0 = r.elem0 + (uint64_t)sub * kSub;
             m.seg = k;
             m.len = aligned ? umin32(kSub, r.len - sub * kSub) : 0u;  // nothing is read from a misaligned page
-            m.esc_base = p_base;
-            m.esc_count = p_count;
+            m.sub_in_tile = sub;
             uint32_t f = 0;
-            if (t == p_last && sub + 1 == r.n_subs) f |= kFlagLastSub;
-            if (r.local == 0 && sub == 0) f |= kFlagHeader;
-            if (r.local + 1 == r.tiles) f |= kFlagLastTile;
+            if (kOnePass) {
+                m.esc_base = (uint32_t)t;
+                m.esc_count = 0;
+                if (sub + 1 == r.n_subs) f |= kFlagLastSub;
+                if (t == p_last && sub + 1 == r.n_subs) {
+                    f |= kFlagPieceEnd;
+                    if (p_first == t_begin) f |= kFlagPieceOpens;
+                    if (p_last + 1 == t_end) f |= kFlagPieceCloses;
+                }
+            } else {
+                m.esc_base = p_base;
+                m.esc_count = p_count;
+                if (t == p_last && sub + 1 == r.n_subs) f |= kFlagLastSub;
+                if (r.local == 0 && sub == 0) f |= kFlagHeader;
+                if (r.local + 1 == r.tiles) f |= kFlagLastTile;
+            }
             const bool tma = m.len == kSub;
             if (tma) f |= kFlagInSmem;
             m.flags = f;
@@ -239,20 +251,33 @@ struct PendingEsc {
     uint8_t *raw_base;
     bool pos_aligned;
     int32_t *status;
+    uint32_t *slot;         // one-pass: the tile's record slot
+    uint32_t tile_off;      // one-pass: offset of the sub-tile in its tile
 };
 
 // Every consumer thread takes records tid, tid + 256, ...: consecutive
-// threads write consecutive positions and exponents.
+// threads write consecutive positions and exponents (one-pass: consecutive
+// slot entries, the first kSlotCap records of the tile).
+template <bool kOnePass>
 __device__ __forceinline__ void copy_out_escapes(const uint32_t *stg, const PendingEsc &p, int tid) {
-    for (uint32_t i = tid; i < p.cnt; i += kThreads) {
-        const uint64_t g = p.first + i;
-        if (g >= p.lim) {  // more escapes than the histograms said
-            set_status(p.status, SZ_ERR_CORRUPT);
-            break;
+    if constexpr (kOnePass) {
+        for (uint32_t i = tid; i < p.cnt; i += kThreads) {
+            const uint64_t g = p.first + i;
+            if (g >= kSlotCap) break;
+            const uint32_t rec = stg[i];
+            p.slot[g] = (rec & 0xFF0000u) | (p.tile_off + (rec & 0xFFFFu));
         }
-        const uint32_t rec = stg[i];
-        store_u32_le(p.pos_base + 4 * g, (uint32_t)(p.elem0 + (rec & 0xFFFFu)), p.pos_aligned);
-        p.raw_base[g] = (uint8_t)(rec >> 16);
+    } else {
+        for (uint32_t i = tid; i < p.cnt; i += kThreads) {
+            const uint64_t g = p.first + i;
+            if (g >= p.lim) {  // more escapes than the histograms said
+                set_status(p.status, SZ_ERR_CORRUPT);
+                break;
+            }
+            const uint32_t rec = stg[i];
+            store_u32_le(p.pos_base + 4 * g, (uint32_t)(p.elem0 + (rec & 0xFFFFu)), p.pos_aligned);
+            p.raw_base[g] = (uint8_t)(rec >> 16);
+        }
     }
 }
 
@@ -295,14 +320,15 @@ __device__ __forceinline__ bool warp_escape_scan(const uint32_t (&esc)[kChunks],
     return true;  // some chunk of the warp has several escapes
 }
 
-template <bool kBatched>
+template <bool kBatched, bool kOnePass>
 __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     uint32_t cur = 0xFFFFFFFFu;
     uint8_t *out = nullptr;
     uint64_t n = 0, e_total = 0;
     bool codes_aligned = false, pos_aligned = false;
-    uint32_t running = 0;  // escapes of the current piece so far
+    uint32_t running = 0;  // escapes of the current piece so far (one-pass: of the tile)
+    uint32_t piece_acc = 0;  // one-pass: escapes of the current piece so far
     PendingEsc pend{};
 
     // The wait for stage j+1 is folded into sub-tile j's scan barrier: one
@@ -321,18 +347,18 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const EncMeta m = sh.meta[s];
         if (m.flags & kFlagEnd) {
             consumer_sync();  // the last sub-tile's staged records are complete
-            copy_out_escapes(sh.esc[(j + 1) & 1], pend, tid);
+            copy_out_escapes<kOnePass>(sh.esc[(j + 1) & 1], pend, tid);
             return;
         }
         if (m.seg != cur) {  // every consumer is past the previous sub-tile's compute
             s_lut[tid] = 0x80;
             consumer_sync();
-            const SegMeta &g = a.meta[m.seg];
-            if (tid < 16) s_lut[g.codebook[tid]] = (uint8_t)tid;
+            const uint8_t *cbk = kOnePass ? a.codebooks_in + 16 * (size_t)m.seg : a.meta[m.seg].codebook;
+            if (tid < 16) s_lut[cbk[tid]] = (uint8_t)tid;
             const sz_segment seg = load_segment(a.batch, m.seg);
             out = a.out + seg.out_offset;
             n = seg.n_elems;
-            e_total = g.n_escapes;
+            e_total = kOnePass ? 0 : a.meta[m.seg].n_escapes;
             codes_aligned = (n % 8) == 0;
             pos_aligned = ((kHeader + n + (n + 1) / 2) & 3) == 0;
             cur = m.seg;
@@ -426,7 +452,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
         const uint32_t sub_total = field16(tot, 0) + field16(tot, 1) + field16(tot, 2) + field16(tot, 3);
 
         // ---- the previous sub-tile's staged records, coalesced
-        copy_out_escapes(sh.esc[(j + 1) & 1], pend, tid);
+        copy_out_escapes<kOnePass>(sh.esc[(j + 1) & 1], pend, tid);
         pend.cnt = 0;
 
         // ---- this sub-tile's records, in element order
@@ -435,8 +461,11 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             uint8_t *pos_base = out + pos_off;
             uint8_t *raw_base = pos_base + 4 * e_total;
             // the records this sub-tile may write: [first, last) of the segment
-            const uint64_t first = (uint64_t)m.esc_base + running;
-            const uint64_t lim = umin64(e_total, (uint64_t)m.esc_base + m.esc_count);
+            // (one-pass: of the tile's slot)
+            const uint64_t first = kOnePass ? (uint64_t)running : (uint64_t)m.esc_base + running;
+            const uint64_t lim = kOnePass ? (uint64_t)kSlotCap : umin64(e_total, (uint64_t)m.esc_base + m.esc_count);
+            uint32_t *slot = kOnePass ? a.slots + (size_t)m.esc_base * kSlotCap : nullptr;
+            const uint32_t tile_off = m.sub_in_tile * kSub;
             const bool staged = sub_total <= kEscStage;
             uint32_t *stg = sh.esc[j & 1];
             uint32_t chunk_base = 0;
@@ -462,6 +491,9 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
                     const uint32_t raw = (x >> 7) & 0xFFu;
                     if (staged) {
                         stg[idx] = (raw << 16) | (off + q);
+                    } else if (kOnePass) {
+                        const uint64_t g = first + idx;
+                        if (g < lim) slot[g] = (raw << 16) | (tile_off + off + q);
                     } else {
                         const uint64_t g = first + idx;
                         if (g >= lim) {  // more escapes than the histograms said
@@ -486,10 +518,23 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
                 pend.raw_base = raw_base;
                 pend.pos_aligned = pos_aligned;
                 pend.status = status;
+                pend.slot = slot;
+                pend.tile_off = tile_off;
             }
         }
         running += sub_total;
-        if (m.flags & kFlagLastSub) {
+        if (kOnePass && (m.flags & kFlagLastSub)) {  // end of a tile: its count, and the piece's
+            piece_acc += running;
+            if (tid == 0) {
+                a.tile_cnt[m.esc_base] = running;
+                if (m.flags & kFlagPieceEnd) {
+                    if (m.flags & kFlagPieceOpens) a.rcnt[blockIdx.x].first_cnt = piece_acc;
+                    else if (m.flags & kFlagPieceCloses) a.rcnt[blockIdx.x].last_cnt = piece_acc;
+                }
+            }
+            if (m.flags & kFlagPieceEnd) piece_acc = 0;
+            running = 0;
+        } else if (!kOnePass && (m.flags & kFlagLastSub)) {
             if (tid == 0) {
                 if (running != m.esc_count) set_status(status, SZ_ERR_CORRUPT);
                 else if (m.flags & kFlagLastTile) a.out_bytes[m.seg] = container_size(n, e_total);
@@ -501,7 +546,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     }
 }
 
-template <bool kBatched>
+template <bool kBatched, bool kOnePass>
 __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     EncShared &sh = *reinterpret_cast<EncShared *>(smem_raw);
@@ -515,8 +560,9 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
     }
     seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
 
-    // Segments with no elements have no tiles: CTA 0 writes their header.
-    if (blockIdx.x == 0 && tid < kThreads) {
+    // Segments with no elements have no tiles: CTA 0 writes their header
+    // (one-pass: the escape placement does).
+    if (!kOnePass && blockIdx.x == 0 && tid < kThreads) {
         const uint32_t ns = kBatched ? a.batch.n_segs : 1;
         for (uint32_t k = tid; k < ns; k += kThreads) {
             const sz_segment s = load_segment(a.batch, k);
@@ -542,35 +588,31 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
     }
 
     if (tid >= kThreads) {
-        if (tid == kThreads) encode_producer<kBatched>(a, sh);
+        if (tid == kThreads) encode_producer<kBatched, kOnePass>(a, sh);
     } else {
-        encode_consumers<kBatched>(a, sh);
+        encode_consumers<kBatched, kOnePass>(a, sh);
     }
 }
 
-// One CTA per range of the partition the histogram kernel used.
-cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s) {
+// One CTA per range of the partition the histogram kernel used (one-pass:
+// of the partition the escape placement will use).
+template <bool kBatched, bool kOnePass>
+cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
     const size_t smem = sizeof(EncShared);
     const int grid = (int)umax64(1, div_up(a.batch.n_tiles, a.range_tiles));
-    cudaError_t e;
-    if (batched) {
-        e = cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        encode_kernel<true><<<grid, kPipeThreads, smem, s>>>(a);
-    } else {
-        e = cudaFuncSetAttribute(encode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        encode_kernel<false><<<grid, kPipeThreads, smem, s>>>(a);
-    }
+    const cudaError_t e =
+        cudaFuncSetAttribute(encode_kernel<kBatched, kOnePass>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    encode_kernel<kBatched, kOnePass><<<grid, kPipeThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 
-int encode_blocks_per_sm() {
-    const size_t smem = sizeof(EncShared);
-    cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, encode_kernel<true>, kPipeThreads, smem);
-    return occ > 0 ? occ : 1;
+cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s) {
+    return batched ? launch_encode_t<true, false>(a, s) : launch_encode_t<false, false>(a, s);
+}
+
+cudaError_t launch_encode_one_pass(const EncodeArgs &a, bool batched, cudaStream_t s) {
+    return batched ? launch_encode_t<true, true>(a, s) : launch_encode_t<false, true>(a, s);
 }
 
 }  // namespace sz

@@ -37,6 +37,7 @@ constexpr uint64_t kHeader = 48;
 constexpr uint32_t kMaxSmemSegs = 256;  // segment starts cached in shared memory
 constexpr uint64_t kMaxRanges = 1024;   // ranges of one call (workspace bound)
 constexpr uint64_t kRangesPerSM = 3;    // encode CTAs resident per SM
+constexpr uint32_t kSlotCap = 4096;     // one-pass encode: escape records staged per tile (6.25 %)
 
 // Per-segment record kept in the workspace between kernels (32 bytes).
 struct SegMeta {
@@ -188,6 +189,44 @@ __device__ inline TileRef resolve_tile(const Batch &b, const sz_segment &s, uint
     return r;
 }
 
+// 16 codebook entries, all different (one thread, byte loads: any alignment).
+__device__ inline bool codebook16_distinct(const uint8_t *cb) {
+    uint64_t lo = 0, hi = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        lo |= (uint64_t)cb[i] << (8 * i);
+        hi |= (uint64_t)cb[8 + i] << (8 * i);
+    }
+    bool ok = true;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+#pragma unroll
+        for (int k = i + 1; k < 16; ++k)
+            ok &= ((((i < 8) ? lo : hi) >> (8 * (i & 7))) & 0xFFu) != ((((k < 8) ? lo : hi) >> (8 * (k & 7))) & 0xFFu);
+    return ok;
+}
+
+// 256-bit codebook membership in 8 registers, selected without local memory.
+__device__ __forceinline__ bool in_set8(const uint32_t (&set)[8], uint32_t x) {
+    const uint32_t w = x >> 5;
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v = (w == (uint32_t)i) ? set[i] : v;
+    return (v >> (x & 31)) & 1u;
+}
+
+// Little-endian u32 at p, 4-byte aligned or not.
+__device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligned) {
+    if (aligned) {
+        *reinterpret_cast<uint32_t *>(p) = v;
+    } else {
+        p[0] = (uint8_t)v;
+        p[1] = (uint8_t)(v >> 8);
+        p[2] = (uint8_t)(v >> 16);
+        p[3] = (uint8_t)(v >> 24);
+    }
+}
+
 // ------------------------------------------------------------ status words
 __device__ inline void set_status(int32_t *status, int32_t code) {
     if (status != nullptr) atomicCAS(reinterpret_cast<int *>(status), 0, code);
@@ -322,6 +361,38 @@ struct EncodeArgs {
     uint64_t range_tiles;     // tiles per range = per CTA
     uint64_t wait_limit_ns;
     uint32_t debug_flags;
+    // one-pass mode (caller codebooks, no histogram pass)
+    const uint8_t *codebooks_in;  // [n_segs][16]
+    uint32_t *tile_cnt;           // [n_tiles] escapes of each tile
+    uint32_t *slots;              // [n_tiles][kSlotCap] records: raw << 16 | offset in the tile
+    RangeRec *rcnt;               // [ranges] first_cnt / last_cnt: escapes of the first / last piece
+};
+
+// A tile whose escapes overflowed its record slot, left for the rescan.
+struct OvfItem {
+    uint64_t tile;  // global tile index
+    uint64_t base;  // index of the tile's first escape record in its segment
+    uint64_t e;     // escapes of the segment
+    uint32_t cnt;   // escapes of the tile
+    uint32_t seg;
+};
+
+// The escape placement that follows a one-pass encode.
+struct PlaceArgs {
+    Batch batch;
+    const uint16_t *const *pages;
+    const uint16_t *base;
+    const uint8_t *codebooks_in;  // [n_segs][16]
+    uint8_t *out;
+    uint64_t out_cap;
+    uint64_t *out_bytes;          // [n_segs]
+    int32_t *status;              // [n_segs]
+    const uint32_t *tile_cnt;     // [n_tiles]
+    const uint32_t *slots;        // [n_tiles][kSlotCap]
+    const RangeRec *rcnt;         // [ranges]
+    uint64_t range_tiles;
+    uint32_t *ovf_count;          // overflowed tiles listed so far (zero on entry)
+    OvfItem *ovf;                 // [n_tiles]
 };
 
 struct DecodeArgs {
