@@ -23,7 +23,6 @@ struct PlaceShared {
     uint32_t warp[kWarps];
     uint32_t base[kThreads];  // per tile of the current chunk: index of its first record in the segment
     uint32_t cnt[kThreads];   // per tile of the current chunk: its records
-    uint32_t flat[kThreads + 1];  // per tile: first of its slot records in the chunk's flat order
     uint64_t elem0[kThreads];     // per tile: its first element in the segment's stream
     int32_t status;           // the segment's status as thread 0 read it
 };
@@ -182,7 +181,7 @@ template <bool kBatched>
 __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
     __shared__ PlaceShared sh;
     seg_cache_fill(sh.segc, a.batch);  // ends with __syncthreads
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (blockIdx.x == 0) place_empty_segments(a);
 
     const uint64_t R = a.range_tiles;
@@ -235,46 +234,37 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
         const bool pos_aligned = (pos_off & 3) == 0;
 
         // the piece's tiles, kThreads at a time: the first record index of
-        // each; then the slot records of all of them as one flat array (four
-        // loads in flight per thread); then the tiles whose slot overflowed
+        // each; then one warp per tile moves its slot records (coalesced,
+        // four loads in flight per lane); tiles whose slot overflowed are
+        // listed for the rescan kernel
         uint64_t carry = pre;
         for (uint64_t c0 = ps; c0 < pe; c0 += kThreads) {
             const uint64_t tt = c0 + tid;
             const uint32_t cnt = tt < pe ? a.tile_cnt[tt] : 0u;
-            uint32_t total = 0, flat_total = 0;
+            uint32_t total = 0;
             const uint32_t excl = block_excl_scan(cnt, &total, sh);
-            const uint32_t flat = block_excl_scan(cnt <= kSlotCap ? cnt : 0u, &flat_total, sh);
             sh.cnt[tid] = cnt;
             sh.base[tid] = (uint32_t)(carry + excl);
-            sh.flat[tid] = flat;
             sh.elem0[tid] = tt < pe ? resolve_tile(a.batch, seg, k, tt).elem0 : 0;
-            if (tid == 0) sh.flat[kThreads] = flat_total;
             __syncthreads();
             const uint32_t nt = (uint32_t)umin64(kThreads, pe - c0);
-            for (uint32_t f0 = tid; f0 < flat_total; f0 += 4 * kThreads) {
-                uint32_t rec[4], ti[4], fi[4];
+            for (uint32_t i = wid; i < nt; i += kWarps) {
+                const uint32_t ci = sh.cnt[i];
+                if (ci > kSlotCap) continue;
+                const uint32_t *slot = a.slots + (c0 + i) * kSlotCap;
+                const uint64_t bi = sh.base[i], e0 = sh.elem0[i];
+                for (uint32_t j0 = lane; j0 < ci; j0 += 128) {
+                    uint32_t rec[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    fi[u] = f0 + u * kThreads;
-                    ti[u] = 0;
-                    rec[u] = 0;
-                    if (fi[u] < flat_total) {
-                        uint32_t lo = 0, hi = nt;  // last tile i with flat[i] <= fi
-                        while (hi - lo > 1) {
-                            const uint32_t mid = (lo + hi) >> 1;
-                            if (sh.flat[mid] <= fi[u]) lo = mid; else hi = mid;
-                        }
-                        ti[u] = lo;
-                        rec[u] = a.slots[(c0 + lo) * kSlotCap + (fi[u] - sh.flat[lo])];
+                    for (int u = 0; u < 4; ++u) rec[u] = (j0 + 32 * u < ci) ? slot[j0 + 32 * u] : 0u;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t jj = j0 + 32 * u;
+                        if (jj >= ci) break;
+                        const uint64_t g = bi + jj;
+                        store_u32_le(pos_base + 4 * g, (uint32_t)(e0 + (rec[u] & 0xFFFFu)), pos_aligned);
+                        raw_base[g] = (uint8_t)(rec[u] >> 16);
                     }
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (fi[u] >= flat_total) continue;
-                    const uint32_t i = ti[u];
-                    const uint64_t g = (uint64_t)sh.base[i] + (fi[u] - sh.flat[i]);
-                    store_u32_le(pos_base + 4 * g, (uint32_t)(sh.elem0[i] + (rec[u] & 0xFFFFu)), pos_aligned);
-                    raw_base[g] = (uint8_t)(rec[u] >> 16);
                 }
             }
             if (tid < nt && cnt > kSlotCap) {  // left for the rescan kernel
