@@ -57,6 +57,11 @@ def parse_args():
                         "workload's buffer), one JSON line per size")
     p.add_argument("--sweep-max", type=int, default=1 << 32, help="largest sweep size in bytes")
     p.add_argument("--sweep-reps", type=int, default=20)
+    p.add_argument("--transfer", action="store_true",
+                   help="transfer instead: the workload's cache moved GPU -> pinned host -> GPU in chunks, "
+                        "raw vs compressed (encode / decode overlapped with the copies); one JSON line")
+    p.add_argument("--transfer-chunk", type=int, default=4, help="tensors per chunk")
+    p.add_argument("--transfer-reps", type=int, default=3)
     return p.parse_args()
 
 
@@ -323,6 +328,60 @@ def run_sweep(args):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------- transfer
+def run_transfer(args):
+    """The cache handed from one place to another over a link: here PCIe
+    through pinned host memory (the only link one GPU has), device-to-host
+    and host-to-device copies on their own streams, chunk by chunk.  Raw:
+    the BF16 values cross.  Compressed: each chunk is encoded before it
+    crosses and decoded after (kernels overlapped with the other chunks'
+    copies).  Device time from the first operation to the last."""
+    import torch
+
+    from lossless_bf16_kv_splitzip_b200.transfer import SplitZipChunks, host_transfer
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = workload_config(args.tensors)
+    S, n = cfg["tensors"], cfg["elems_per_tensor"]
+    h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
+    host = h_in.numpy().view(np.uint16)
+    if S % 2 == 0:
+        kvgen.contiguous_cache(WORKLOAD, layers=S // 2, out=host)
+    else:
+        for k in range(S):
+            host[k] = kvgen.contiguous_tensor(WORKLOAD, k // 2, k % 2)
+    src = h_in.to(dev)
+    del h_in, host
+    out = torch.empty_like(src)
+    staging = torch.empty(2 * S * n + 4096 * S, dtype=torch.uint8, pin_memory=True)
+    codec = SplitZipChunks(src, out, args.transfer_chunk, dev)
+    res = {}
+    for name, cd in (("raw", None), ("compressed", codec)):
+        times = []
+        for r in range(1 + args.transfer_reps):
+            out.zero_()
+            t = host_transfer(cd, src, out, args.transfer_chunk, staging)
+            torch.cuda.synchronize(dev)
+            if r:
+                times.append(t.seconds)
+            assert torch.equal(out, src), name
+            link = t.link_bytes
+        if cd is not None:
+            assert codec.statuses_ok()
+        res[name] = (float(np.median(times)), link)
+    t_raw, b_raw = res["raw"]
+    t_c, b_c = res["compressed"]
+    line = {"transfer": "GPU -> pinned host -> GPU (PCIe), %d chunks of %d tensors" % (len(codec.chunks),
+                                                                                     args.transfer_chunk),
+            "config": cfg, "raw_ms": round(t_raw * 1e3, 3), "compressed_ms": round(t_c * 1e3, 3),
+            "speedup": round(t_raw / t_c, 4), "ratio": round(b_raw / b_c, 5),
+            "raw_link_gbs": round(b_raw / t_raw / 1e9, 2), "compressed_link_gbs": round(b_c / t_c / 1e9, 2),
+            "effective_gbs": round(b_raw / t_c / 1e9, 2), "round_trip": True, "reps": args.transfer_reps,
+            "timing": "CUDA events, first operation to last, median of reps after one warm-up"}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ our arm
 def main():
     args = parse_args()
@@ -332,6 +391,10 @@ def main():
     if args.sweep:
         if int(os.environ.get("RANK", "0")) == 0:
             run_sweep(args)
+        return
+    if args.transfer:
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_transfer(args)
         return
 
     import torch
