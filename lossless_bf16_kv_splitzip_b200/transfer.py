@@ -266,3 +266,90 @@ def recv_chunks(codec, n_chunks: int, max_segs: int, src: int, device, group=Non
         if total:
             dist.irecv(payload, src, group=group).wait()
         codec.decode(c, payload, sizes)
+
+
+# ------------------------------------------------------- host round trip
+def host_round_trip(codec: SplitZipChunks, h_in, h_out, staging, align: int = 4096):
+    """One GPU, through the public calls: the pinned host cache ``h_in``
+    ([S, n] int16) is uploaded chunk by chunk into the codec's ``src``,
+    encoded, its containers packed and downloaded into ``staging``,
+    uploaded again, decoded into the codec's ``out`` and downloaded into
+    ``h_out``.  Uploads and downloads run on their own streams (input
+    uploads apart from container uploads, container downloads apart from
+    output downloads), so both directions of the link stay busy while the
+    kernels run in between.  Returns (device seconds, bytes uploaded, bytes
+    downloaded)."""
+    import torch
+    src, out = codec.src, codec.out
+    dev = src.device
+    chunks = codec.chunks
+    s_in, s_enc, s_pack, s_cd, s_cu, s_dec, s_out = (torch.cuda.Stream(dev) for _ in range(7))
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+
+    def events():
+        return [torch.cuda.Event() for _ in chunks]
+    up, enc_done, pack_done, down, cup, unpacked, dec_done = (events() for _ in range(7))
+    cur = torch.cuda.current_stream(dev)
+    cur.synchronize()
+    start.record(s_in)
+    for st in (s_enc, s_pack, s_cd, s_cu, s_dec, s_out):
+        st.wait_event(start)
+
+    def launch_front(c):  # upload chunk c's input and encode it
+        a, b = chunks[c]
+        with torch.cuda.stream(s_in):
+            src[a:b].copy_(h_in[a:b], non_blocking=True)
+        up[c].record(s_in)
+        s_enc.wait_event(up[c])
+        codec.encode_async(c, s_enc)
+        enc_done[c].record(s_enc)
+
+    ahead = min(2, len(chunks))
+    for c in range(ahead):
+        launch_front(c)
+    pos = 0
+    n_up = n_down = 0
+    for c, (a, b) in enumerate(chunks):
+        enc_done[c].synchronize()  # the host needs the sizes to size the copies
+        sizes = codec.sizes(c)
+        nb = pack_offsets(sizes)[1]
+        if pos + nb > staging.numel():
+            raise ValueError("staging buffer too small: %d bytes needed" % (pos + nb))
+        with torch.cuda.stream(s_pack):
+            s_pack.wait_event(enc_done[c])
+            if c >= kBuffers:
+                s_pack.wait_event(down[c - kBuffers])
+            payload = codec.pack(c, sizes)
+        pack_done[c].record(s_pack)
+        with torch.cuda.stream(s_cd):
+            s_cd.wait_event(pack_done[c])
+            staging[pos: pos + nb].copy_(payload, non_blocking=True)
+        down[c].record(s_cd)
+        with torch.cuda.stream(s_cu):
+            s_cu.wait_event(down[c])
+            if c >= kBuffers:
+                s_cu.wait_event(unpacked[c - kBuffers])
+            land = codec.rx_payload[c % kBuffers][:nb]
+            land.copy_(staging[pos: pos + nb], non_blocking=True)
+        cup[c].record(s_cu)
+        with torch.cuda.stream(s_dec):
+            s_dec.wait_event(cup[c])
+            codec.unpack(c, land, sizes)
+            unpacked[c].record(s_dec)
+            codec.rx[c].decode(codec.out_ptrs[c], s_dec)
+        dec_done[c].record(s_dec)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(dec_done[c])
+            h_out[a:b].copy_(out[a:b], non_blocking=True)
+        if c + ahead < len(chunks):
+            launch_front(c + ahead)
+        pos += (nb + align - 1) // align * align
+        n_up += 2 * (b - a) * src.shape[1] + nb
+        n_down += nb + 2 * (b - a) * src.shape[1]
+    for st in (s_in, s_enc, s_pack, s_cd, s_cu, s_dec):
+        s_out.wait_stream(st)
+    end.record(s_out)
+    end.synchronize()
+    cur.wait_stream(s_out)
+    return start.elapsed_time(end) / 1e3, n_up, n_down

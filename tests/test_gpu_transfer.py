@@ -41,3 +41,21 @@ def test_host_transfer_round_trip(per_chunk):
     res_raw = host_transfer(None, src, raw_out, per_chunk, staging)
     torch.cuda.synchronize()
     assert torch.equal(raw_out, src) and res_raw.link_bytes == 2 * S * n
+
+
+def test_host_round_trip_pipelined():
+    host = kvgen.contiguous_cache(1, layers=3, tokens=1024)  # 6 tensors
+    S, n = host.shape
+    h_in = torch.from_numpy(host.view(np.int16)).pin_memory()
+    h_out = torch.zeros_like(h_in).pin_memory()
+    d_in = torch.zeros((S, n), dtype=torch.int16, device=DEV)
+    d_out = torch.zeros_like(d_in)
+    codec = SplitZipChunks(d_in, d_out, 2, DEV)
+    staging = torch.empty(2 * S * n + 4096 * S, dtype=torch.uint8, pin_memory=True)
+    from lossless_bf16_kv_splitzip_b200.transfer import host_round_trip
+    t, n_up, n_down = host_round_trip(codec, h_in, h_out, staging)
+    torch.cuda.synchronize()
+    assert codec.statuses_ok()
+    assert torch.equal(h_out, h_in)
+    comp = sum(len(oracle.encode(host[k])) for k in range(S))
+    assert n_up == 2 * S * n + comp and n_down == comp + 2 * S * n and t > 0
