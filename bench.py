@@ -34,7 +34,10 @@ sys.path.insert(0, ROOT)
 import kvgen  # noqa: E402
 
 METRIC = "encode / decode GB/s (uncompressed) and % of HBM roofline; compression ratio"
-WORKLOAD = 2
+WORKLOAD = 2          # the headline workload (and the sweep's and transfer's)
+L2_BYTES = 126 * 10**6
+WORKLOAD_NAMES = {0: "tiny-k-1m", 1: "llama3-8b-kv-4k", 2: "llama3-8b-kv-32k",
+                  3: "llama3-70b-kv-8k-heavy-tail", 4: "paged-kv-256-requests"}
 HEADER = 48
 FALLBACK_HBM_GBS = 6650.0
 
@@ -45,6 +48,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="splitzip", choices=["splitzip", "reference"])
+    p.add_argument("--workload", type=int, default=WORKLOAD, choices=sorted(WORKLOAD_NAMES),
+                   help="0 tiny K tensor, 1 Llama-3-8B 4K, 2 Llama-3-8B 32K (default, the headline), "
+                        "3 Llama-3-70B 8K heavy tails, 4 paged batch of 256 requests")
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -65,20 +71,108 @@ def parse_args():
     return p.parse_args()
 
 
-def workload_config(tensors=0):
-    layers, tokens = kvgen.CONTIGUOUS[WORKLOAD]
+def workload_config(tensors=0, workload=WORKLOAD):
+    """The contiguous workloads (0-3): S tensors of n elements."""
+    if workload == 0:
+        n = kvgen.HEADS * 1024 * kvgen.HEAD_DIM
+        return {"workload": WORKLOAD_NAMES[0],
+                "shape": "[%d heads][1024 tokens][%d dim] bf16, 0.1%% of values scaled by 2^+-(20..40)"
+                         % (kvgen.HEADS, kvgen.HEAD_DIM),
+                "tensors": 1, "elems_per_tensor": n, "bytes": 2 * n, "codebooks": "one",
+                "seed": "0x%X" % (kvgen.SEED_BASE + 0),
+                "l2": "input fits the 126 MB L2: a 512 MiB write flushes it before every step; "
+                      "ms_per_step is the sum of the phases"}
+    layers, tokens = kvgen.CONTIGUOUS[workload]
     n = kvgen.HEADS * tokens * kvgen.HEAD_DIM
     t = 2 * layers if tensors <= 0 else min(tensors, 2 * layers)
+    name = WORKLOAD_NAMES[workload]
     return {
-        "workload": "llama3-8b-kv-32k" if t == 2 * layers else "llama3-8b-kv-32k, first %d tensors" % t,
+        "workload": name if t == 2 * layers else "%s, first %d tensors" % (name, t),
         "shape": "[%d layers][K,V][%d heads][%d tokens][%d dim] bf16" % (layers, kvgen.HEADS, tokens, kvgen.HEAD_DIM),
         "tensors": t,
         "elems_per_tensor": n,
         "bytes": 2 * t * n,
         "codebooks": "one per (layer, K/V) tensor",
-        "seed": "0x%X" % (kvgen.SEED_BASE + WORKLOAD),
+        "seed": "0x%X" % (kvgen.SEED_BASE + workload),
         "l2": "inputs (%d MiB) exceed the 126 MB L2; no flush between steps" % (2 * t * n >> 20),
     }
+
+
+def host_cache(cfg, workload, out):
+    """Fill ``out`` ([S, n] uint16 view) with the workload's tensors."""
+    S = cfg["tensors"]
+    if workload == 0:
+        out[0] = kvgen.tiny_k_tensor()
+    elif S % 2 == 0:
+        kvgen.contiguous_cache(workload, layers=S // 2, out=out)
+    else:
+        for k in range(S):
+            out[k] = kvgen.contiguous_tensor(workload, k // 2, k % 2)
+
+
+class Inputs:
+    """One rank's batch on the device: the plan, the page (or tensor)
+    pointers in and out, the uncompressed bytes, and the host units."""
+
+    def __init__(self, args, dev, sz):
+        import torch
+        self.workload = w = args.workload
+        self.contiguous = w != 4
+        if self.contiguous:
+            cfg = workload_config(args.tensors, w)
+            S, n = cfg["tensors"], cfg["elems_per_tensor"]
+            # generated on the host straight into pinned memory, then resident in HBM
+            self.h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
+            host_cache(cfg, w, self.h_in.numpy().view(np.uint16))
+            self.d_in = self.h_in.to(dev, non_blocking=False)
+            self.d_out = torch.empty_like(self.d_in)
+            self.plan = sz.BatchPlan([n] * S, n, device=dev)
+            self.in_ptrs = torch.tensor([self.d_in.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64,
+                                        device=dev)
+            self.out_ptrs = torch.tensor([self.d_out.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64,
+                                         device=dev)
+            self.n_units = S
+        else:
+            b = kvgen.paged_batch()
+            P = kvgen.PAGE_ELEMS
+            lens = [int(v) * kvgen.HEADS * kvgen.HEAD_DIM for v in b.lengths]
+            self.plan = sz.BatchPlan(lens, P, device=dev)
+            self.pool_in = torch.zeros((b.pool_pages, P), dtype=torch.int16, device=dev)
+            for r in range(b.n_requests):
+                idx = torch.from_numpy(b.page_table[r]).to(dev)
+                self.pool_in[idx] = torch.from_numpy(b.pages[r].view(np.int16)).to(dev)
+            src = np.concatenate(b.page_table)
+            dst = np.random.default_rng(kvgen.SEED_BASE + 44).permutation(b.pool_pages)[: src.size]
+            self.pool_out = torch.zeros_like(self.pool_in)
+            self.src_idx = torch.from_numpy(src).to(dev)
+            self.dst_idx = torch.from_numpy(dst).to(dev)
+            self.in_ptrs = torch.from_numpy(src * (2 * P) + self.pool_in.data_ptr()).to(dev)
+            self.out_ptrs = torch.from_numpy(dst * (2 * P) + self.pool_out.data_ptr()).to(dev)
+            self.batch = b
+            self.n_units = b.n_requests
+            cfg = {"workload": WORKLOAD_NAMES[4],
+                   "shape": "%d requests of %d..%d tokens (log-uniform, rounded up to 16), pages [%d heads][16 "
+                            "tokens][%d dim] bf16 scattered in a %d-page pool; decoded into a second pool under "
+                            "another page table" % (b.n_requests, int(b.lengths.min()), int(b.lengths.max()),
+                                                     kvgen.HEADS, kvgen.HEAD_DIM, b.pool_pages),
+                   "requests": b.n_requests, "pages": int(src.size), "bytes": 2 * sum(lens),
+                   "codebooks": "one per request", "seed": "0x%X" % (kvgen.SEED_BASE + 4),
+                   "l2": "inputs (%d MiB) exceed the 126 MB L2; no flush between steps" % ((2 * sum(lens)) >> 20)}
+        self.cfg = cfg
+        self.U = int(cfg["bytes"])
+        self.flush_l2 = self.U < 2 * L2_BYTES
+
+    def unit(self, k):
+        """Unit k (tensor or request stream) as host uint16."""
+        if self.contiguous:
+            return self.h_in[k].numpy().view(np.uint16)
+        return self.batch.request_stream(k)
+
+    def round_trip_ok(self):
+        import torch
+        if self.contiguous:
+            return bool(torch.equal(self.d_out, self.d_in))
+        return bool(torch.equal(self.pool_out[self.dst_idx], self.pool_in[self.src_idx]))
 
 
 PROFILE_FILES = {
@@ -88,21 +182,36 @@ PROFILE_FILES = {
 }
 
 
-def kernel_source_hash():
+# the sources each profiled kernel is built from
+PROFILE_SOURCES = {
+    "encode_kernel": ("sz_encode.cu", "sz_internal.cuh"),
+    "decode": ("sz_decode.cu", "sz_internal.cuh"),
+    "histogram+select": ("sz_hist.cu", "sz_internal.cuh"),
+}
+
+
+def kernel_source_hash(files=None, tree=None):
+    """sha256 (16 hex digits) of the named kernel sources, or of all of
+    them; ``tree`` maps a file name to its bytes instead of reading it."""
     import glob
     import hashlib
+    csrc = os.path.join(ROOT, "lossless_bf16_kv_splitzip_b200", "csrc")
+    names = sorted(files) if files else sorted(os.path.basename(p) for p in glob.glob(os.path.join(csrc, "*")))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "lossless_bf16_kv_splitzip_b200", "csrc", "*"))):
-        h.update(os.path.basename(p).encode())
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for name in names:
+        h.update(name.encode())
+        if tree is not None:
+            h.update(tree[name])
+        else:
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(phase, tensors, total_tensors):
     """DRAM bytes per launch from the committed ncu summary of that kernel
     (dram__bytes_read.sum + dram__bytes_write.sum, scaled from the 8-tensor
-    capture to the launch's tensor count); None when the kernel sources
+    capture to the launch's tensor count); None when that kernel's sources
     changed since the counters were taken."""
     name = PROFILE_FILES.get(phase)
     if name is None:
@@ -114,7 +223,7 @@ def profiled_traffic(phase, tensors, total_tensors):
                 if ":" in line and not line.startswith(("|", "#", " ")):
                     k, v = line.split(":", 1)
                     fields[k.strip()] = v.strip()
-        if fields.get("kernel_source_sha256") != kernel_source_hash():
+        if fields.get("kernel_source_sha256", "").split(" ")[0] != kernel_source_hash(PROFILE_SOURCES[phase]):
             return None
         return int(int(fields["traffic_per_full_launch_bytes"]) * tensors / total_tensors)
     except Exception:
@@ -183,65 +292,80 @@ class ClockSampler:
 # ------------------------------------------------------------- reference arm
 def run_reference(args):
     """The CPU oracle on bounded samples: each step encodes and decodes one
-    (layer, K/V) tensor of the workload, single-threaded."""
+    unit of the workload (a (layer, K/V) tensor, or a request), in order,
+    single-threaded."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     oracle.build()
-    cfg = workload_config()
-    n = cfg["elems_per_tensor"]
+    w = args.workload
+    if w == 4:
+        b = kvgen.paged_batch()
+        n_units = b.n_requests
+        cfg = {"workload": WORKLOAD_NAMES[4], "requests": n_units,
+               "bytes": int(2 * b.lengths.sum() * kvgen.HEADS * kvgen.HEAD_DIM)}
+        unit_of = b.request_stream
+        what = "one request's pages"
+    else:
+        cfg = workload_config(0, w)
+        n_units = cfg["tensors"]
+
+        def unit_of(i):
+            return kvgen.tiny_k_tensor() if w == 0 else kvgen.contiguous_tensor(w, i // 2, i % 2)
+        what = "one %d MiB tensor" % (cfg["elems_per_tensor"] * 2 >> 20)
     cache = {}
 
-    def tensor(i):
+    def unit(i):
         if i not in cache:
-            cache[i] = kvgen.contiguous_tensor(WORKLOAD, i // 2, i % 2)
+            cache[i] = unit_of(i)
         return cache[i]
 
-    times = []
+    times, nbytes = [], []
     for s in range(args.warmup + args.steps):
-        x = tensor(s % cfg["tensors"])
+        x = unit(s % n_units)
         t0 = time.perf_counter()
         blob = oracle.encode(x)
-        y = oracle.decode(blob, n)
+        y = oracle.decode(blob, x.size)
         dt = time.perf_counter() - t0
-        assert y[0] == x[0]
+        assert np.array_equal(y[:16], x[:16])
         if s >= args.warmup:
             times.append(dt)
+            nbytes.append(2 * x.size)
         if len(cache) > 4:
             cache.pop(next(iter(cache)))
     per_step = float(np.mean(times))
-    value = 2 * n / per_step / 1e9
+    value = float(np.sum(nbytes)) / float(np.sum(times)) / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u16", "data": "synthetic", "config": cfg,
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": "each step: oracle encode + decode of one 64 MiB (layer, K/V) tensor, "
-                                   "tensors taken in order"},
+                         "sample": "each step: oracle encode + decode of %s, units taken in order" % what},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(host_cache, seconds):
-    """The oracle as it stands (one thread) on the first tensors of the
+def cpu_baseline(inputs, seconds):
+    """The oracle as it stands (one thread) on the first units of the
     workload until about `seconds` of CPU work have run."""
     import oracle
     oracle.build()
-    n = host_cache.shape[1]
-    done, t_total = 0, 0.0
-    while done < host_cache.shape[0] and t_total < seconds:
-        x = host_cache[done].view(np.uint16)
+    done, t_total, nbytes = 0, 0.0, 0
+    while done < inputs.n_units and t_total < seconds:
+        x = inputs.unit(done)
         t0 = time.perf_counter()
         blob = oracle.encode(x)
-        oracle.decode(blob, n)
+        oracle.decode(blob, x.size)
         t_total += time.perf_counter() - t0
+        nbytes += 2 * x.size
         done += 1
-    return {"value": round(2 * n * done / t_total / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "oracle encode + decode of the first %d of %d (layer, K/V) tensors (%.1f s)"
-                      % (done, host_cache.shape[0], t_total)}
+    kind = "requests" if inputs.workload == 4 else "(layer, K/V) tensors" if inputs.workload else "tensor"
+    return {"value": round(nbytes / t_total / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "oracle encode + decode of the first %d of %d %s (%.1f s)"
+                      % (done, inputs.n_units, kind, t_total)}
 
 
 # ------------------------------------------------------------ latency sweep
@@ -415,26 +539,17 @@ def main():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    cfg = workload_config(args.tensors)
-    S, n = cfg["tensors"], cfg["elems_per_tensor"]
-    U = 2 * S * n  # uncompressed bytes per step on this rank
-
-    # inputs: generated on the host straight into pinned memory, then resident in HBM
-    h_in = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
-    host = h_in.numpy().view(np.uint16)
-    if S % 2 == 0:
-        kvgen.contiguous_cache(WORKLOAD, layers=S // 2, out=host)
-    else:
-        for k in range(S):
-            host[k] = kvgen.contiguous_tensor(WORKLOAD, k // 2, k % 2)
-    d_in = h_in.to(dev, non_blocking=False)
-    d_out = torch.empty_like(d_in)
-    plan = sz.BatchPlan([n] * S, n, device=dev)
-    in_ptrs = torch.tensor([d_in.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=dev)
-    out_ptrs = torch.tensor([d_out.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=dev)
+    inp = Inputs(args, dev, sz)
+    cfg, plan, in_ptrs, out_ptrs = inp.cfg, inp.plan, inp.in_ptrs, inp.out_ptrs
+    U = inp.U  # uncompressed bytes per step on this rank
+    seg_n = np.array(plan.seg_elems, dtype=np.int64)
+    S = plan.n_segs
     stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if inp.flush_l2 else None
 
     def step(ev=None):
+        if flush is not None:  # an input that fits L2 is flushed out of it before every step
+            flush.fill_(1)
         if ev is not None:
             ev[0].record(stream)
         plan.histogram(in_ptrs, stream)
@@ -471,6 +586,8 @@ def main():
     t_dec = np.array([e[2].elapsed_time(e[3]) for e in evs]) / 1e3
     total_s = evs[0][0].elapsed_time(evs[-1][3]) / 1e3
     ms_step = total_s / args.steps * 1e3
+    if flush is not None:  # the flushes between steps are not the codec's time
+        ms_step = float(np.mean(t_hist + t_enc + t_dec)) * 1e3
     if world > 1:
         t = torch.tensor([ms_step, t_hist.mean(), t_enc.mean(), t_dec.mean()], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -482,27 +599,28 @@ def main():
     sizes = plan.sizes.cpu().numpy().astype(np.int64)
     assert int(plan.enc_status.abs().sum()) == 0 and int(plan.dec_status.abs().sum()) == 0
     comp = int(sizes.sum())
-    esc = int(((sizes - (HEADER + n + (n + 1) // 2)) // 5).sum())
-    round_trip_ok = bool(torch.equal(d_out, d_in))
+    esc = int(((sizes - (HEADER + seg_n + (seg_n + 1) // 2)) // 5).sum())
+    round_trip_ok = inp.round_trip_ok()
 
     # ---- self-checks of the last step (bit-exactness against the oracle is
     # the parity tests' job): every tensor round-trips, and every container's
     # header states its length and escape count consistently
     hdr_ok = True
-    for k in (0, S - 1):
+    for k in sorted({0, S - 1}):
         off = int(plan.out_offset[k])
         h = plan.container[off: off + HEADER].cpu().numpy()
         hn = int(h[8:16].view(np.uint64)[0])
         he = int(h[16:24].view(np.uint64)[0])
-        hdr_ok &= bytes(h[:4]) == b"SZKV" and hn == n and HEADER + n + (n + 1) // 2 + 5 * he == int(sizes[k])
-    parity = {"decode_round_trip_all_tensors": round_trip_ok, "header_size_consistent": bool(hdr_ok)}
+        nk = int(seg_n[k])
+        hdr_ok &= bytes(h[:4]) == b"SZKV" and hn == nk and HEADER + nk + (nk + 1) // 2 + 5 * he == int(sizes[k])
+    parity = {"decode_round_trip_all_units": round_trip_ok, "header_size_consistent": bool(hdr_ok)}
 
     # ---- roofline (algorithmic bytes / event time, per phase)
     peak, peak_kind = measured_peak()
     phases = {
-        "histogram+select": (2 * S * n, th),
-        "encode_kernel": (2 * S * n + comp, te),
-        "decode": (comp + 2 * S * n, td),
+        "histogram+select": (U, th),
+        "encode_kernel": (U + comp, te),
+        "decode": (comp + U, td),
     }
     roof = {}
     for name, (b, t) in phases.items():
@@ -510,18 +628,19 @@ def main():
         roof[name] = {"achieved": round(a, 1), "frac": round(a / peak, 4), "ms": round(t * 1e3, 4),
                       "algorithmic_bytes": b}
     dom = max(phases, key=lambda k: phases[k][1])
-    enc_e2e_bytes = 2 * S * n + comp
+    enc_e2e_bytes = U + comp
     encode_s = th + te
-    layers_full = kvgen.CONTIGUOUS[WORKLOAD][0]
+    # the committed ncu summaries cover the headline workload only
+    traffic = profiled_traffic(dom, S, 2 * kvgen.CONTIGUOUS[WORKLOAD][0]) if inp.workload == WORKLOAD else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": roof[dom]["achieved"], "peak": peak, "unit": "GB/s",
-                "frac": roof[dom]["frac"], "traffic": profiled_traffic(dom, S, 2 * layers_full),
+                "frac": roof[dom]["frac"], "traffic": traffic,
                 "peak_kind": peak_kind + " (copy, MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"}
 
     # ---- one pass with the codebooks kept from the timed steps (codebook
     # reuse): the input is read once; the containers must be the same bytes
     one_pass = None
     if not args.no_one_pass:
-        plan1 = sz.BatchPlan([n] * S, n, device=dev)
+        plan1 = sz.BatchPlan(plan.seg_elems, plan.page_elems, device=dev)
         cbs = plan.codebooks.clone()
         for _ in range(3):
             plan1.encode_one_pass(in_ptrs, cbs, stream)
@@ -539,7 +658,7 @@ def main():
         torch.cuda.synchronize(dev)
         t1 = float(np.mean([a0.elapsed_time(a1) for a0, a1 in ev1])) / 1e3
         one_pass = {"encode_gbs": round(U / t1 / 1e9, 2), "ms": round(t1 * 1e3, 4),
-                    "roofline_frac": round((2 * S * n + comp) / t1 / 1e9 / peak, 4),
+                    "roofline_frac": round((U + comp) / t1 / 1e9 / peak, 4),
                     "same_containers_as_two_pass": same, "steps": k1,
                     "codebooks": "kept from the two-pass encode of the same tensors",
                     "launches": "one-pass encode, escape placement, overflow rescan"}
@@ -551,11 +670,12 @@ def main():
     # tensors, uploads and downloads on their own streams so that both
     # directions of the link stay busy while the kernels run in between.
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0:
+    if not args.no_e2e and args.e2e_steps > 0 and inp.contiguous:
         from lossless_bf16_kv_splitzip_b200.transfer import SplitZipChunks, host_round_trip
+        h_in, d_in, d_out = inp.h_in, inp.d_in, inp.d_out
         per_chunk = 4
         rt = SplitZipChunks(d_in, d_out, per_chunk, dev)
-        h_out = torch.empty((S, n), dtype=torch.int16, pin_memory=True)
+        h_out = torch.empty(tuple(h_in.shape), dtype=torch.int16, pin_memory=True)
         staging = torch.empty(comp + 4096 * S + (1 << 20), dtype=torch.uint8, pin_memory=True)
         times = []
         for it in range(args.e2e_steps + 1):
@@ -582,7 +702,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(h_in.numpy(), args.cpu_seconds)
+        cpu = cpu_baseline(inp, args.cpu_seconds)
 
     if rank == 0:
         value = world * U / (ms_step / 1e3) / 1e9
@@ -594,7 +714,7 @@ def main():
             "encode_roofline_frac": round(enc_e2e_bytes / encode_s / 1e9 / peak, 4),
             "decode_roofline_frac": roof["decode"]["frac"],
             "encode_one_pass": one_pass,
-            "ratio": round(U / comp, 5), "escape_frac": round(esc / (S * n), 6),
+            "ratio": round(U / comp, 5), "escape_frac": round(esc / (U // 2), 6),
             "roofline": roofline, "roofline_phases": roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * args.steps,  # hist, encode, esc_index, decode
             "clocks": clock_info, "parity": parity,
