@@ -21,7 +21,7 @@ using namespace sz;
 
 namespace {
 
-constexpr uint64_t kMaxElems = 0xFFFFFFFFull;  // positions are u32: n < 2^32
+constexpr uint64_t kMaxElems = 0xFFFFFFFFull;  // largest n: positions are u32, n < 2^32
 constexpr uint64_t kAlign = 256;
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
@@ -207,7 +207,7 @@ extern "C" {
 
 sz_status sz_plan(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes) {
     if (!max_compressed_bytes || !workspace_bytes) return SZ_ERR_NULL;
-    if (n_elems > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n_elems > kMaxElems) return SZ_ERR_TOO_LARGE;
     *max_compressed_bytes = SZ_MAX_BYTES(n_elems);
     *workspace_bytes = single_ws(n_elems).total;
     return SZ_OK;
@@ -216,7 +216,7 @@ sz_status sz_plan(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *wo
 sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_codebook16,
                                 uint32_t *d_hist256_or_null, void *d_ws, uint64_t ws_bytes, void *stream) {
     if (!d_codebook16 || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
-    if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
@@ -236,7 +236,7 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
                     uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
                     void *stream) {
     if (!d_codebook16 || !d_out || !d_out_bytes || !d_status || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
-    if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
     const Ws w = single_ws(n);
@@ -271,7 +271,7 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
 sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uint64_t n, int32_t *d_status,
                     void *d_ws, uint64_t ws_bytes, void *stream) {
     if (!d_in || !d_status || !d_ws || (n > 0 && !d_out)) return SZ_ERR_NULL;
-    if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
     if (!aligned16(d_in) || (n > 0 && !aligned16(d_out)) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
@@ -302,7 +302,7 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
     bool multi_page = false;
     for (uint32_t k = 0; k < n_segs; ++k) {
         const uint64_t n = h_seg_elems[k];
-        if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+        if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
         multi_page |= n > page_elems;
         h_segs[k].n_elems = n;
         h_segs[k].page_begin = pages;
@@ -402,7 +402,7 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
 
 sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes) {
     if (!max_compressed_bytes || !workspace_bytes) return SZ_ERR_NULL;
-    if (n_elems > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n_elems > kMaxElems) return SZ_ERR_TOO_LARGE;
     *max_compressed_bytes = container_size(n_elems, n_elems);
     *workspace_bytes = ws1_layout(single_batch(n_elems).n_tiles).total;
     return SZ_OK;
@@ -412,7 +412,7 @@ sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_
                              uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
                              uint64_t ws_bytes, void *stream) {
     if (!d_codebook16 || !d_out || !d_out_bytes || !d_status || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
-    if (n > kMaxElems - 1) return SZ_ERR_TOO_LARGE;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
     const Batch b = single_batch(n);

@@ -29,7 +29,7 @@ def test_library_is_built_for_sm100a():
     assert "sm_100a" in sz.sz_version()
 
 
-@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 65536, 65537, 1 << 25, (1 << 32) - 2])
+@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 65536, 65537, 1 << 25, (1 << 32) - 2, (1 << 32) - 1])
 def test_plan_worst_case_bound(n):
     cap, ws = sz.sz_plan(n)
     assert cap == 48 + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
