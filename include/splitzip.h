@@ -130,19 +130,21 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
  *                   sz_plan's max_compressed_bytes always suffices for a
  *                   codebook from sz_histogram_codebook.
  *   d_out_bytes     out: uint64 container size (0 on a device error)
- *   d_status_or_null  out: int32 device status (SZ_OK, SZ_ERR_CORRUPT when
- *                   the workspace histogram does not describe d_in,
- *                   SZ_ERR_CAPACITY, SZ_ERR_INVALID, SZ_ERR_DEVICE_TIMEOUT)
+ *   d_status        out (required): int32 device status (SZ_OK,
+ *                   SZ_ERR_CORRUPT when the workspace histogram does not
+ *                   describe d_in, SZ_ERR_CAPACITY, SZ_ERR_INVALID,
+ *                   SZ_ERR_DEVICE_TIMEOUT); set to SZ_OK first
  *   d_ws, ws_bytes  the workspace passed to sz_histogram_codebook for this
  *                   same input (its histogram gives the escape count).
- * The escape stream is compacted in element order across tiles: every
- * tile's first escape index comes from the workspace's per-tile histograms
- * (an exclusive scan of the tiles' escape counts under this codebook), so
- * no tile waits on another; a pipeline wait that runs out gives
- * SZ_ERR_DEVICE_TIMEOUT.
+ * The escape stream is compacted in element order across tiles without
+ * any block waiting for another: the histogram call kept the exponent
+ * counts of the first and last segment piece of every CTA's range of tiles,
+ * and from those each CTA's first escape index follows (placed by the
+ * histogram call for its own codebook, again here for another one).  A
+ * pipeline wait that runs out gives SZ_ERR_DEVICE_TIMEOUT.
  */
 sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
-                    uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status_or_null, void *d_ws,
+                    uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
                     uint64_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------- decode */
@@ -159,7 +161,8 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
  *                   strictly ascending, an escaped exponent that is in the
  *                   codebook, or a nonzero placeholder / odd-tail nibble.
  *                   d_out holds no meaningful data unless it reads SZ_OK.
- *   d_ws, ws_bytes  workspace of sz_plan's size (per-tile escape offsets).
+ *   d_ws, ws_bytes  workspace of sz_plan's size (the first escape index of
+ *                   every 16,384-element sub-tile, found by binary search).
  */
 sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uint64_t n,
                     int32_t *d_status, void *d_ws, uint64_t ws_bytes, void *stream);
@@ -204,7 +207,7 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
 
 /*
  * sz_histogram_codebook_batched -- exponent histogram and top-16 codebook
- * of every segment (two kernel launches for the whole batch).  The
+ * of every segment (a memset and one kernel launch for the whole batch).  The
  * codebooks and escape counts stay in the workspace for sz_encode_batched.
  *   d_segs          the table from sz_plan_batched, in device memory
  *   n_tiles         from sz_plan_batched
