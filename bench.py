@@ -370,7 +370,8 @@ def cpu_baseline(inputs, seconds):
 
 # ------------------------------------------------------------ latency sweep
 def run_sweep(args):
-    """Encode (histogram + codebook + container) and decode latency of one
+    """Encode (histogram + codebook + container: sz_compress, and the
+    two-call sz_histogram_codebook + sz_encode) and decode latency of one
     stream through the single-stream C ABI, for power-of-two sizes from
     64 KiB to 4 GiB.  A stream of b bytes is the first b bytes of the
     workload's buffer ([layer][K,V][head][token][dim]), coded as one stream
@@ -413,36 +414,45 @@ def run_sweep(args):
         x = d_flat[:n]
         c_cap, w_need = sz.sz_plan(n)
         with torch.cuda.stream(stream):
-            def enc():
+            def enc():  # one call: histogram, codebook and container
+                sz.sz_compress(x, n, out, c_cap, size, cb, est, ws, w_need, stream)
+
+            def enc2():  # the two-call path
                 sz.sz_histogram_codebook(x, n, cb, None, ws, w_need, stream)
                 sz.sz_encode(x, n, cb, out, c_cap, size, est, ws, w_need, stream)
 
             def dcd():
                 sz.sz_decode(out, c_cap, dec, n, dst, ws, w_need, stream)
 
-            enc(); dcd()
-            g_enc, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            enc2(); enc(); dcd()
+            g_enc, g_enc2, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_enc2, stream=stream):
+                enc2()
             with torch.cuda.graph(g_enc, stream=stream):
                 enc()
             with torch.cuda.graph(g_dec, stream=stream):
                 dcd()
-            te, td = [], []
+            te, te2, td = [], [], []
             for _ in range(3 + args.sweep_reps):
-                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
                 flush.fill_(1)
+                ev[4].record(stream); g_enc2.replay(); ev[5].record(stream)
+                flush.fill_(3)
                 ev[0].record(stream); g_enc.replay(); ev[1].record(stream)
                 flush.fill_(2)
                 ev[2].record(stream); g_dec.replay(); ev[3].record(stream)
                 stream.synchronize()
                 te.append(ev[0].elapsed_time(ev[1]) / 1e3)
+                te2.append(ev[4].elapsed_time(ev[5]) / 1e3)
                 td.append(ev[2].elapsed_time(ev[3]) / 1e3)
-            te, td = float(np.median(te[3:])), float(np.median(td[3:]))
+            te, te2, td = float(np.median(te[3:])), float(np.median(te2[3:])), float(np.median(td[3:]))
             assert int(est.item()) == 0 and int(dst.item()) == 0, (b, int(est.item()), int(dst.item()))
             comp = int(size.item())
             ok = bool(torch.equal(dec[:n], x))
-            del g_enc, g_dec
+            del g_enc, g_enc2, g_dec
         line = {"sweep": "single stream, first bytes of llama3-8b-kv-32k", "bytes": b, "elems": n,
-                "encode_us": round(te * 1e6, 2), "decode_us": round(td * 1e6, 2),
+                "encode_us": round(te * 1e6, 2), "encode_two_call_us": round(te2 * 1e6, 2),
+                "decode_us": round(td * 1e6, 2),
                 "encode_gbs": round(b / te / 1e9, 2), "decode_gbs": round(b / td / 1e9, 2),
                 "encode_roofline_frac": round((b + comp) / te / 1e9 / peak, 4),
                 "decode_roofline_frac": round((b + comp) / td / 1e9 / peak, 4),

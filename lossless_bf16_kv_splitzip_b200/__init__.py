@@ -72,6 +72,7 @@ def lib():
             "sz_encode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, vp, u64, vp],
             "sz_decode_batched": [u32, vp, u64, vp, u64, vp, u64, vp, vp, u64, vp],
             "sz_encode_static": [vp, u64, vp, u64, vp, vp, vp, vp],
+            "sz_compress": [vp, u64, vp, u64, vp, vp, vp, vp, u64, vp],
             "sz_plan_one_pass": [u64, pu64, pu64],
             "sz_encode_one_pass": [vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
             "sz_workspace_one_pass_batched": [u32, u64, pu64],
@@ -140,6 +141,11 @@ def sz_histogram_codebook(d_in, n, d_codebook16, d_hist256=None, d_ws=None, ws_b
 def sz_encode(d_in, n, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, ws_bytes, stream=None):
     _check(lib().sz_encode(_p(d_in), n, _p(d_codebook16), _p(d_out), out_cap, _p(d_out_bytes), _p(d_status),
                            _p(d_ws), ws_bytes, _s(stream)), "sz_encode")
+
+
+def sz_compress(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16, d_status, d_ws, ws_bytes, stream=None):
+    _check(lib().sz_compress(_p(d_in), n, _p(d_out), out_cap, _p(d_out_bytes), _p(d_codebook16), _p(d_status),
+                             _p(d_ws), ws_bytes, _s(stream)), "sz_compress")
 
 
 def sz_decode(d_in, in_bytes, d_out, n, d_status, d_ws, ws_bytes, stream=None):
@@ -262,6 +268,23 @@ def encode(x, stream=None, workspace=None):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     sz_histogram_codebook(x, n, cb, None, ws, wsb, stream)
     sz_encode(x, n, cb, out, cap, size, status, ws, wsb, stream)
+    return out, size, status
+
+
+def compress(x, stream=None, workspace=None, codebook=None):
+    """Histogram, codebook and container of a contiguous 16-bit CUDA tensor
+    in one call (one launch up to 32,768 elements).  Returns (container,
+    size int64 tensor [1], status int32 tensor [1])."""
+    torch = _torch()
+    x = _u16_view(x.contiguous())
+    n = x.numel()
+    cap, wsb = sz_plan(n)
+    dev = x.device
+    ws = workspace if workspace is not None else torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    size = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sz_compress(x, n, out, cap, size, codebook, status, ws, ws.numel(), stream)
     return out, size, status
 
 

@@ -12,6 +12,10 @@ cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_encode_one_pass(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_place(const PlaceArgs &a, bool batched, int sms, cudaStream_t s);
+cudaError_t launch_tiny_encode(const uint16_t *in, uint64_t n, uint8_t *out, uint64_t out_cap, uint64_t *out_bytes,
+                               uint8_t *codebook_out, int32_t *status, cudaStream_t s);
+cudaError_t launch_tiny_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
+                               cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
@@ -23,6 +27,7 @@ namespace {
 
 constexpr uint64_t kMaxElems = 0xFFFFFFFFull;  // largest n: positions are u32, n < 2^32
 constexpr uint64_t kAlign = 256;
+constexpr uint64_t kTinyEncodeMax = 32768;  // sz_compress: one block up to this many elements
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<uint32_t> g_debug_flags{0};
@@ -275,9 +280,10 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     if (!aligned16(d_in) || (n > 0 && !aligned16(d_out)) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (n <= kTile) return cuda_status(launch_tiny_decode(d_in, in_bytes, d_out, n, d_status, s));  // one launch
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
     DecodeArgs a{};
     a.batch = single_batch(n);
@@ -290,6 +296,44 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     a.debug_flags = g_debug_flags.load();
     SZ_TRY_CUDA(launch_esc_index(a, false, s));
     return cuda_status(launch_decode(a, false, dev.sms * dev.dec_occ, s));
+}
+
+sz_status sz_compress(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap, uint64_t *d_out_bytes,
+                      uint8_t *d_codebook16_or_null, int32_t *d_status, void *d_ws, uint64_t ws_bytes, void *stream) {
+    if (!d_out || !d_out_bytes || !d_status || !d_ws || (n > 0 && !d_in)) return SZ_ERR_NULL;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
+    if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
+    const Ws w = single_ws(n);
+    if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // one block, one launch: measured faster up to 32,768 elements (22.6 vs
+    // 26.6 us at 64 KiB), slower at a full tile (36.9 vs 32.8 us at 128 KiB)
+    if (n <= kTinyEncodeMax)
+        return cuda_status(launch_tiny_encode(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, s));
+    DeviceInfo dev;
+    if (!device_info(dev)) return SZ_ERR_CUDA;
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 + 4, s));  // seg_hist, seg_done
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
+    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
+    SelectCtx c = select_ctx(single_batch(n), d_ws, w, dev);
+    c.codebooks_out = d_codebook16_or_null;
+    HistArgs h = hist_args(c, d_ws, w);
+    h.base = d_in;
+    SZ_TRY_CUDA(launch_hist(h, false, s));
+    EncodeArgs a{};  // the codebook the histogram kernel chose: no reselect
+    a.batch = c.batch;
+    a.base = d_in;
+    a.out = d_out;
+    a.out_cap = out_cap;
+    a.out_bytes = d_out_bytes;
+    a.status = d_status;
+    a.meta = c.meta;
+    a.rrec = c.rrec;
+    a.range_tiles = c.range_tiles;
+    a.wait_limit_ns = g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    return cuda_status(launch_encode(a, false, s));
 }
 
 sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t page_elems, sz_segment *h_segs,

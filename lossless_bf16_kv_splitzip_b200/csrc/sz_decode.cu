@@ -469,6 +469,88 @@ __global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArg
     }
 }
 
+// ----------------------------------------------------------- small streams
+// A stream of at most one tile (65,536 elements) in one launch of one block:
+// no sub-tile index kernel and no memset.  Thread t decodes chunks t,
+// t + 256, ... straight from the container and stores them; after one
+// barrier (every placeholder value is stored) one thread per escape record
+// checks it -- inside the stream, after its predecessor, exponent outside
+// the codebook, placeholder nibble 0 -- and overwrites its value.  The same
+// checks as the large path, so the same containers are accepted.
+__global__ void __launch_bounds__(kThreads) tiny_decode_kernel(const uint8_t *c, uint64_t cap, uint16_t *out,
+                                                               uint64_t n, int32_t *status) {
+    const uint32_t tid = threadIdx.x;
+    if (tid == 0) *status = SZ_OK;
+    __syncthreads();
+    const Header h = read_header(c, cap, n);
+    if (!h.ok) {
+        if (tid == 0) set_status(status, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
+        return;
+    }
+    const DecTables T = make_tables(h.cb_lo, h.cb_hi);
+    const uint8_t *sm = c + kHeader;
+    const uint8_t *codes = c + kHeader + n;
+    const uint32_t nn = (uint32_t)n;  // at most 65,536
+    for (uint32_t off = tid * kChunk; off < nn; off += kThreads * kChunk) {
+        const uint32_t cnt = umin32(kChunk, nn - off);
+        uint4 smv;
+        uint64_t cw = 0;
+        if (cnt == (uint32_t)kChunk && (n % 8) == 0) {
+            smv = *reinterpret_cast<const uint4 *>(sm + off);
+            cw = *reinterpret_cast<const unsigned long long *>(codes + off / 2);
+        } else {
+            uint32_t sw[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                if (j < (int)cnt) sw[j >> 2] |= (uint32_t)sm[off + j] << (8 * (j & 3));
+            smv = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+#pragma unroll
+            for (int b = 0; b < kChunk / 2; ++b)
+                if (2 * b < (int)cnt) cw |= (uint64_t)codes[off / 2 + b] << (8 * b);
+            if ((cnt & 1) && ((cw >> (4 * cnt)) & 0xFu) != 0) set_status(status, SZ_ERR_CORRUPT);  // odd tail
+            if (cnt < (uint32_t)kChunk) cw &= (1ull << (4 * cnt)) - 1ull;
+        }
+        uint4 o0, o1;
+        decode_chunk(smv, cw, T, o0, o1);
+        if (cnt == (uint32_t)kChunk) {
+            st_stream_v4(out + off, o0);
+            st_stream_v4(out + off + 8, o1);
+        } else {
+            const uint32_t w[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+            for (int j = 0; j < kChunk; ++j)
+                if (j < (int)cnt) out[off + j] = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
+        }
+    }
+    __syncthreads();
+    uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+        const uint32_t x = cb_entry(h.cb_lo, h.cb_hi, q);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cbset[i] |= ((x >> 5) == (uint32_t)i) ? (1u << (x & 31)) : 0u;
+    }
+    const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
+    const uint8_t *raw = pos + 4 * h.e;
+    for (uint64_t i = tid; i < h.e; i += kThreads) {
+        const uint64_t p = load_u32_any(pos + 4 * i);
+        const uint32_t x = raw[i];
+        bool bad = p >= n || in_set8(cbset, x) || (i > 0 && load_u32_any(pos + 4 * (i - 1)) >= p);
+        if (!bad && ((codes[p >> 1] >> (4 * (p & 1))) & 0xFu) != 0) bad = true;  // placeholder must be 0
+        if (!bad) {
+            const uint32_t smb = sm[p];
+            out[p] = (uint16_t)(((smb & 0x80u) << 8) | (x << 7) | (smb & 0x7Fu));
+        }
+        if (bad) set_status(status, SZ_ERR_CORRUPT);
+    }
+}
+
+cudaError_t launch_tiny_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
+                               cudaStream_t s) {
+    tiny_decode_kernel<<<1, kThreads, 0, s>>>(c, cap, out, n, status);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {
     const uint64_t entries = kSubsPerTile * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
     const uint64_t grid = div_up(entries, 256);

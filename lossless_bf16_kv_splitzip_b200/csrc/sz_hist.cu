@@ -340,11 +340,4 @@ cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-int hist_blocks_per_sm() {
-    int occ = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, hist_kernel<true, false>, kThreads,
-                                                  kHistWords * sizeof(uint32_t));
-    return occ > 0 ? occ : 1;
-}
-
 }  // namespace sz

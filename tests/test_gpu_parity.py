@@ -268,7 +268,9 @@ def corruptions(blob, n):
     return out
 
 
-@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11])
+# sizes up to one tile take the one-block decode, larger ones the
+# index + pipelined decode: both must reject every corruption
+@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11, 65536 + 3001, 3 * 65536 + 16 * 17])
 def test_corrupt_containers_rejected(n):
     x = kvgen.mixed_small(n, seed=21 + n)
     blob = gpu_encode(x)
@@ -285,6 +287,42 @@ def test_odd_tail_nibble_rejected():
     c = bytearray(gpu_encode(x))
     c[H + 3 + 1] |= 0x10
     assert gpu_decode(bytes(c), 3)[0] == sz.SZ_ERR_CORRUPT
+    n = 2 * 65536 + 1001  # the pipelined decode's path
+    x = kvgen.mixed_small(n, seed=23)
+    c = bytearray(gpu_encode(x))
+    c[H + n + (n + 1) // 2 - 1] |= 0x10  # high nibble of the last code byte
+    assert gpu_decode(bytes(c), n)[0] == sz.SZ_ERR_CORRUPT
+
+
+# -------------------------------------------------- one-call compression
+@pytest.mark.parametrize("n", [0, 1, 17, 4095, 16385, 32767, 32768, 32769, 65537, 3 * 65536 + 100, 262147])
+def test_compress_one_call_equals_oracle(n):
+    """sz_compress: one block and one launch up to 32,768 elements, the
+    histogram and encode kernels beyond; the same bytes as the oracle (and
+    as the two-call path), and the codebook it reports is the header's."""
+    x = kvgen.mixed_small(n, seed=300 + n % 101)
+    cb = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    out, size, status = sz.compress(to_dev(x), codebook=cb)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = out[: int(size.item())].cpu().numpy().tobytes()
+    assert got == oracle.encode(x)
+    assert bytes(cb.cpu().numpy()) == got[24:40]
+
+
+@pytest.mark.parametrize("n", [30000, 70000])  # the one-block path and the kernels' path
+def test_compress_capacity_checked_on_device(n):
+    x = kvgen.uniform_u16(n, seed=301)  # incompressible: many escapes
+    d = to_dev(x)
+    cap, wsb = sz.sz_plan(x.size)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=DEV)
+    small = H + x.size + (x.size + 1) // 2 + 64
+    out = torch.empty(small, dtype=torch.uint8, device=DEV)
+    size = torch.ones(1, dtype=torch.int64, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sz.sz_compress(d, x.size, out, small, size, None, st, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(st.item()) == sz.SZ_ERR_CAPACITY and int(size.item()) == 0
 
 
 # -------------------------------------------------------- bounded waits
