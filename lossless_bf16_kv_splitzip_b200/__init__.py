@@ -273,7 +273,7 @@ def encode(x, stream=None, workspace=None):
 
 def compress(x, stream=None, workspace=None, codebook=None):
     """Histogram, codebook and container of a contiguous 16-bit CUDA tensor
-    in one call (one launch up to 32,768 elements).  Returns (container,
+    in one call (two launches up to 2^21 elements).  Returns (container,
     size int64 tensor [1], status int32 tensor [1])."""
     torch = _torch()
     x = _u16_view(x.contiguous())

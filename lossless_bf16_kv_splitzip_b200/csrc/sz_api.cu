@@ -12,10 +12,10 @@ cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_encode_one_pass(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_place(const PlaceArgs &a, bool batched, int sms, cudaStream_t s);
-cudaError_t launch_tiny_encode(const uint16_t *in, uint64_t n, uint8_t *out, uint64_t out_cap, uint64_t *out_bytes,
-                               uint8_t *codebook_out, int32_t *status, cudaStream_t s);
-cudaError_t launch_tiny_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
-                               cudaStream_t s);
+cudaError_t launch_small_encode(const uint16_t *in, uint64_t n, const SmallWs &w, uint8_t *out, uint64_t out_cap,
+                                uint64_t *out_bytes, uint8_t *codebook_out, int32_t *status, cudaStream_t s);
+cudaError_t launch_small_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
+                                cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
@@ -27,7 +27,8 @@ namespace {
 
 constexpr uint64_t kMaxElems = 0xFFFFFFFFull;  // largest n: positions are u32, n < 2^32
 constexpr uint64_t kAlign = 256;
-constexpr uint64_t kTinyEncodeMax = 32768;  // sz_compress: one block up to this many elements
+constexpr uint64_t kSmallEncodeMax = 1ull << 21;  // sz_compress: 4,096-element blocks up to this many elements (measured crossover 4-8 MiB)
+constexpr uint64_t kSmallDecodeMax = 1ull << 21;  // sz_decode: one launch of 4,096-element blocks up to this (measured crossover 4-8 MiB)
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<uint32_t> g_debug_flags{0};
@@ -125,7 +126,28 @@ Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, ui
     return b;
 }
 
-Ws single_ws(uint64_t n) { return ws_layout(1, single_batch(n).n_tiles); }
+// ---- sz_compress's short-stream scratch, for S = ceil(n / 4096) slices
+//   [0, 1024) stream counts, [1024, 1028) slices counted, [1028, 1032)
+//   slices encoded (zeroed together), [1280, 1312) SegMeta, [1536, ...)
+//   first escape index per slice, then u32[S][256] counts per slice
+struct WsSmall {
+    uint64_t meta, block_off, block_hist, total;
+};
+WsSmall small_layout(uint64_t n) {
+    const uint64_t nb = umax64(1, div_up(n, (uint64_t)kThreads * kChunk));
+    WsSmall w;
+    w.meta = 1280;
+    w.block_off = 1536;
+    w.block_hist = round_up(w.block_off + 4 * nb, kAlign);
+    w.total = round_up(w.block_hist + 1024 * nb, kAlign);
+    return w;
+}
+
+Ws single_ws(uint64_t n) {
+    Ws w = ws_layout(1, single_batch(n).n_tiles);
+    if (n <= kSmallEncodeMax) w.total = umax64(w.total, small_layout(n).total);
+    return w;
+}
 
 template <class T>
 T *at(void *ws, uint64_t off) {
@@ -281,10 +303,10 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (n <= kTile) return cuda_status(launch_tiny_decode(d_in, in_bytes, d_out, n, d_status, s));  // one launch
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
+    if (n <= kSmallDecodeMax) return cuda_status(launch_small_decode(d_in, in_bytes, d_out, n, d_status, s));
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
     DecodeArgs a{};
     a.batch = single_batch(n);
     a.base = d_out;
@@ -307,10 +329,19 @@ sz_status sz_compress(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // one block, one launch: measured faster up to 32,768 elements (22.6 vs
-    // 26.6 us at 64 KiB), slower at a full tile (36.9 vs 32.8 us at 128 KiB)
-    if (n <= kTinyEncodeMax)
-        return cuda_status(launch_tiny_encode(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, s));
+    if (n <= kSmallEncodeMax) {  // short stream: one memset, two launches over 4,096-element slices
+        const WsSmall ws = small_layout(n);
+        SZ_TRY_CUDA(cudaMemsetAsync(d_ws, 0, 1032, s));
+        SmallWs sw;
+        sw.seg_hist = at<uint32_t>(d_ws, 0);
+        sw.done = at<uint32_t>(d_ws, 1024);
+        sw.done2 = at<uint32_t>(d_ws, 1028);
+        sw.meta = at<SegMeta>(d_ws, ws.meta);
+        sw.block_off = at<uint32_t>(d_ws, ws.block_off);
+        sw.block_hist = at<uint32_t>(d_ws, ws.block_hist);
+        return cuda_status(
+            launch_small_encode(d_in, n, sw, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, s));
+    }
     DeviceInfo dev;
     if (!device_info(dev)) return SZ_ERR_CUDA;
     SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 + 4, s));  // seg_hist, seg_done

@@ -470,29 +470,46 @@ __global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArg
 }
 
 // ----------------------------------------------------------- small streams
-// A stream of at most one tile (65,536 elements) in one launch of one block:
-// no sub-tile index kernel and no memset.  Thread t decodes chunks t,
-// t + 256, ... straight from the container and stores them; after one
-// barrier (every placeholder value is stored) one thread per escape record
-// checks it -- inside the stream, after its predecessor, exponent outside
-// the codebook, placeholder nibble 0 -- and overwrites its value.  The same
-// checks as the large path, so the same containers are accepted.
-__global__ void __launch_bounds__(kThreads) tiny_decode_kernel(const uint8_t *c, uint64_t cap, uint16_t *out,
-                                                               uint64_t n, int32_t *status) {
+// A short stream decoded by a grid of blocks in one launch, without the
+// sub-tile index kernel: block b decodes elements [b*S, (b+1)*S) (S a
+// multiple of 16), thread t chunks t, t + 256, ... straight from the
+// container, and after one barrier (every placeholder value stored) checks
+// and patches the escape records of its slice.  Its records [lo, hi) come
+// from two binary searches, the block's end search being the next block's
+// start search, so the slices tile [0, e): the last block checks hi = e, a
+// block with hi < lo reports it, and every record is checked against its
+// predecessor -- the large path's checks, on the same containers.  The
+// status word is set to SZ_OK by the caller's memset.
+constexpr uint32_t kSmallSlice = 4096;  // elements per block
+
+__device__ __forceinline__ uint64_t lower_pos(const uint8_t *pos, uint64_t e, uint64_t key) {
+    uint64_t lo = 0, hi = e;  // first record with position >= key
+    while (lo < hi) {
+        const uint64_t mid = (lo + hi) >> 1;
+        if (load_u32_any(pos + 4 * mid) < key) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(kThreads) small_decode_kernel(const uint8_t *c, uint64_t cap, uint16_t *out,
+                                                                uint64_t n, uint32_t slice, int32_t *status) {
+    __shared__ uint64_t s_range[2];
     const uint32_t tid = threadIdx.x;
-    if (tid == 0) *status = SZ_OK;
-    __syncthreads();
     const Header h = read_header(c, cap, n);
     if (!h.ok) {
-        if (tid == 0) set_status(status, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
+        if (tid == 0 && blockIdx.x == 0) set_status(status, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
         return;
     }
-    const DecTables T = make_tables(h.cb_lo, h.cb_hi);
+    const uint64_t first = (uint64_t)blockIdx.x * slice;
+    const uint64_t last = umin64(first + slice, n);
     const uint8_t *sm = c + kHeader;
     const uint8_t *codes = c + kHeader + n;
-    const uint32_t nn = (uint32_t)n;  // at most 65,536
-    for (uint32_t off = tid * kChunk; off < nn; off += kThreads * kChunk) {
-        const uint32_t cnt = umin32(kChunk, nn - off);
+    const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
+    const uint8_t *raw = pos + 4 * h.e;
+    if (tid < 2) s_range[tid] = (tid == 0) ? lower_pos(pos, h.e, first) : lower_pos(pos, h.e, last);
+    const DecTables T = make_tables(h.cb_lo, h.cb_hi);
+    for (uint64_t off = first + tid * kChunk; off < last; off += kThreads * kChunk) {
+        const uint32_t cnt = (uint32_t)umin64(kChunk, n - off);
         uint4 smv;
         uint64_t cw = 0;
         if (cnt == (uint32_t)kChunk && (n % 8) == 0) {
@@ -522,7 +539,10 @@ __global__ void __launch_bounds__(kThreads) tiny_decode_kernel(const uint8_t *c,
                 if (j < (int)cnt) out[off + j] = (uint16_t)(w[j >> 1] >> (16 * (j & 1)));
         }
     }
-    __syncthreads();
+    __syncthreads();  // the block's values stored; the searches done
+    const uint64_t lo = s_range[0], hi = s_range[1];
+    if (tid == 0 && (hi < lo || (last == n && hi != h.e))) set_status(status, SZ_ERR_CORRUPT);
+    if (hi < lo) return;
     uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
@@ -530,12 +550,10 @@ __global__ void __launch_bounds__(kThreads) tiny_decode_kernel(const uint8_t *c,
 #pragma unroll
         for (int i = 0; i < 8; ++i) cbset[i] |= ((x >> 5) == (uint32_t)i) ? (1u << (x & 31)) : 0u;
     }
-    const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
-    const uint8_t *raw = pos + 4 * h.e;
-    for (uint64_t i = tid; i < h.e; i += kThreads) {
+    for (uint64_t i = lo + tid; i < hi; i += kThreads) {
         const uint64_t p = load_u32_any(pos + 4 * i);
         const uint32_t x = raw[i];
-        bool bad = p >= n || in_set8(cbset, x) || (i > 0 && load_u32_any(pos + 4 * (i - 1)) >= p);
+        bool bad = p < first || p >= last || in_set8(cbset, x) || (i > 0 && load_u32_any(pos + 4 * (i - 1)) >= p);
         if (!bad && ((codes[p >> 1] >> (4 * (p & 1))) & 0xFu) != 0) bad = true;  // placeholder must be 0
         if (!bad) {
             const uint32_t smb = sm[p];
@@ -545,9 +563,10 @@ __global__ void __launch_bounds__(kThreads) tiny_decode_kernel(const uint8_t *c,
     }
 }
 
-cudaError_t launch_tiny_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
-                               cudaStream_t s) {
-    tiny_decode_kernel<<<1, kThreads, 0, s>>>(c, cap, out, n, status);
+cudaError_t launch_small_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
+                                cudaStream_t s) {
+    const uint64_t blocks = umax64(1, div_up(n, kSmallSlice));
+    small_decode_kernel<<<(unsigned)blocks, kThreads, 0, s>>>(c, cap, out, n, kSmallSlice, status);
     return cudaGetLastError();
 }
 

@@ -595,43 +595,51 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
 }
 
 // ----------------------------------------------------------- small streams
-// A stream of at most one tile (65,536 elements) compressed by one block in
-// one launch: exponent counts in lane-private shared columns (bank = lane),
-// the top-16 select (rank by count descending, exponent ascending), then the
-// container -- the input read a second time, from L2.  Escape records go
-// out in element order: per round of 256 chunks an exclusive scan of the
-// threads' escape counts places each thread's records.
-constexpr uint32_t kTinyColWords = 256 * 32;
+constexpr uint32_t kTinyColWords = 256 * 32;  // exponent counts: 256 bins x 32 lane columns
 
-__global__ void __launch_bounds__(kThreads) tiny_encode_kernel(const uint16_t *in, uint64_t n, uint8_t *out,
-                                                               uint64_t out_cap, uint64_t *out_bytes,
-                                                               uint8_t *codebook_out, int32_t *status) {
+// A short stream over a grid of blocks, each one 4,096-element slice (one
+// chunk per thread), in two launches after one memset: the counting kernel
+// keeps every slice's 256 exponent counts and adds them to the stream's;
+// the block that completes the count (one atomic completion count, no
+// wait) selects the top 16 and turns the slices' counts into each slice's
+// first escape index.  The encode kernel then writes every slice's bytes
+// and records in place; its last block to finish writes the size if no
+// block reported an error.  status and size are reset by the first kernel.
+constexpr uint32_t kSlice = kThreads * kChunk;  // 4,096 elements per block
+
+__global__ void __launch_bounds__(kThreads) small_hist_kernel(const uint16_t *in, uint64_t n, SmallWs w,
+                                                              uint8_t *codebook_out, int32_t *status,
+                                                              uint64_t *out_bytes) {
     extern __shared__ __align__(16) uint32_t s_col[];  // kTinyColWords
     __shared__ uint32_t s_cnt[256];
     __shared__ uint32_t s_warp[kWarps];
+    __shared__ uint32_t s_carry;
     __shared__ uint8_t s_cb[16];
     __shared__ unsigned long long s_top;
+    __shared__ int s_last;
     const uint32_t tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const uint32_t nn = (uint32_t)n;  // at most 65,536
+    const uint32_t nb = (uint32_t)umax64(1, div_up(n, kSlice));  // an empty stream: one block
     for (uint32_t i = tid; i < kTinyColWords; i += kThreads) s_col[i] = 0;
     if (tid == 0) {
-        *status = SZ_OK;
-        *out_bytes = 0;
+        if (blockIdx.x == 0) {
+            *status = SZ_OK;
+            *out_bytes = 0;
+        }
         s_top = 0;
+        s_carry = 0;
     }
     __syncthreads();
-
-    // ---- exponent counts
+    const uint64_t off = (uint64_t)blockIdx.x * kSlice + tid * kChunk;
     const uint32_t col = smem_u32(s_col) + lane * 4;
-    for (uint32_t off = tid * kChunk; off < nn; off += kThreads * kChunk) {
-        const uint32_t cnt = umin32(kChunk, nn - off);
+    if (off < n) {
+        const uint32_t cnt = (uint32_t)umin64(kChunk, n - off);
         if (cnt == (uint32_t)kChunk) {
             const uint4 v0 = ld_stream_v4(in + off), v1 = ld_stream_v4(in + off + 8);
-            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const uint32_t x[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
             for (int q = 0; q < 8; ++q) {  // (half & 0x7F80) = exponent * 128 = the byte offset of its row
-                asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(col + (w[q] & 0x7F80u)) : "memory");
-                asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(col + ((w[q] >> 16) & 0x7F80u)) : "memory");
+                asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(col + (x[q] & 0x7F80u)) : "memory");
+                asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(col + ((x[q] >> 16) & 0x7F80u)) : "memory");
             }
         } else {
             for (uint32_t j = 0; j < cnt; ++j)
@@ -642,8 +650,17 @@ __global__ void __launch_bounds__(kThreads) tiny_encode_kernel(const uint16_t *i
     uint32_t c = 0;
 #pragma unroll 8
     for (uint32_t i = 0; i < 32; ++i) c += s_col[tid * 32 + ((i + tid) & 31)];
+    w.block_hist[(size_t)blockIdx.x * 256 + tid] = c;
+    if (c) atomicAdd(&w.seg_hist[tid], c);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(w.done, 1u) + 1 == nb;
+    __syncthreads();
+    if (!s_last) return;
+    // ---- the last block: select, escape count, first escape index per slice
+    __threadfence();
+    c = __ldcg(w.seg_hist + tid);
     s_cnt[tid] = c;
-    s_lut[tid] = 0x80;
     __syncthreads();
     uint32_t rank = 0;
 #pragma unroll 8
@@ -653,75 +670,31 @@ __global__ void __launch_bounds__(kThreads) tiny_encode_kernel(const uint16_t *i
     }
     if (rank < 16) {
         s_cb[rank] = (uint8_t)tid;
-        s_lut[tid] = (uint8_t)rank;
         atomicAdd(&s_top, (unsigned long long)c);
     }
     __syncthreads();
-    const uint64_t e_total = n - s_top;
-    if (container_size(n, e_total) > out_cap) {
-        if (tid == 0) *status = SZ_ERR_CAPACITY;
-        return;
+    if (tid < 16) {
+        w.meta->codebook[tid] = s_cb[tid];
+        if (codebook_out) codebook_out[tid] = s_cb[tid];
     }
-    if (tid < 16 && codebook_out) codebook_out[tid] = s_cb[tid];
-    if (tid < 6) {
-        uint64_t v = 0;
-        if (tid == 0) v = 0x00000101564B5A53ull;  // "SZKV", version 1, dtype 1, flags 0
-        if (tid == 1) v = n;
-        if (tid == 2) v = e_total;
-        if (tid == 3 || tid == 4)
-            for (int i = 7; i >= 0; --i) v = (v << 8) | s_cb[8 * (tid - 3) + i];
-        reinterpret_cast<uint64_t *>(out)[tid] = v;
+    if (tid == 0) {
+        w.meta->n_escapes = n - s_top;
+        w.meta->valid = 1;
+        w.meta->pad = 0;
     }
-
-    // ---- container: sm and code streams, escape records in element order
-    const bool codes_aligned = (n % 8) == 0;
-    const uint64_t pos_off = kHeader + n + (n + 1) / 2;
-    const bool pos_aligned = (pos_off & 3) == 0;
-    uint8_t *out_sm = out + kHeader;
-    uint8_t *codes = out + kHeader + n;
-    uint8_t *pos = out + pos_off;
-    uint8_t *raw = pos + 4 * e_total;
-    uint32_t done = 0;
-    for (uint32_t base = 0; base < nn; base += kThreads * kChunk) {
-        const uint32_t off = base + tid * kChunk;
-        uint32_t esc = 0, cnt = 0;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-        if (off < nn) {
-            cnt = umin32(kChunk, nn - off);
-            if (cnt == (uint32_t)kChunk) {
-                v0 = ld_stream_v4(in + off);
-                v1 = ld_stream_v4(in + off + 8);
-            } else {
-                read_chunk_global(in + off, cnt, v0, v1);
-            }
-            uint4 smv;
-            uint64_t cw;
-            uint32_t m;
-            encode_chunk(v0, v1, smv, cw, m);
-            uint32_t keep = 0;
+    uint32_t cbq[16];
 #pragma unroll
-            for (int q = 0; q < kChunk; ++q)
-                if (q < (int)cnt) keep |= esc_bit_of_elem(q);
-            esc = esc_in_element_order(m & keep);
-            if (cnt < (uint32_t)kChunk) cw &= (1ull << (4 * cnt)) - 1ull;  // odd tail nibble = 0
-            if (cnt == (uint32_t)kChunk) {
-                st_stream_v4(out_sm + off, smv);
-            } else {
+    for (int q = 0; q < 16; ++q) cbq[q] = s_cb[q];
+    for (uint32_t base = 0; base < nb; base += kThreads) {
+        const uint32_t b = base + tid;
+        uint32_t esc = 0;
+        if (b < nb) {
+            uint32_t in_cb = 0;
 #pragma unroll
-                for (int q = 0; q < kChunk; ++q)
-                    if (q < (int)cnt) out_sm[off + q] = (uint8_t)byte_of(smv, q);
-            }
-            if (cnt == (uint32_t)kChunk && codes_aligned) {
-                st_stream_u64(codes + off / 2, cw);
-            } else {
-#pragma unroll
-                for (int b = 0; b < kChunk / 2; ++b)
-                    if (2 * b < (int)cnt) codes[off / 2 + b] = (uint8_t)(cw >> (8 * b));
-            }
+            for (int q = 0; q < 16; ++q) in_cb += __ldcg(w.block_hist + (size_t)b * 256 + cbq[q]);
+            esc = (uint32_t)umin64(kSlice, n - (uint64_t)b * kSlice) - in_cb;
         }
-        // exclusive scan of the threads' escape counts, in thread order
-        const uint32_t k = __popc(esc);
-        uint32_t incl = k;
+        uint32_t incl = esc;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
@@ -731,39 +704,135 @@ __global__ void __launch_bounds__(kThreads) tiny_encode_kernel(const uint16_t *i
         __syncthreads();
         uint32_t before = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const uint32_t x = s_warp[w];
-            before += ((uint32_t)w < wid) ? x : 0u;
+        for (int q = 0; q < kWarps; ++q) {
+            const uint32_t x = s_warp[q];
+            before += ((uint32_t)q < wid) ? x : 0u;
             total += x;
         }
+        const uint32_t carry = s_carry;
+        if (b < nb) w.block_off[b] = carry + before + incl - esc;
         __syncthreads();
-        uint32_t g = done + before + incl - k;
-        while (esc) {
-            const int q = __ffs(esc) - 1;
-            esc &= esc - 1;
-            const uint32_t x = (q < 8) ? ((q < 4) ? (q < 2 ? v0.x : v0.y) : (q < 6 ? v0.z : v0.w))
-                                       : ((q < 12) ? (q < 10 ? v1.x : v1.y) : (q < 14 ? v1.z : v1.w));
-            const uint32_t val = (x >> (16 * (q & 1))) & 0xFFFFu;
-            if (g < e_total) {
-                store_u32_le(pos + 4 * (uint64_t)g, off + q, pos_aligned);
-                raw[g] = (uint8_t)((val >> 7) & 0xFFu);
-            }
-            ++g;
-        }
-        done += total;
-    }
-    if (tid == 0) {
-        if (done != e_total) *status = SZ_ERR_CORRUPT;  // the input changed under us
-        else *out_bytes = container_size(n, e_total);
+        if (tid == 0) s_carry = carry + total;
+        __syncthreads();
     }
 }
 
-cudaError_t launch_tiny_encode(const uint16_t *in, uint64_t n, uint8_t *out, uint64_t out_cap, uint64_t *out_bytes,
-                               uint8_t *codebook_out, int32_t *status, cudaStream_t s) {
-    const size_t smem = kTinyColWords * sizeof(uint32_t);
-    tiny_encode_kernel<<<1, kThreads, smem, s>>>(in, n, out, out_cap, out_bytes, codebook_out, status);
+__global__ void __launch_bounds__(kThreads) small_encode_kernel(const uint16_t *in, uint64_t n, SmallWs w,
+                                                                uint8_t *out, uint64_t out_cap,
+                                                                uint64_t *out_bytes, int32_t *status) {
+    __shared__ uint32_t s_warp[kWarps];
+    __shared__ int s_last;
+    const uint32_t tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const uint32_t nb = (uint32_t)umax64(1, div_up(n, kSlice));  // an empty stream: one block
+    s_lut[tid] = 0x80;
+    __syncthreads();
+    if (tid < 16) s_lut[w.meta->codebook[tid]] = (uint8_t)tid;
+    const uint64_t e_total = w.meta->n_escapes;
+    if (container_size(n, e_total) > out_cap) {  // the same decision in every block
+        if (tid == 0 && blockIdx.x == 0) set_status(status, SZ_ERR_CAPACITY);
+        return;
+    }
+    if (blockIdx.x == 0 && tid < 6) {
+        uint64_t v = 0;
+        if (tid == 0) v = 0x00000101564B5A53ull;  // "SZKV", version 1, dtype 1, flags 0
+        if (tid == 1) v = n;
+        if (tid == 2) v = e_total;
+        if (tid == 3 || tid == 4)
+            for (int i = 7; i >= 0; --i) v = (v << 8) | w.meta->codebook[8 * (tid - 3) + i];
+        reinterpret_cast<uint64_t *>(out)[tid] = v;
+    }
+    __syncthreads();  // the LUT is complete
+    const uint64_t pos_off = kHeader + n + (n + 1) / 2;
+    const bool pos_aligned = (pos_off & 3) == 0;
+    uint8_t *codes = out + kHeader + n;
+    uint8_t *pos = out + pos_off;
+    uint8_t *raw = pos + 4 * e_total;
+    const uint64_t off = (uint64_t)blockIdx.x * kSlice + tid * kChunk;
+    uint32_t esc = 0;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    if (off < n) {
+        const uint32_t cnt = (uint32_t)umin64(kChunk, n - off);
+        if (cnt == (uint32_t)kChunk) {
+            v0 = ld_stream_v4(in + off);
+            v1 = ld_stream_v4(in + off + 8);
+        } else {
+            read_chunk_global(in + off, cnt, v0, v1);
+        }
+        uint4 smv;
+        uint64_t cw;
+        uint32_t m;
+        encode_chunk(v0, v1, smv, cw, m);
+        uint32_t keep = 0;
+#pragma unroll
+        for (int q = 0; q < kChunk; ++q)
+            if (q < (int)cnt) keep |= esc_bit_of_elem(q);
+        esc = esc_in_element_order(m & keep);
+        if (cnt < (uint32_t)kChunk) cw &= (1ull << (4 * cnt)) - 1ull;  // odd tail nibble = 0
+        if (cnt == (uint32_t)kChunk) {
+            st_stream_v4(out + kHeader + off, smv);
+        } else {
+#pragma unroll
+            for (int q = 0; q < kChunk; ++q)
+                if (q < (int)cnt) out[kHeader + off + q] = (uint8_t)byte_of(smv, q);
+        }
+        if (cnt == (uint32_t)kChunk && (n % 8) == 0) {
+            st_stream_u64(codes + off / 2, cw);
+        } else {
+#pragma unroll
+            for (int b = 0; b < kChunk / 2; ++b)
+                if (2 * b < (int)cnt) codes[off / 2 + b] = (uint8_t)(cw >> (8 * b));
+        }
+    }
+    const uint32_t k = __popc(esc);
+    uint32_t incl = k;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= (uint32_t)d) incl += y;
+    }
+    if (lane == 31) s_warp[wid] = incl;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) {
+        const uint32_t x = s_warp[q];
+        before += ((uint32_t)q < wid) ? x : 0u;
+        total += x;
+    }
+    const uint64_t b0 = w.block_off[blockIdx.x];
+    const uint64_t b1 = blockIdx.x + 1 < nb ? (uint64_t)w.block_off[blockIdx.x + 1] : e_total;
+    uint64_t g = b0 + before + incl - k;
+    while (esc) {
+        const int q = __ffs(esc) - 1;
+        esc &= esc - 1;
+        const uint32_t x = (q < 8) ? ((q < 4) ? (q < 2 ? v0.x : v0.y) : (q < 6 ? v0.z : v0.w))
+                                   : ((q < 12) ? (q < 10 ? v1.x : v1.y) : (q < 14 ? v1.z : v1.w));
+        if (g < b1) {  // never past the slice's share
+            store_u32_le(pos + 4 * g, (uint32_t)(off + q), pos_aligned);
+            raw[g] = (uint8_t)((x >> (16 * (q & 1) + 7)) & 0xFFu);
+        }
+        ++g;
+    }
+    if (tid == 0 && b0 + total != b1) set_status(status, SZ_ERR_CORRUPT);  // the input changed
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(w.done2, 1u) + 1 == nb;
+    __syncthreads();
+    if (s_last && tid == 0) {
+        __threadfence();
+        if (*reinterpret_cast<volatile int32_t *>(status) == SZ_OK) *out_bytes = container_size(n, e_total);
+    }
+}
+
+cudaError_t launch_small_encode(const uint16_t *in, uint64_t n, const SmallWs &w, uint8_t *out, uint64_t out_cap,
+                                uint64_t *out_bytes, uint8_t *codebook_out, int32_t *status, cudaStream_t s) {
+    const uint32_t nb = (uint32_t)umax64(1, div_up(n, kSlice));
+    small_hist_kernel<<<nb, kThreads, kTinyColWords * sizeof(uint32_t), s>>>(in, n, w, codebook_out, status,
+                                                                            out_bytes);
+    small_encode_kernel<<<nb, kThreads, 0, s>>>(in, n, w, out, out_cap, out_bytes, status);
     return cudaGetLastError();
 }
+
 
 // One CTA per range of the partition the histogram kernel used (one-pass:
 // of the partition the escape placement will use).

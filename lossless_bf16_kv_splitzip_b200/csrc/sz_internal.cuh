@@ -377,6 +377,16 @@ struct OvfItem {
     uint32_t seg;
 };
 
+// Scratch of the short-stream path of one-call compression (sz_compress).
+struct SmallWs {
+    uint32_t *seg_hist;    // [256] stream counts          } zero on entry
+    uint32_t *done;        // slices counted               }
+    uint32_t *done2;       // slices encoded               }
+    SegMeta *meta;
+    uint32_t *block_off;   // [slices] first escape index of each slice
+    uint32_t *block_hist;  // [slices][256]
+};
+
 // The escape placement that follows a one-pass encode.
 struct PlaceArgs {
     Batch batch;

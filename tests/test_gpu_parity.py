@@ -28,6 +28,7 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 H = 48
 DEV = "cuda:0"
+SHORT = 1 << 21  # streams up to this many elements take the short-stream encode / decode
 
 
 def to_dev(x_np):
@@ -78,6 +79,12 @@ RAGGED = [0, 1, 2, 3, 7, 8, 15, 16, 17, 31, 33, 100, 255, 4095, 4096, 4097, 8191
 @pytest.mark.parametrize("n", RAGGED)
 def test_ragged_sizes_bit_exact(n):
     assert_parity(kvgen.mixed_small(n, seed=5000 + n))
+
+
+# ragged streams longer than the short-stream limit: the pipelined paths
+@pytest.mark.parametrize("n", [SHORT + 1, SHORT + 16383, SHORT + 65537 + 7])
+def test_ragged_large_sizes_bit_exact(n):
+    assert_parity(kvgen.mixed_small(n, seed=n % 1000))
 
 
 @pytest.mark.parametrize("n", [1, 16, 17, 16384, 16385, 70001])
@@ -268,9 +275,9 @@ def corruptions(blob, n):
     return out
 
 
-# sizes up to one tile take the one-block decode, larger ones the
-# index + pipelined decode: both must reject every corruption
-@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11, 65536 + 3001, 3 * 65536 + 16 * 17])
+# short streams take the one-launch decode, longer ones the index +
+# pipelined decode: both must reject every corruption
+@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11, 65536 + 3001, SHORT + 3001, SHORT + 16 * 17])
 def test_corrupt_containers_rejected(n):
     x = kvgen.mixed_small(n, seed=21 + n)
     blob = gpu_encode(x)
@@ -287,7 +294,7 @@ def test_odd_tail_nibble_rejected():
     c = bytearray(gpu_encode(x))
     c[H + 3 + 1] |= 0x10
     assert gpu_decode(bytes(c), 3)[0] == sz.SZ_ERR_CORRUPT
-    n = 2 * 65536 + 1001  # the pipelined decode's path
+    n = SHORT + 1001  # the pipelined decode's path
     x = kvgen.mixed_small(n, seed=23)
     c = bytearray(gpu_encode(x))
     c[H + n + (n + 1) // 2 - 1] |= 0x10  # high nibble of the last code byte
@@ -295,11 +302,12 @@ def test_odd_tail_nibble_rejected():
 
 
 # -------------------------------------------------- one-call compression
-@pytest.mark.parametrize("n", [0, 1, 17, 4095, 16385, 32767, 32768, 32769, 65537, 3 * 65536 + 100, 262147])
+@pytest.mark.parametrize("n", [0, 1, 17, 4095, 4096, 4097, 32769, 65537, 3 * 65536 + 100, SHORT, SHORT + 1])
 def test_compress_one_call_equals_oracle(n):
-    """sz_compress: one block and one launch up to 32,768 elements, the
-    histogram and encode kernels beyond; the same bytes as the oracle (and
-    as the two-call path), and the codebook it reports is the header's."""
+    """sz_compress: short streams by 4,096-element blocks in two launches,
+    longer ones by the histogram and encode kernels; the same bytes as the
+    oracle (and as the two-call path), and the codebook it reports is the
+    header's."""
     x = kvgen.mixed_small(n, seed=300 + n % 101)
     cb = torch.zeros(16, dtype=torch.uint8, device=DEV)
     out, size, status = sz.compress(to_dev(x), codebook=cb)
@@ -310,7 +318,7 @@ def test_compress_one_call_equals_oracle(n):
     assert bytes(cb.cpu().numpy()) == got[24:40]
 
 
-@pytest.mark.parametrize("n", [30000, 70000])  # the one-block path and the kernels' path
+@pytest.mark.parametrize("n", [30000, SHORT + 70000])  # the short-stream path and the kernels' path
 def test_compress_capacity_checked_on_device(n):
     x = kvgen.uniform_u16(n, seed=301)  # incompressible: many escapes
     d = to_dev(x)
@@ -345,7 +353,7 @@ def test_stage_wait_times_out_cleanly():
 
 
 def test_decode_stage_wait_times_out_cleanly():
-    x = kvgen.mixed_small(4 * 16384 + 5, seed=32)
+    x = kvgen.mixed_small(SHORT + 5, seed=32)  # the pipelined decode (it has the waits)
     blob = oracle.encode(x)
     c = torch.from_numpy(np.frombuffer(blob, np.uint8).copy()).to(DEV)
     try:
