@@ -40,6 +40,9 @@ WORKLOAD_NAMES = {0: "tiny-k-1m", 1: "llama3-8b-kv-4k", 2: "llama3-8b-kv-32k",
                   3: "llama3-70b-kv-8k-heavy-tail", 4: "paged-kv-256-requests"}
 HEADER = 48
 FALLBACK_HBM_GBS = 6650.0
+# B200 HBM3e data-sheet bandwidth (8 TB/s; 7.7 TB/s on HGX boards).  Fractions
+# of it are reported beside the fractions of the measured copy bandwidth.
+SPEC_HBM_GBS = 8000.0
 
 
 def parse_args():
@@ -456,6 +459,8 @@ def run_sweep(args):
                 "encode_gbs": round(b / te / 1e9, 2), "decode_gbs": round(b / td / 1e9, 2),
                 "encode_roofline_frac": round((b + comp) / te / 1e9 / peak, 4),
                 "decode_roofline_frac": round((b + comp) / td / 1e9 / peak, 4),
+                "encode_roofline_frac_of_spec": round((b + comp) / te / 1e9 / SPEC_HBM_GBS, 4),
+                "decode_roofline_frac_of_spec": round((b + comp) / td / 1e9 / SPEC_HBM_GBS, 4),
                 "ratio": round(b / comp, 5), "round_trip": ok,
                 "peak_gbs": peak, "peak_kind": peak_kind, "reps": args.sweep_reps,
                 "timing": "CUDA graph replay between events, median; L2 flushed (512 MiB write) before each"}
@@ -635,7 +640,8 @@ def main():
     roof = {}
     for name, (b, t) in phases.items():
         a = b / t / 1e9
-        roof[name] = {"achieved": round(a, 1), "frac": round(a / peak, 4), "ms": round(t * 1e3, 4),
+        roof[name] = {"achieved": round(a, 1), "frac": round(a / peak, 4),
+                      "frac_of_spec": round(a / SPEC_HBM_GBS, 4), "ms": round(t * 1e3, 4),
                       "algorithmic_bytes": b}
     dom = max(phases, key=lambda k: phases[k][1])
     enc_e2e_bytes = U + comp
@@ -644,6 +650,7 @@ def main():
     traffic = profiled_traffic(dom, S, 2 * kvgen.CONTIGUOUS[WORKLOAD][0]) if inp.workload == WORKLOAD else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": roof[dom]["achieved"], "peak": peak, "unit": "GB/s",
                 "frac": roof[dom]["frac"], "traffic": traffic,
+                "spec_peak": SPEC_HBM_GBS, "frac_of_spec": roof[dom]["frac_of_spec"],
                 "peak_kind": peak_kind + " (copy, MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"}
 
     # ---- one pass with the codebooks kept from the timed steps (codebook
@@ -669,6 +676,7 @@ def main():
         t1 = float(np.mean([a0.elapsed_time(a1) for a0, a1 in ev1])) / 1e3
         one_pass = {"encode_gbs": round(U / t1 / 1e9, 2), "ms": round(t1 * 1e3, 4),
                     "roofline_frac": round((U + comp) / t1 / 1e9 / peak, 4),
+                    "roofline_frac_of_spec": round((U + comp) / t1 / 1e9 / SPEC_HBM_GBS, 4),
                     "same_containers_as_two_pass": same, "steps": k1,
                     "codebooks": "kept from the two-pass encode of the same tensors",
                     "launches": "one-pass encode, escape placement, overflow rescan"}
@@ -723,6 +731,8 @@ def main():
             "encode_gbs": round(U / encode_s / 1e9, 2), "decode_gbs": round(U / td / 1e9, 2),
             "encode_roofline_frac": round(enc_e2e_bytes / encode_s / 1e9 / peak, 4),
             "decode_roofline_frac": roof["decode"]["frac"],
+            "encode_roofline_frac_of_spec": round(enc_e2e_bytes / encode_s / 1e9 / SPEC_HBM_GBS, 4),
+            "decode_roofline_frac_of_spec": roof["decode"]["frac_of_spec"],
             "encode_one_pass": one_pass,
             "ratio": round(U / comp, 5), "escape_frac": round(esc / (U // 2), 6),
             "roofline": roofline, "roofline_phases": roof,
