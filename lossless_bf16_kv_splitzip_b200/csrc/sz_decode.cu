@@ -8,19 +8,24 @@
 // Two launches.  (1) esc_index_kernel: for every 16,384-element sub-tile,
 // the index of its first escape in the ascending position stream (one
 // binary search per sub-tile, all in parallel); it also checks each
-// segment's header.  (2) decode_kernel, warp-specialised like the encode:
-//   producer warp   TMA bulk copies of the sub-tile's sm bytes (16 KiB) and
-//                   codes (8 KiB) into a 2-stage ring (3 CTAs per SM); its 32 lanes also
-//                   load the sub-tile's escape records, check them (inside
-//                   the sub-tile, strictly ascending, raw exponent outside
-//                   the codebook) and store them in the stage together with
-//                   a chunk -> first-escape map;
+// segment's header.  (2) decode_kernel, warp-specialised like the encode,
+// 3 CTAs per SM, tiles dealt round robin (CTA b takes tiles b, b + grid,
+// ...), so that the CTAs' stores land close together in memory:
+//   producer thread  TMA bulk copies of the sub-tile's sm bytes (16 KiB),
+//                    codes (8 KiB) and a 16-byte aligned superset of its
+//                    escape positions and exponents into a 2-stage ring;
 //   8 consumer warps turn codes + sm bytes into BF16 with register-only
-//                   PRMT lookups, patch their chunk's escapes in registers
-//                   (checking the placeholder code is 0), and write 16-byte
-//                   stores.
+//                    PRMT lookups and write 16-byte stores (the escaped
+//                    places get codebook[0]); then, after one barrier, one
+//                    thread per escape checks its record (inside the
+//                    sub-tile, strictly ascending, raw exponent outside the
+//                    codebook, placeholder code 0) and overwrites the value.
 // Monotone sub-tile starts plus in-sub-tile checks prove the whole escape
 // stream well formed.  Every mbarrier wait is bounded.
+//
+// Streams of up to 2^21 elements take one launch instead: small_decode_kernel,
+// one block per 4,096-element slice, each finding its slice's escape records
+// by binary search.
 #include "sz_internal.cuh"
 
 namespace sz {
@@ -217,8 +222,6 @@ struct __align__(128) DecShared {
 template <bool kBatched>
 __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
-    const uint64_t t_begin = (uint64_t)blockIdx.x * a.tiles_per_cta;
-    const uint64_t t_end = umin64(t_begin + a.tiles_per_cta, a.batch.n_tiles);
     uint32_t j = 0;
     uint32_t cur = 0xFFFFFFFFu;
     sz_segment seg{};
@@ -226,7 +229,7 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     const uint8_t *c = nullptr;
     uint64_t cap = 0;
     bool tma_ok = false;
-    for (uint64_t t = t_begin; t < t_end; ++t) {
+    for (uint64_t t = blockIdx.x; t < a.batch.n_tiles; t += gridDim.x) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
             cur = k;
@@ -363,8 +366,8 @@ __device__ __forceinline__ void decode_store_chunk(const DecMeta &m, DecShared &
     decode_chunk(smv, codes, T, o0, o1);
     if (m.dst == nullptr) return;
     if (cnt == (uint32_t)kChunk) {
-        st_stream_v4(m.dst + off, o0);
-        st_stream_v4(m.dst + off + 8, o1);
+        *reinterpret_cast<uint4 *>(m.dst + off) = o0;
+        *reinterpret_cast<uint4 *>(m.dst + off + 8) = o1;
     } else {
         const uint32_t w[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
@@ -385,7 +388,7 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
         consumer_sync();
         if (!sh.go) {  // the same decision in every consumer thread
             if (tid == 0 && a.batch.n_tiles > 0) {
-                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.tiles_per_cta, a.batch.n_tiles - 1);
+                const uint64_t t0 = umin64((uint64_t)blockIdx.x, a.batch.n_tiles - 1);
                 set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
             }
             return;
@@ -584,9 +587,8 @@ cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStre
     DecodeArgs a = a0;
     if (a.batch.n_tiles == 0) return cudaSuccess;
     const size_t smem = sizeof(DecShared);
+    // tiles are dealt round robin: CTA b decodes tiles b, b + grid, ...
     grid = (int)umax64(1, umin64((uint64_t)grid, a.batch.n_tiles));
-    a.tiles_per_cta = div_up(a.batch.n_tiles, (uint64_t)grid);
-    grid = (int)div_up(a.batch.n_tiles, a.tiles_per_cta);
     cudaError_t e;
     if (batched) {
         e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
