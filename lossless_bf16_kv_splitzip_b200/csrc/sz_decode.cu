@@ -9,8 +9,8 @@
 // the index of its first escape in the ascending position stream (one
 // binary search per sub-tile, all in parallel); it also checks each
 // segment's header.  (2) decode_kernel, warp-specialised like the encode,
-// 3 CTAs per SM, tiles dealt round robin (CTA b takes tiles b, b + grid,
-// ...), so that the CTAs' stores land close together in memory:
+// 3 CTAs per SM, groups of tiles (about 65,536 elements each) dealt round
+// robin, so that the CTAs' stores land close together in memory:
 //   producer thread  TMA bulk copies of the sub-tile's sm bytes (16 KiB),
 //                    codes (8 KiB) and a 16-byte aligned superset of its
 //                    escape positions and exponents into a 2-stage ring;
@@ -215,6 +215,16 @@ struct __align__(128) DecShared {
     int go;
 };
 
+// Tiles are dealt round robin in groups of about kTile elements: one tile
+// of a contiguous tensor, several when pages are smaller than a tile, so
+// that a CTA meets a new segment (header, codebook tables) at most once per
+// group.  Group g holds tiles [g * group, (g + 1) * group).
+__host__ __device__ inline uint64_t tiles_per_group(const Batch &b) {
+    const uint64_t tile_elems = b.page_elems < (uint64_t)kTile ? b.page_elems : (uint64_t)kTile;
+    const uint64_t g = (uint64_t)kTile / (tile_elems > 0 ? tile_elems : 1);
+    return g > 0 ? g : 1;
+}
+
 // ------------------------------------------------------------ producer
 // One thread: per sub-tile, wait for the stage to be free, then bulk-copy
 // the sm bytes, the codes and (when they fit and stay inside the buffer) a
@@ -229,7 +239,9 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     const uint8_t *c = nullptr;
     uint64_t cap = 0;
     bool tma_ok = false;
-    for (uint64_t t = blockIdx.x; t < a.batch.n_tiles; t += gridDim.x) {
+    const uint64_t group = tiles_per_group(a.batch);
+    for (uint64_t t = (uint64_t)blockIdx.x * group; t < a.batch.n_tiles;
+         t = (t + 1) % group == 0 ? t + 1 + (uint64_t)(gridDim.x - 1) * group : t + 1) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
             cur = k;
@@ -388,7 +400,7 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
         consumer_sync();
         if (!sh.go) {  // the same decision in every consumer thread
             if (tid == 0 && a.batch.n_tiles > 0) {
-                const uint64_t t0 = umin64((uint64_t)blockIdx.x, a.batch.n_tiles - 1);
+                const uint64_t t0 = umin64((uint64_t)blockIdx.x * tiles_per_group(a.batch), a.batch.n_tiles - 1);
                 set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
             }
             return;
@@ -587,8 +599,8 @@ cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStre
     DecodeArgs a = a0;
     if (a.batch.n_tiles == 0) return cudaSuccess;
     const size_t smem = sizeof(DecShared);
-    // tiles are dealt round robin: CTA b decodes tiles b, b + grid, ...
-    grid = (int)umax64(1, umin64((uint64_t)grid, a.batch.n_tiles));
+    // groups of tiles are dealt round robin: CTA b decodes groups b, b + grid, ...
+    grid = (int)umax64(1, umin64((uint64_t)grid, div_up(a.batch.n_tiles, tiles_per_group(a.batch))));
     cudaError_t e;
     if (batched) {
         e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
