@@ -46,7 +46,10 @@ T3_SCALE_LOG2 = 7.0
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 to BF16 (nearest, ties to even); returns uint16 bits."""
+    """Round float32 to BF16 (nearest, ties to even); returns uint16 bits.
+
+    For finite values and infinities (a NaN whose payload sits in the low 16
+    bits would round to infinity); the generators here draw no NaN."""
     u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
     lsb = (u >> np.uint32(16)) & np.uint32(1)
     r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
