@@ -23,10 +23,12 @@ import numpy as np
 from ._build import LIB_PATH, build, is_stale
 
 __all__ = [
-    "SzError", "sz_plan", "sz_histogram_codebook", "sz_encode", "sz_decode", "sz_plan_batched",
-    "sz_histogram_codebook_batched", "sz_encode_batched", "sz_encode_static", "sz_decode_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags",
-    "sz_tile_elems", "sz_version", "encode", "decode", "BatchPlan", "lib", "HEADER_BYTES",
-    "max_bytes", "STATUS",
+    "SzError", "sz_segment", "sz_plan", "sz_histogram_codebook", "sz_encode", "sz_compress", "sz_decode",
+    "sz_plan_batched", "sz_histogram_codebook_batched", "sz_encode_batched", "sz_decode_batched",
+    "sz_encode_static", "sz_plan_one_pass", "sz_encode_one_pass", "sz_workspace_one_pass_batched",
+    "sz_encode_one_pass_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags", "sz_tile_elems",
+    "sz_version", "encode", "compress", "encode_one_pass", "decode", "BatchPlan", "lib",
+    "HEADER_BYTES", "max_bytes", "STATUS",
 ]
 
 HEADER_BYTES = 48

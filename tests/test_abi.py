@@ -24,6 +24,20 @@ def test_library_exports_every_declared_symbol():
     assert sz.sz_tile_elems() == 65536
 
 
+def test_binding_wraps_every_declared_symbol_by_its_name():
+    # the Python layer has one function per C entry point, same name, exported
+    names = sz.header_symbols(open(HEADER).read())
+    for n in names:
+        assert callable(getattr(sz, n, None)), n
+        assert n in sz.__all__, n
+    for n in sz.__all__:
+        assert hasattr(sz, n), n
+    # and argument types are declared for every entry point the header names
+    L = sz.lib()
+    for n in names:
+        assert getattr(L, n).argtypes is not None, n
+
+
 def test_library_is_built_for_sm100a():
     # the cubin is embedded for sm_100a; the host code reports its target
     assert "sm_100a" in sz.sz_version()
