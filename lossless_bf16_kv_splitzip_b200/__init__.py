@@ -245,6 +245,24 @@ def _torch():
     return torch
 
 
+def _nbytes(t) -> int:
+    """Bytes a contiguous tensor holds: the size the library is told."""
+    return t.numel() * t.element_size()
+
+
+def _workspace(workspace, wsb, dev):
+    """The caller's workspace (checked: contiguous, on the device, large
+    enough) or a new one of the planned size."""
+    torch = _torch()
+    if workspace is None:
+        return torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    if not workspace.is_contiguous() or workspace.device != dev:
+        raise ValueError("workspace must be a contiguous tensor on %s" % dev)
+    if _nbytes(workspace) < wsb:
+        raise ValueError("workspace holds %d bytes, the call needs %d" % (_nbytes(workspace), wsb))
+    return workspace
+
+
 def _u16_view(x):
     torch = _torch()
     if x.dtype in (torch.bfloat16, torch.float16, torch.int16):
@@ -263,13 +281,13 @@ def encode(x, stream=None, workspace=None):
     n = x.numel()
     cap, wsb = sz_plan(n)
     dev = x.device
-    ws = workspace if workspace is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
+    ws = _workspace(workspace, wsb, dev)
     cb = torch.empty(16, dtype=torch.uint8, device=dev)
     out = torch.empty(cap, dtype=torch.uint8, device=dev)
     size = torch.zeros(1, dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    sz_histogram_codebook(x, n, cb, None, ws, wsb, stream)
-    sz_encode(x, n, cb, out, cap, size, status, ws, wsb, stream)
+    sz_histogram_codebook(x, n, cb, None, ws, _nbytes(ws), stream)
+    sz_encode(x, n, cb, out, cap, size, status, ws, _nbytes(ws), stream)
     return out, size, status
 
 
@@ -282,11 +300,11 @@ def compress(x, stream=None, workspace=None, codebook=None):
     n = x.numel()
     cap, wsb = sz_plan(n)
     dev = x.device
-    ws = workspace if workspace is not None else torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    ws = _workspace(workspace, wsb, dev)
     out = torch.empty(cap, dtype=torch.uint8, device=dev)
     size = torch.zeros(1, dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    sz_compress(x, n, out, cap, size, codebook, status, ws, ws.numel(), stream)
+    sz_compress(x, n, out, cap, size, codebook, status, ws, _nbytes(ws), stream)
     return out, size, status
 
 
@@ -300,11 +318,11 @@ def encode_one_pass(x, codebook, stream=None, workspace=None):
     n = x.numel()
     cap, wsb = sz_plan_one_pass(n)
     dev = x.device
-    ws = workspace if workspace is not None else torch.empty(max(wsb, 256), dtype=torch.uint8, device=dev)
+    ws = _workspace(workspace, wsb, dev)
     out = torch.empty(cap, dtype=torch.uint8, device=dev)
     size = torch.zeros(1, dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    sz_encode_one_pass(x, n, codebook, out, cap, size, status, ws, ws.numel(), stream)
+    sz_encode_one_pass(x, n, codebook, out, cap, size, status, ws, _nbytes(ws), stream)
     return out, size, status
 
 
@@ -313,12 +331,16 @@ def decode(container, n, out=None, stream=None, workspace=None):
     tensor (bit patterns).  Returns (out, status int32 tensor [1])."""
     torch = _torch()
     dev = container.device
+    if not container.is_contiguous():
+        raise ValueError("the container must be a contiguous tensor")
     _, wsb = sz_plan(n)
-    ws = workspace if workspace is not None else torch.empty(wsb, dtype=torch.uint8, device=dev)
+    ws = _workspace(workspace, wsb, dev)
     if out is None:
         out = torch.empty(n, dtype=torch.int16, device=dev)
+    elif not out.is_contiguous() or out.device != dev or _nbytes(out) < 2 * n:
+        raise ValueError("out must be a contiguous tensor on %s with room for %d 16-bit values" % (dev, n))
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    sz_decode(container, container.numel(), out, n, status, ws, wsb, stream)
+    sz_decode(container, _nbytes(container), out, n, status, ws, _nbytes(ws), stream)
     return out, status
 
 
@@ -375,7 +397,9 @@ class BatchPlan:
         another plan's container buffer for the same segment lengths (its
         offsets are the same), e.g. to decode into another page size."""
         c = self.container if container is None else container
-        sz_decode_batched(self.n_segs, self.d_segs, self.n_tiles, c, c.numel(),
+        if not c.is_contiguous():
+            raise ValueError("the container must be a contiguous tensor")
+        sz_decode_batched(self.n_segs, self.d_segs, self.n_tiles, c, _nbytes(c),
                           d_page_ptrs, self.page_elems, self.dec_status, self.ws, self.ws.numel(), stream)
 
     def container_bytes(self, k: int, size: int) -> "np.ndarray":

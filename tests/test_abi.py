@@ -148,3 +148,32 @@ def test_batched_argument_errors():
     assert L.sz_histogram_codebook_batched(2, A, 4, A, 16384, None, A, A, 16, None) == sz.SZ_ERR_WORKSPACE
     assert L.sz_decode_batched(2, A, 4, A + 4, 1 << 20, A, 16384, A, A, 1 << 20, None) == sz.SZ_ERR_ALIGN
     assert L.sz_decode_batched(2, A, 4, A, 1 << 20, A, 16384, A, A, 16, None) == sz.SZ_ERR_WORKSPACE
+
+
+def test_helpers_check_caller_buffers_before_any_call():
+    # every check below raises on the host, before the library is called, so
+    # host tensors serve: an undersized workspace or output buffer would
+    # otherwise be written past its end by the device
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(70_000, dtype=torch.bfloat16)
+    _, wsb = sz.sz_plan(x.numel())
+    small_ws = torch.empty(wsb - 1, dtype=torch.uint8)
+    for helper in (sz.encode, sz.compress):
+        with pytest.raises(ValueError, match="workspace"):
+            helper(x, workspace=small_ws)
+    _, wsb1 = sz.sz_plan_one_pass(x.numel())
+    with pytest.raises(ValueError, match="workspace"):
+        sz.encode_one_pass(x, torch.arange(16, dtype=torch.uint8), workspace=torch.empty(wsb1 - 1, dtype=torch.uint8))
+    # the workspace size is counted in bytes, whatever its dtype
+    with pytest.raises(ValueError, match="workspace"):
+        sz.encode(x, workspace=torch.empty((wsb - 1) // 4, dtype=torch.int32))
+    blob = torch.zeros(1000, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="room for 300"):
+        sz.decode(blob, 300, out=torch.empty(299, dtype=torch.int16))
+    with pytest.raises(ValueError, match="room for 300"):
+        sz.decode(blob, 300, out=torch.empty(600, dtype=torch.int16)[::2])
+    with pytest.raises(ValueError, match="contiguous"):
+        sz.decode(torch.zeros(2000, dtype=torch.uint8)[::2], 300)
+    assert sz.sz_plan(300)[1] > 0
+    with pytest.raises(ValueError, match="workspace"):
+        sz.decode(blob, 300, workspace=torch.empty(0, dtype=torch.uint8))
