@@ -1,7 +1,7 @@
 /*
  * sz_oracle.h -- plain single-threaded CPU reference of the SplitZip BF16
  * exponent codec.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and
- * the bench's CPU-baseline leg use it to judge the CUDA library; the CUDA
+ * the bench's CPU-baseline leg use it to check the CUDA library; the CUDA
  * library never includes, links or calls it, and it shares no code with it.
  *
  * Source of the method: "SplitZip: Ultra Fast Lossless KV Compression for

@@ -1,6 +1,6 @@
 """Pins of the CPU oracle against facts that do not come from the oracle.
 
-The oracle (oracle/sz_oracle.c) is the judge of the CUDA library, so it is
+The oracle (oracle/sz_oracle.c) is what the CUDA library is checked against, so it is
 itself checked here against what the SplitZip explainer and arithmetic fix:
 
 * field split vs IEEE-754 arithmetic (frexp) on all 65,536 BF16 patterns
