@@ -60,6 +60,13 @@
  *   - Vector path: device buffers must be 16-byte aligned (SZ_ERR_ALIGN
  *     otherwise); there is no scalar fallback for misaligned buffers.
  *   - Element counts are limited to n < 2^32 (escape positions are u32).
+ *   - A device error leaves the affected container's size word(s) at 0: a
+ *     size is written only after every CTA that worked on that container
+ *     finished its share without an error.  A status of SZ_OK with a
+ *     nonzero size is a complete container.
+ *   - The calling thread's current device must have an ordinal below 64
+ *     (per-device facts are kept in a 64-entry table); a larger ordinal
+ *     returns SZ_ERR_INVALID before anything is enqueued.
  */
 #ifndef SPLITZIP_H
 #define SPLITZIP_H
@@ -129,7 +136,9 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
  *                   the exact size against out_cap (SZ_ERR_CAPACITY).
  *                   sz_plan's max_compressed_bytes always suffices for a
  *                   codebook from sz_histogram_codebook.
- *   d_out_bytes     out: uint64 container size (0 on a device error)
+ *   d_out_bytes     out: uint64 container size (0 on a device error: the
+ *                   size is written by the CTA that completes the stream's
+ *                   tile count, and only when no CTA reported an error)
  *   d_status        out (required): int32 device status (SZ_OK,
  *                   SZ_ERR_CORRUPT when the workspace histogram does not
  *                   describe d_in, SZ_ERR_CAPACITY, SZ_ERR_INVALID,
@@ -141,7 +150,9 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
  * counts of the first and last segment piece of every CTA's range of tiles,
  * and from those each CTA's first escape index follows (placed by the
  * histogram call for its own codebook, again here for another one).  A
- * pipeline wait that runs out gives SZ_ERR_DEVICE_TIMEOUT.
+ * pipeline wait that runs out gives SZ_ERR_DEVICE_TIMEOUT.  The same
+ * workspace may serve several sz_encode calls after one histogram call
+ * (with other codebooks, or after an error).
  */
 sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook16, uint8_t *d_out,
                     uint64_t out_cap, uint64_t *d_out_bytes, int32_t *d_status, void *d_ws,
@@ -282,16 +293,18 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
  * two-call path (sz_histogram_codebook + sz_encode) writes with the same
  * codebook.
  *
- * Two kernels: the encode writes the sign+mantissa and code streams in place
- * and parks each 65,536-element tile's escape records (up to 4,096 per tile,
- * 6.25 %) in the workspace; a placement kernel then counts each segment's
- * escapes, writes the header and the size, and moves the records into place
- * (a tile with more than 4,096 escapes has its input read again, by a third
- * kernel that spreads such tiles over the GPU).
+ * Three kernels: the encode writes the sign+mantissa and code streams in
+ * place and parks each 65,536-element tile's escape records (up to 4,096 per
+ * tile, 6.25 %) in the workspace; a placement kernel then counts each
+ * segment's escapes, writes the header and moves the records into place; a
+ * third kernel reads again the input of every tile with more than 4,096
+ * escapes (spread over the GPU), and its last block writes every segment's
+ * size (0 for a segment with an error).
  *
  * sz_plan_one_pass -- worst-case container (every element an escape:
  * 48 + n + ceil(n/2) + 5n) and workspace bytes (16,420 bytes per tile,
- * about 1/8 of the input's bytes, plus 16 bytes per range).  Host only.
+ * about 1/8 of the input's bytes, plus 16 bytes per range and 4 per
+ * segment).  Host only.
  */
 sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes);
 
@@ -349,7 +362,8 @@ sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, 
  *   d_out, out_cap, d_out_bytes, d_status  as for sz_encode
  *   d_codebook16_or_null  optional out: the 16-entry codebook
  * The container is byte for byte the one sz_histogram_codebook + sz_encode
- * write.  The first call on a device looks up the array's device address
+ * write (the same kernels run; their waits follow sz_set_wait_limit_ns).
+ * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
  * All calls on a device share the one array: calls that overlap on the GPU
  * (other streams, other host threads) race and must be serialised by the
@@ -364,8 +378,8 @@ sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uin
 /* ------------------------------------------------------------ diagnostics */
 /*
  * sz_set_wait_limit_ns -- upper bound, in nanoseconds of device time, of
- * every device-side wait (a pipeline stage of the encode or decode kernel
- * waiting for its bulk copy).
+ * every device-side wait of every entry point (a pipeline stage of the
+ * encode or decode kernel waiting for its bulk copy).
  * Default 1e9 (one second).  A wait that runs out sets
  * SZ_ERR_DEVICE_TIMEOUT in the segment's status and the kernel returns.
  * Applies to calls made after it, process-wide.

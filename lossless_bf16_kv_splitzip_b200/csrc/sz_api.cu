@@ -33,26 +33,8 @@ constexpr uint64_t kSmallDecodeMax = 1ull << 21;  // sz_decode: one launch of 4,
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<uint32_t> g_debug_flags{0};
 
-struct DeviceInfo {
-    bool ready = false;
-    int sms = 0, dec_occ = 1;
-};
 std::mutex g_dev_mu;
-DeviceInfo g_dev[64];
-
-bool device_info(DeviceInfo &out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-    std::lock_guard<std::mutex> lock(g_dev_mu);
-    DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
-        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-        d.dec_occ = decode_blocks_per_sm();
-        d.ready = true;
-    }
-    out = d;
-    return true;
-}
+DeviceInfo g_dev[kMaxDevices];
 
 uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -61,19 +43,21 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 // ranges (256-byte aligned parts)
 //   seg_hist   u32[S][256]     exponent counts per segment      } zeroed together
 //   seg_done   u32[S]          tiles counted so far per segment } by the histogram call
+//   enc_done   u32[S]          tiles of complete encode pieces  } (and by the encode call)
 //   meta       SegMeta[S]      codebook and escape count per segment
 //   rhist      u32[G][2][256]  counts of each range's first and last piece
 //   rrec       RangeRec[G]     escape placement of each range's pieces
 //   sub_start  u32[4T + S]     first escape index of each sub-tile (decode; 4 = sub-tiles per tile)
 struct Ws {
-    uint64_t seg_hist, seg_done, meta, rhist, rrec, sub_start, total;
+    uint64_t seg_hist, seg_done, enc_done, meta, rhist, rrec, sub_start, total;
 };
 Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
     const uint64_t g = umin64(n_tiles, kMaxRanges);
     Ws w;
     w.seg_hist = 0;
     w.seg_done = 1024 * n_segs;
-    w.meta = round_up(w.seg_done + 4 * n_segs, kAlign);
+    w.enc_done = 1028 * n_segs;
+    w.meta = round_up(w.enc_done + 4 * n_segs, kAlign);
     w.rhist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
     w.rrec = round_up(w.rhist + 2048 * g, kAlign);
     w.sub_start = round_up(w.rrec + sizeof(RangeRec) * g, kAlign);
@@ -81,25 +65,52 @@ Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
     return w;
 }
 
-// ---- one-pass workspace for T tiles and G = min(T, kMaxRanges) ranges
-//   ovf_count u32                 tiles listed for the rescan (zeroed per call)
+// ---- one-pass workspace for S segments, T tiles and G = min(T, kMaxRanges)
+// ranges
+//   ovf_count   u32               tiles listed for the rescan      } zeroed
+//   blocks_done u32               rescan blocks finished           } per call
 //   rcnt      RangeRec[G]         escapes of each range's first and last piece
+//   seg_e     u32[S]              escape count of each segment
 //   tile_cnt  u32[T]              escapes of each tile
 //   ovf       OvfItem[T]          tiles whose records overflowed their slot
 //   slots     u32[T][kSlotCap]    each tile's first kSlotCap escape records
 struct Ws1 {
-    uint64_t ovf_count, rcnt, tile_cnt, ovf, slots, total;
+    uint64_t ovf_count, blocks_done, rcnt, seg_e, tile_cnt, ovf, slots, total;
 };
-Ws1 ws1_layout(uint64_t n_tiles) {
+Ws1 ws1_layout(uint64_t n_segs, uint64_t n_tiles) {
     const uint64_t g = umin64(n_tiles, kMaxRanges);
     Ws1 w;
     w.ovf_count = 0;
+    w.blocks_done = 4;
     w.rcnt = kAlign;
-    w.tile_cnt = round_up(w.rcnt + sizeof(RangeRec) * g, kAlign);
+    w.seg_e = round_up(w.rcnt + sizeof(RangeRec) * g, kAlign);
+    w.tile_cnt = round_up(w.seg_e + 4 * n_segs, kAlign);
     w.ovf = round_up(w.tile_cnt + 4 * n_tiles, kAlign);
     w.slots = round_up(w.ovf + sizeof(OvfItem) * n_tiles, kAlign);
     w.total = round_up(w.slots + 4ull * kSlotCap * n_tiles, kAlign);
     return w;
+}
+
+}  // namespace
+
+namespace sz {
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+uint32_t debug_flags() { return g_debug_flags.load(); }
+
+sz_status device_info(DeviceInfo &out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SZ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SZ_ERR_INVALID;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SZ_ERR_CUDA;
+        d.dec_occ = decode_blocks_per_sm();
+        d.ready = true;
+    }
+    out = d;
+    return SZ_OK;
 }
 
 Batch single_batch(uint64_t n) {
@@ -115,6 +126,10 @@ Batch single_batch(uint64_t n) {
     b.single.tile_begin = 0;
     return b;
 }
+
+}  // namespace sz
+
+namespace {
 
 Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, uint64_t page_elems) {
     Batch b{};
@@ -189,11 +204,11 @@ sz_status one_pass(const Batch &b, const uint16_t *const *d_pages, const uint16_
                           const uint8_t *d_codebooks, uint8_t *d_out, uint64_t out_cap, uint64_t *d_out_bytes,
                           int32_t *d_status, void *d_ws, const Ws1 &w, cudaStream_t s) {
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     const uint64_t ns = b.segs ? b.n_segs : 1;
     SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, 8 * ns, s));
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * ns, s));
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.ovf_count), 0, 4, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.ovf_count), 0, 8, s));  // ovf_count, blocks_done
     EncodeArgs a{};
     a.batch = b;
     a.pages = d_pages;
@@ -203,8 +218,8 @@ sz_status one_pass(const Batch &b, const uint16_t *const *d_pages, const uint16_
     a.out_bytes = d_out_bytes;
     a.status = d_status;
     a.range_tiles = plan_ranges(b.n_tiles, (uint64_t)dev.sms).tiles;
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
     a.codebooks_in = d_codebooks;
     a.tile_cnt = at<uint32_t>(d_ws, w.tile_cnt);
     a.slots = at<uint32_t>(d_ws, w.slots);
@@ -225,10 +240,53 @@ sz_status one_pass(const Batch &b, const uint16_t *const *d_pages, const uint16_
     p.range_tiles = a.range_tiles;
     p.ovf_count = at<uint32_t>(d_ws, w.ovf_count);
     p.ovf = at<OvfItem>(d_ws, w.ovf);
+    p.seg_e = at<uint32_t>(d_ws, w.seg_e);
+    p.blocks_done = at<uint32_t>(d_ws, w.blocks_done);
     return cuda_status(launch_place(p, b.segs != nullptr, dev.sms, s));
 }
 
 }  // namespace
+
+namespace sz {
+
+sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap,
+                             uint64_t *d_out_bytes, uint8_t *d_codebook16_or_null, int32_t *d_status,
+                             const CompressScratch &w, const DeviceInfo &dev, cudaStream_t s) {
+    SZ_TRY_CUDA(cudaMemsetAsync(w.zero, 0, w.zero_bytes, s));  // seg_hist, seg_done, enc_done
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
+    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
+    SelectCtx c{};
+    c.batch = single_batch(n);
+    c.seg_hist = w.seg_hist;
+    c.rhist = w.rhist;
+    c.meta = w.meta;
+    c.rrec = w.rrec;
+    c.range_tiles = plan_ranges(c.batch.n_tiles, (uint64_t)dev.sms).tiles;
+    c.codebooks_out = d_codebook16_or_null;
+    HistArgs h{};
+    h.sel = c;
+    h.base = d_in;
+    h.seg_hist = w.seg_hist;
+    h.seg_done = w.seg_done;
+    h.rhist = w.rhist;
+    SZ_TRY_CUDA(launch_hist(h, false, s));
+    EncodeArgs a{};  // the codebook the histogram kernel chose: no reselect
+    a.batch = c.batch;
+    a.base = d_in;
+    a.out = d_out;
+    a.out_cap = out_cap;
+    a.out_bytes = d_out_bytes;
+    a.status = d_status;
+    a.meta = c.meta;
+    a.rrec = c.rrec;
+    a.range_tiles = c.range_tiles;
+    a.enc_done = w.enc_done;
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
+    return cuda_status(launch_encode(a, false, s));
+}
+
+}  // namespace sz
 
 extern "C" {
 
@@ -248,9 +306,9 @@ sz_status sz_histogram_codebook(const uint16_t *d_in, uint64_t n, uint8_t *d_cod
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 + 4, s));  // seg_hist, seg_done
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, w.meta - w.seg_hist, s));  // seg_hist, seg_done, enc_done
     SelectCtx c = select_ctx(single_batch(n), d_ws, w, dev);
     c.codebooks_out = d_codebook16;
     c.hist_out = d_hist256_or_null;
@@ -269,7 +327,7 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // escape count and range records for this codebook, from the piece
     // counts sz_histogram_codebook left in the workspace (nothing to do when
@@ -279,6 +337,7 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
     ra.codebook_in = d_codebook16;
     ra.status = d_status;
     ra.out_bytes = d_out_bytes;
+    ra.enc_done = at<uint32_t>(d_ws, w.enc_done);
     SZ_TRY_CUDA(launch_reselect(ra, s));
     EncodeArgs a{};
     a.batch = ra.sel.batch;
@@ -290,8 +349,9 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
     a.meta = ra.sel.meta;
     a.rrec = ra.sel.rrec;
     a.range_tiles = ra.sel.range_tiles;
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
+    a.enc_done = ra.enc_done;
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
     return cuda_status(launch_encode(a, false, s));
 }
 
@@ -306,7 +366,7 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
     if (n <= kSmallDecodeMax) return cuda_status(launch_small_decode(d_in, in_bytes, d_out, n, d_status, s));
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     DecodeArgs a{};
     a.batch = single_batch(n);
     a.base = d_out;
@@ -314,8 +374,8 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     a.in_cap = in_bytes;
     a.status = d_status;
     a.sub_start = at<uint32_t>(d_ws, w.sub_start);
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
     SZ_TRY_CUDA(launch_esc_index(a, false, s));
     return cuda_status(launch_decode(a, false, dev.sms * dev.dec_occ, s));
 }
@@ -343,28 +403,17 @@ sz_status sz_compress(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t
             launch_small_encode(d_in, n, sw, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, s));
     }
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1024 + 4, s));  // seg_hist, seg_done
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
-    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
-    SelectCtx c = select_ctx(single_batch(n), d_ws, w, dev);
-    c.codebooks_out = d_codebook16_or_null;
-    HistArgs h = hist_args(c, d_ws, w);
-    h.base = d_in;
-    SZ_TRY_CUDA(launch_hist(h, false, s));
-    EncodeArgs a{};  // the codebook the histogram kernel chose: no reselect
-    a.batch = c.batch;
-    a.base = d_in;
-    a.out = d_out;
-    a.out_cap = out_cap;
-    a.out_bytes = d_out_bytes;
-    a.status = d_status;
-    a.meta = c.meta;
-    a.rrec = c.rrec;
-    a.range_tiles = c.range_tiles;
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
-    return cuda_status(launch_encode(a, false, s));
+    if (const sz_status st = device_info(dev)) return st;
+    CompressScratch cs;
+    cs.zero = at<uint8_t>(d_ws, w.seg_hist);
+    cs.zero_bytes = w.meta - w.seg_hist;
+    cs.seg_hist = at<uint32_t>(d_ws, w.seg_hist);
+    cs.seg_done = at<uint32_t>(d_ws, w.seg_done);
+    cs.enc_done = at<uint32_t>(d_ws, w.enc_done);
+    cs.meta = at<SegMeta>(d_ws, w.meta);
+    cs.rhist = at<uint32_t>(d_ws, w.rhist);
+    cs.rrec = at<RangeRec>(d_ws, w.rrec);
+    return compress_pipelined(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, cs, dev, s);
 }
 
 sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t page_elems, sz_segment *h_segs,
@@ -407,9 +456,9 @@ sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_seg
     const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, 1028 * (uint64_t)n_segs, s));  // seg_hist, seg_done
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.seg_hist), 0, w.meta - w.seg_hist, s));  // seg_hist, seg_done, enc_done
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
     SelectCtx c = select_ctx(make_batch(n_segs, d_segs, n_tiles, page_elems), d_ws, w, dev);
     c.codebooks_out = d_codebooks_or_null;
@@ -430,9 +479,10 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, 8 * (uint64_t)n_segs, s));
+    SZ_TRY_CUDA(cudaMemsetAsync(at<uint8_t>(d_ws, w.enc_done), 0, 4 * (uint64_t)n_segs, s));
     const SelectCtx c = select_ctx(make_batch(n_segs, d_segs, n_tiles, page_elems), d_ws, w, dev);
     EncodeArgs a{};
     a.batch = c.batch;
@@ -444,8 +494,9 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.meta = c.meta;
     a.rrec = c.rrec;
     a.range_tiles = c.range_tiles;
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
+    a.enc_done = at<uint32_t>(d_ws, w.enc_done);
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
     return cuda_status(launch_encode(a, true, s));
 }
 
@@ -459,7 +510,7 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     const Ws w = ws_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
-    if (!device_info(dev)) return SZ_ERR_CUDA;
+    if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
     DecodeArgs a{};
@@ -469,8 +520,8 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.in_cap = in_cap;
     a.status = d_status;
     a.sub_start = at<uint32_t>(d_ws, w.sub_start);
-    a.wait_limit_ns = g_wait_limit_ns.load();
-    a.debug_flags = g_debug_flags.load();
+    a.wait_limit_ns = wait_limit_ns();
+    a.debug_flags = debug_flags();
     SZ_TRY_CUDA(launch_esc_index(a, true, s));
     return cuda_status(launch_decode(a, true, dev.sms * dev.dec_occ, s));
 }
@@ -479,7 +530,7 @@ sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uin
     if (!max_compressed_bytes || !workspace_bytes) return SZ_ERR_NULL;
     if (n_elems > kMaxElems) return SZ_ERR_TOO_LARGE;
     *max_compressed_bytes = container_size(n_elems, n_elems);
-    *workspace_bytes = ws1_layout(single_batch(n_elems).n_tiles).total;
+    *workspace_bytes = ws1_layout(1, single_batch(n_elems).n_tiles).total;
     return SZ_OK;
 }
 
@@ -491,17 +542,16 @@ sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
     const Batch b = single_batch(n);
-    const Ws1 w = ws1_layout(b.n_tiles);
+    const Ws1 w = ws1_layout(1, b.n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     return one_pass(b, nullptr, d_in, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, w,
                     static_cast<cudaStream_t>(stream));
 }
 
 sz_status sz_workspace_one_pass_batched(uint32_t n_segs, uint64_t n_tiles, uint64_t *workspace_bytes) {
-    (void)n_segs;
     if (!workspace_bytes) return SZ_ERR_NULL;
     if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
-    *workspace_bytes = ws1_layout(n_tiles).total;
+    *workspace_bytes = ws1_layout(n_segs, n_tiles).total;
     return SZ_OK;
 }
 
@@ -516,7 +566,7 @@ sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, 
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
     if (!aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const Ws1 w = ws1_layout(n_tiles);
+    const Ws1 w = ws1_layout(n_segs, n_tiles);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     return one_pass(make_batch(n_segs, d_segs, n_tiles, page_elems), d_pages, nullptr, d_codebooks, d_out, out_cap,
                     d_out_bytes, d_status, d_ws, w, static_cast<cudaStream_t>(stream));

@@ -30,7 +30,6 @@ constexpr uint32_t kFlagEnd = 1u;        // no more sub-tiles
 constexpr uint32_t kFlagInSmem = 2u;     // data came by TMA into the stage
 constexpr uint32_t kFlagLastSub = 4u;    // last sub-tile of its piece (the range's tiles of one segment)
 constexpr uint32_t kFlagHeader = 8u;     // first sub-tile of the segment: write the header
-constexpr uint32_t kFlagLastTile = 16u;  // last tile of the segment: write the size
 // one-pass mode (kFlagLastSub then marks the last sub-tile of a tile)
 constexpr uint32_t kFlagPieceEnd = 32u;     // last sub-tile of the piece
 constexpr uint32_t kFlagPieceOpens = 64u;   // the piece opens the range
@@ -39,12 +38,15 @@ constexpr uint32_t kFlagPieceCloses = 128u; // the piece closes the range
 struct EncMeta {
     const uint16_t *src;  // global address of the sub-tile's first element
     uint64_t elem0;       // first element of the sub-tile in the segment stream
+    uint64_t piece_end;   // global tile after the piece's last tile
     uint32_t seg;
     uint32_t len;         // elements of the sub-tile
     uint32_t flags;
     uint32_t esc_base;    // first escape index of the piece (one-pass: the global tile)
     uint32_t esc_count;   // escapes the piece must produce (one-pass: unused)
     uint32_t sub_in_tile; // sub-tile index within its tile
+    uint32_t piece_tiles; // tiles of the piece
+    uint32_t seg_tiles;   // tiles of the segment
 };
 
 struct __align__(128) EncShared {
@@ -155,6 +157,7 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
     uint64_t e_total = 0;
     uint32_t p_base = 0, p_count = 0;  // the piece's first escape index and escape count
     uint64_t p_first = 0, p_last = 0;  // the piece's first and last tile
+    uint64_t seg_end = 0;              // tile after the segment's last tile
     for (uint64_t t = t_begin; t < t_end; ++t) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {  // a new piece: the range's tiles of segment k
@@ -175,7 +178,7 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             if (!valid) set_status(a.status + k, SZ_ERR_INVALID);
             else if (!fits) set_status(a.status + k, SZ_ERR_CAPACITY);
             else if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
-            const uint64_t seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
+            seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
             p_first = t;
             p_last = umin64(seg_end, t_end) - 1;
             if (t == t_begin) {  // opens the range
@@ -206,6 +209,9 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             m.seg = k;
             m.len = aligned ? umin32(kSub, r.len - sub * kSub) : 0u;  // nothing is read from a misaligned page
             m.sub_in_tile = sub;
+            m.piece_end = p_last + 1;
+            m.piece_tiles = (uint32_t)(p_last + 1 - p_first);
+            m.seg_tiles = (uint32_t)(seg_end - seg.tile_begin);
             uint32_t f = 0;
             if (kOnePass) {
                 m.esc_base = (uint32_t)t;
@@ -221,7 +227,6 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
                 m.esc_count = p_count;
                 if (t == p_last && sub + 1 == r.n_subs) f |= kFlagLastSub;
                 if (r.local == 0 && sub == 0) f |= kFlagHeader;
-                if (r.local + 1 == r.tiles) f |= kFlagLastTile;
             }
             const bool tma = m.len == kSub;
             if (tma) f |= kFlagInSmem;
@@ -320,6 +325,19 @@ __device__ __forceinline__ bool warp_escape_scan(const uint32_t (&esc)[kChunks],
     return true;  // some chunk of the warp has several escapes
 }
 
+// A stage wait ran out.  The pieces of this CTA's range before tile `from`
+// are complete: their records are written and they were counted.  Every
+// segment with a piece at or after `from` gets SZ_ERR_DEVICE_TIMEOUT, and
+// none of them is counted here, so their sizes are never written.
+__device__ void timeout_from(const EncodeArgs &a, const SegCache &c, uint64_t from, uint64_t t_end) {
+    for (uint64_t t = from; t < t_end;) {
+        const uint32_t k = find_segment(c, a.batch, t);  // the segment that holds tile t
+        set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
+        const sz_segment sk = load_segment(a.batch, k);
+        t = sk.tile_begin + segment_tiles(sk.n_elems, a.batch.page_elems);
+    }
+}
+
 template <bool kBatched, bool kOnePass>
 __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -330,6 +348,9 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     uint32_t running = 0;  // escapes of the current piece so far (one-pass: of the tile)
     uint32_t piece_acc = 0;  // one-pass: escapes of the current piece so far
     PendingEsc pend{};
+    const uint64_t t_begin = umin64((uint64_t)blockIdx.x * a.range_tiles, a.batch.n_tiles);
+    const uint64_t t_end = umin64(t_begin + a.range_tiles, a.batch.n_tiles);
+    uint64_t counted_end = t_begin;  // thread 0: the pieces before this tile are complete
 
     // The wait for stage j+1 is folded into sub-tile j's scan barrier: one
     // consumer barrier per sub-tile.
@@ -338,10 +359,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kEncStages);
         if (!sh.go[j & 1]) {  // the same decision in every consumer thread
-            if (tid == 0 && a.batch.n_tiles > 0) {
-                const uint64_t t0 = umin64((uint64_t)blockIdx.x * a.range_tiles, a.batch.n_tiles - 1);
-                set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
-            }
+            if (tid == 0) timeout_from(a, sh.segc, counted_end, t_end);
             return;
         }
         const EncMeta m = sh.meta[s];
@@ -534,12 +552,32 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             }
             if (m.flags & kFlagPieceEnd) piece_acc = 0;
             running = 0;
-        } else if (!kOnePass && (m.flags & kFlagLastSub)) {
+        }
+        if (m.flags & (kOnePass ? kFlagPieceEnd : kFlagLastSub)) {
+            // End of a piece.  Its last records go out now instead of one
+            // sub-tile later, so that once the barrier below is passed every
+            // record of the piece is written.  Two-pass: the piece's escape
+            // count is checked, then its tiles are added to the segment's
+            // completion count; the piece that completes it writes the size,
+            // if no piece of the segment reported an error -- a segment with
+            // an error keeps size 0.
+            consumer_sync();
+            copy_out_escapes<kOnePass>(sh.esc[j & 1], pend, tid);
+            pend.cnt = 0;
+            consumer_sync();
             if (tid == 0) {
-                if (running != m.esc_count) set_status(status, SZ_ERR_CORRUPT);
-                else if (m.flags & kFlagLastTile) a.out_bytes[m.seg] = container_size(n, e_total);
+                if (!kOnePass) {
+                    if (running != m.esc_count) set_status(status, SZ_ERR_CORRUPT);
+                    __threadfence();
+                    if (atomicAdd(a.enc_done + m.seg, m.piece_tiles) + m.piece_tiles == m.seg_tiles) {
+                        __threadfence();  // every piece's status is visible
+                        if (*reinterpret_cast<volatile const int32_t *>(status) == SZ_OK)
+                            a.out_bytes[m.seg] = container_size(n, e_total);
+                    }
+                }
+                counted_end = m.piece_end;
             }
-            running = 0;
+            if (!kOnePass) running = 0;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);

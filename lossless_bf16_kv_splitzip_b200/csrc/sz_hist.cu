@@ -303,13 +303,14 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
 
 // Caller codebook for a single tensor: the select again with that codebook,
 // unless it is the one the workspace already holds.  Also resets the
-// encode's status and size words.
+// encode's status, size and completion words.
 __global__ void __launch_bounds__(kThreads) reselect_kernel(const ReselectArgs a) {
     __shared__ SelShared s_sel;
     __shared__ int s_same;
     if (threadIdx.x == 0) {
         *a.status = SZ_OK;
         *a.out_bytes = 0;
+        *a.enc_done = 0;
         s_same = a.sel.meta[0].valid != 0;
     }
     __syncthreads();

@@ -346,6 +346,7 @@ struct ReselectArgs {
     const uint8_t *codebook_in;
     int32_t *status;      // set to SZ_OK here
     uint64_t *out_bytes;  // set to 0 here
+    uint32_t *enc_done;   // set to 0 here
 };
 
 struct EncodeArgs {
@@ -361,6 +362,7 @@ struct EncodeArgs {
     uint64_t range_tiles;     // tiles per range = per CTA
     uint64_t wait_limit_ns;
     uint32_t debug_flags;
+    uint32_t *enc_done;       // [n_segs] tiles whose pieces are complete, zero on entry (two-pass)
     // one-pass mode (caller codebooks, no histogram pass)
     const uint8_t *codebooks_in;  // [n_segs][16]
     uint32_t *tile_cnt;           // [n_tiles] escapes of each tile
@@ -403,6 +405,8 @@ struct PlaceArgs {
     uint64_t range_tiles;
     uint32_t *ovf_count;          // overflowed tiles listed so far (zero on entry)
     OvfItem *ovf;                 // [n_tiles]
+    uint32_t *seg_e;              // [n_segs] escape count of each segment (placement -> rescan)
+    uint32_t *blocks_done;        // rescan blocks finished (zero on entry)
 };
 
 struct DecodeArgs {
@@ -417,5 +421,40 @@ struct DecodeArgs {
     uint64_t wait_limit_ns;
     uint32_t debug_flags;
 };
+
+// ------------------------------------------------------------- host side
+// Process-wide settings of sz_set_wait_limit_ns and sz_debug_set_flags.
+uint64_t wait_limit_ns();
+uint32_t debug_flags();
+
+// The implicit batch of a single-tensor call: one segment, one page.
+Batch single_batch(uint64_t n);
+
+// Device facts the launchers need, looked up once per device ordinal
+// (ordinals 0..kMaxDevices-1; a larger ordinal gives SZ_ERR_INVALID).
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0, dec_occ = 1;
+};
+sz_status device_info(DeviceInfo &out);
+
+// Scratch of the pipelined compression of one stream.  `zero` .. `zero` +
+// zero_bytes must cover seg_hist, seg_done and enc_done (cleared by the call).
+struct CompressScratch {
+    uint8_t *zero;
+    uint64_t zero_bytes;
+    uint32_t *seg_hist;  // [256]
+    uint32_t *seg_done;  // [1]
+    uint32_t *enc_done;  // [1]
+    SegMeta *meta;       // [1]
+    uint32_t *rhist;     // [ranges][2][256]
+    RangeRec *rrec;      // [ranges]
+};
+// Histogram kernel (with the select) and encode kernel of d_in[0..n): the
+// container of sz_histogram_codebook + sz_encode, in one call.
+sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap,
+                             uint64_t *d_out_bytes, uint8_t *d_codebook16_or_null, int32_t *d_status,
+                             const CompressScratch &w, const DeviceInfo &dev, cudaStream_t s);
 
 }  // namespace sz

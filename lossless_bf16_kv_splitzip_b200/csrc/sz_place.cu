@@ -156,7 +156,8 @@ __device__ void rescan_tile(const PlaceArgs &a, const OvfItem &it, const uint8_t
     if (threadIdx.x == 0 && done != it.cnt) set_status(a.status + k, SZ_ERR_CORRUPT);  // the input changed
 }
 
-// Zero-length segments have no tiles: block 0 writes their header.
+// Zero-length segments have no tiles: block 0 writes their header (their
+// size, like every segment's, is written after the rescan).
 __device__ void place_empty_segments(const PlaceArgs &a) {
     const uint32_t ns = a.batch.segs ? a.batch.n_segs : 1u;
     for (uint32_t k = threadIdx.x; k < ns; k += blockDim.x) {
@@ -173,7 +174,7 @@ __device__ void place_empty_segments(const PlaceArgs &a) {
             continue;
         }
         write_header(a.out + s.out_offset, 0, 0, cb);
-        a.out_bytes[k] = kHeader;
+        a.seg_e[k] = 0;
     }
 }
 
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
         const uint8_t *cb = a.codebooks_in + 16 * (size_t)k;
         if (ps == seg.tile_begin && tid == 0) {
             write_header(out, n, e, cb);
-            a.out_bytes[k] = container_size(n, e);
+            a.seg_e[k] = (uint32_t)e;  // the size is written after the rescan
         }
         const uint64_t pos_off = kHeader + n + (n + 1) / 2;
         uint8_t *pos_base = out + pos_off;
@@ -283,11 +284,15 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
 }
 
 // The tiles the placement listed, spread over the whole GPU, one block per
-// tile at a time.  Nothing listed: every block returns at once.
+// tile at a time (nothing listed: every block goes straight to the end).
+// The last block to finish writes every segment's size: the container size
+// for a segment whose status is still SZ_OK after the encode, the placement
+// and the rescans, else 0.
 template <bool kBatched>
 __global__ void __launch_bounds__(kThreads) rescan_kernel(const PlaceArgs a) {
     __shared__ PlaceShared sh;
     __shared__ uint8_t s_esc[256];
+    __shared__ int s_last;
     const uint32_t count = *a.ovf_count;
     uint32_t cur = 0xFFFFFFFFu;
     for (uint32_t i = blockIdx.x; i < count; i += gridDim.x) {
@@ -301,6 +306,19 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const PlaceArgs a) {
             cur = it.seg;
         }
         rescan_tile<kBatched>(a, it, s_esc, sh);
+    }
+    __syncthreads();  // every status this block sets is set
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_last = atomicAdd(a.blocks_done, 1u) + 1 == gridDim.x;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const uint32_t ns = a.batch.segs ? a.batch.n_segs : 1u;
+    for (uint32_t k = threadIdx.x; k < ns; k += blockDim.x) {
+        const int32_t st = *reinterpret_cast<volatile const int32_t *>(a.status + k);
+        a.out_bytes[k] = st == SZ_OK ? container_size(load_segment(a.batch, k).n_elems, a.seg_e[k]) : 0;
     }
 }
 

@@ -13,19 +13,15 @@
 
 #include "sz_internal.cuh"
 
-namespace sz {
-cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s);
-cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
-}  // namespace sz
-
 using namespace sz;
 
 namespace {
 
 // Scratch layout for one tensor of at most SZ_STATIC_MAX_ELEMS elements
 // (4096 tiles, so at most kMaxRanges = 1024 ranges):
-//   [0, 1024)      exponent counts of the tensor, u32[256]
-//   [1024, 1028)   tiles counted so far
+//   [0, 1024)      exponent counts of the tensor, u32[256]      } cleared
+//   [1024, 1028)   tiles counted so far                         } by every
+//   [1028, 1032)   tiles of complete encode pieces              } call
 //   [1280, 1312)   SegMeta (codebook, escape count)
 //   [1536, ...)    counts of each range's first and last piece, u32[1024][2][256]
 //   then           escape placement of each range, RangeRec[1024]
@@ -33,6 +29,7 @@ constexpr uint64_t kMaxTiles = (SZ_STATIC_MAX_ELEMS + kTile - 1) / kTile;
 constexpr uint64_t kRanges = kMaxTiles < kMaxRanges ? kMaxTiles : kMaxRanges;
 constexpr uint64_t kOffSegHist = 0;
 constexpr uint64_t kOffSegDone = 1024;
+constexpr uint64_t kOffEncDone = 1028;
 constexpr uint64_t kOffMeta = 1280;
 constexpr uint64_t kOffRhist = 1536;
 constexpr uint64_t kOffRrec = kOffRhist + 2048 * kRanges;
@@ -41,30 +38,23 @@ static_assert(kStaticScratchBytes == SZ_STATIC_SCRATCH_BYTES, "header and layout
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-struct StaticDevice {
-    bool ready = false;
-    uint8_t *scratch = nullptr;  // device address of g_static_scratch on that device
-    int sms = 0;
-};
 std::mutex g_static_mu;
-StaticDevice g_static_dev[64];
+uint8_t *g_static_addr[kMaxDevices];  // device address of g_static_scratch, per device
 
 // Once per device, with that device current: the device address of the
 // scratch array (in host code the array's name is not a device address).
-bool static_device(StaticDevice &out) {
+sz_status static_scratch(uint8_t *&out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SZ_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SZ_ERR_INVALID;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    StaticDevice &d = g_static_dev[dev];
-    if (!d.ready) {
+    if (g_static_addr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return false;
-        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
-        d.scratch = static_cast<uint8_t *>(p);
-        d.ready = true;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return SZ_ERR_CUDA;
+        g_static_addr[dev] = static_cast<uint8_t *>(p);
     }
-    out = d;
-    return true;
+    out = g_static_addr[dev];
+    return SZ_OK;
 }
 
 }  // namespace
@@ -76,52 +66,23 @@ extern "C" sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t 
     if (n > SZ_STATIC_MAX_ELEMS) return SZ_ERR_TOO_LARGE;
     if ((n > 0 && (reinterpret_cast<uintptr_t>(d_in) & 15) != 0) || (reinterpret_cast<uintptr_t>(d_out) & 15) != 0)
         return SZ_ERR_ALIGN;
-    if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
-    StaticDevice dev;
-    if (!static_device(dev)) return SZ_ERR_CUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    uint8_t *ws = dev.scratch;
-
+    if (out_cap < 48 + n + (n + 1) / 2) return SZ_ERR_CAPACITY;
+    uint8_t *ws = nullptr;
+    if (const sz_status st = static_scratch(ws)) return st;
+    DeviceInfo dev;
+    if (const sz_status st = device_info(dev)) return st;
     // The array keeps the previous call's contents: the tensor counts and
-    // the tile count are accumulated with atomics and must start at zero;
-    // everything else is overwritten before it is read.
-    if (cudaMemsetAsync(ws + kOffSegHist, 0, 1028, s) != cudaSuccess) return SZ_ERR_CUDA;
-    if (cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s) != cudaSuccess) return SZ_ERR_CUDA;
-    if (cudaMemsetAsync(d_status, 0, sizeof(int32_t), s) != cudaSuccess) return SZ_ERR_CUDA;
-
-    Batch b{};
-    b.segs = nullptr;
-    b.n_segs = 1;
-    b.page_elems = n > 0 ? n : 1;
-    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems);
-    b.n_tiles = segment_tiles(n, b.page_elems);
-    b.single.n_elems = n;
-
-    HistArgs h{};
-    h.sel.batch = b;
-    h.sel.seg_hist = reinterpret_cast<uint32_t *>(ws + kOffSegHist);
-    h.sel.rhist = reinterpret_cast<uint32_t *>(ws + kOffRhist);
-    h.sel.meta = reinterpret_cast<SegMeta *>(ws + kOffMeta);
-    h.sel.rrec = reinterpret_cast<RangeRec *>(ws + kOffRrec);
-    h.sel.range_tiles = plan_ranges(b.n_tiles, (uint64_t)dev.sms).tiles;
-    h.sel.codebooks_out = d_codebook16_or_null;
-    h.base = d_in;
-    h.seg_hist = reinterpret_cast<uint32_t *>(ws + kOffSegHist);
-    h.seg_done = reinterpret_cast<uint32_t *>(ws + kOffSegDone);
-    h.rhist = reinterpret_cast<uint32_t *>(ws + kOffRhist);
-    if (launch_hist(h, false, s) != cudaSuccess) return SZ_ERR_CUDA;
-
-    EncodeArgs a{};
-    a.batch = b;
-    a.base = d_in;
-    a.out = d_out;
-    a.out_cap = out_cap;
-    a.out_bytes = d_out_bytes;
-    a.status = d_status;
-    a.meta = h.sel.meta;
-    a.rrec = h.sel.rrec;
-    a.range_tiles = h.sel.range_tiles;
-    a.wait_limit_ns = 1000000000ull;
-    a.debug_flags = 0;
-    return launch_encode(a, false, s) == cudaSuccess ? SZ_OK : SZ_ERR_CUDA;
+    // the two completion counts are accumulated with atomics and are
+    // cleared first; everything else is overwritten before it is read.
+    CompressScratch cs;
+    cs.zero = ws + kOffSegHist;
+    cs.zero_bytes = kOffEncDone + 4;
+    cs.seg_hist = reinterpret_cast<uint32_t *>(ws + kOffSegHist);
+    cs.seg_done = reinterpret_cast<uint32_t *>(ws + kOffSegDone);
+    cs.enc_done = reinterpret_cast<uint32_t *>(ws + kOffEncDone);
+    cs.meta = reinterpret_cast<SegMeta *>(ws + kOffMeta);
+    cs.rhist = reinterpret_cast<uint32_t *>(ws + kOffRhist);
+    cs.rrec = reinterpret_cast<RangeRec *>(ws + kOffRrec);
+    return compress_pipelined(d_in, n, d_out, out_cap, d_out_bytes, d_codebook16_or_null, d_status, cs, dev,
+                              static_cast<cudaStream_t>(stream));
 }

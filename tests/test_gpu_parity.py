@@ -17,6 +17,7 @@ import pytest
 import kvgen
 import oracle
 from conftest import load_golden
+from oracle_pool import oracle_digests
 
 torch = pytest.importorskip("torch")
 import lossless_bf16_kv_splitzip_b200 as sz  # noqa: E402
@@ -244,6 +245,38 @@ def test_stale_workspace_histogram_is_reported():
     assert int(st.item()) == sz.SZ_ERR_CORRUPT and int(size.item()) == 0
 
 
+@pytest.mark.parametrize("tile", [0, 4, 8])
+def test_stale_workspace_on_several_ranges_keeps_size_zero(tile):
+    """A stream of 9 tiles is encoded by 9 CTAs, one tile each.  Its input
+    changes after the histogram in one tile only, so that tile's CTA finds
+    more escapes than the workspace counted: the status is SZ_ERR_CORRUPT
+    and the size stays 0, whichever CTA finishes the stream last."""
+    n = 8 * 65536 + 5
+    a = kvgen.mixed_small(n, seed=13)
+    cap, wsb = sz.sz_plan(n)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=DEV)
+    cb = torch.empty(16, dtype=torch.uint8, device=DEV)
+    sz.sz_histogram_codebook(to_dev(a), n, cb, None, ws, wsb)
+    torch.cuda.synchronize()
+    code = cb.cpu().numpy()
+    outside = next(e for e in range(1, 255) if e not in set(code.tolist()))
+    b = a.copy()
+    lo = tile * 65536
+    idx = np.arange(lo, min(lo + 65536, n), 97)
+    b[idx] = (b[idx] & 0x807F) | (outside << 7)  # escapes the histogram never saw
+    out = torch.empty(cap, dtype=torch.uint8, device=DEV)
+    size = torch.ones(1, dtype=torch.int64, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sz.sz_encode(to_dev(b), n, cb, out, cap, size, st, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(st.item()) == sz.SZ_ERR_CORRUPT and int(size.item()) == 0
+    # the same workspace still encodes the input it describes
+    sz.sz_encode(to_dev(a), n, cb, out, cap, size, st, ws, wsb)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert out[: int(size.item())].cpu().numpy().tobytes() == oracle.encode(a)
+
+
 # ------------------------------------------------------ corrupt containers
 def corruptions(blob, n):
     b = bytearray(blob)
@@ -350,6 +383,46 @@ def test_stage_wait_times_out_cleanly():
         sz.sz_debug_set_flags(0)
         sz.sz_set_wait_limit_ns(1_000_000_000)
     assert gpu_encode(x) == oracle.encode(x)
+
+
+def test_stage_wait_timeout_on_several_ranges_and_one_pass():
+    """Every stage wait runs out on a stream of 9 CTA ranges (two-pass and
+    one-pass encode) and on a batch of several segments: every status is
+    SZ_ERR_DEVICE_TIMEOUT and every size 0."""
+    n = 8 * 65536 + 5
+    x = kvgen.mixed_small(n, seed=33)
+    lens = [3 * 65536 + 7, 16384, 5 * 65536]
+    streams = [kvgen.mixed_small(m, seed=34 + i) for i, m in enumerate(lens)]
+    starts = [0]
+    for m in lens[:-1]:
+        starts.append(starts[-1] + -(-m // 64) * 64)  # 16-byte aligned pages
+    flat = np.zeros(starts[-1] + lens[-1], np.uint16)
+    for s_, x_ in zip(starts, streams):
+        flat[s_: s_ + x_.size] = x_
+    pool = torch.from_numpy(flat.view(np.int16)).to(DEV)
+    plan = sz.BatchPlan(lens, max(lens), device=DEV)
+    ptrs = torch.from_numpy((np.array(starts) * 2 + pool.data_ptr()).astype(np.int64)).to(DEV)
+    try:
+        sz.sz_set_wait_limit_ns(2_000_000)
+        sz.sz_debug_set_flags(1)
+        out, size, status = sz.encode(to_dev(x))
+        out1, size1, status1 = sz.encode_one_pass(to_dev(x), torch.arange(120, 136, dtype=torch.uint8, device=DEV))
+        plan.encode(ptrs)
+        torch.cuda.synchronize()
+        assert int(status.item()) == sz.SZ_ERR_DEVICE_TIMEOUT and int(size.item()) == 0
+        assert int(status1.item()) == sz.SZ_ERR_DEVICE_TIMEOUT and int(size1.item()) == 0
+        assert plan.enc_status.cpu().tolist() == [sz.SZ_ERR_DEVICE_TIMEOUT] * 3
+        assert plan.sizes.cpu().tolist() == [0, 0, 0]
+    finally:
+        sz.sz_debug_set_flags(0)
+        sz.sz_set_wait_limit_ns(1_000_000_000)
+    assert gpu_encode(x) == oracle.encode(x)
+    plan.encode(ptrs)
+    torch.cuda.synchronize()
+    assert plan.enc_status.abs().sum().item() == 0
+    for k, s_ in enumerate(streams):
+        off, z = int(plan.out_offset[k]), int(plan.sizes[k].item())
+        assert plan.container[off: off + z].cpu().numpy().tobytes() == oracle.encode(s_)
 
 
 def test_decode_stage_wait_times_out_cleanly():
@@ -464,17 +537,22 @@ def test_paged_full_workload4():
 
 @pytest.mark.slow
 def test_paged_full_workload4_adversarial():
+    # uniform random 16-bit patterns in every page: about 94 % escapes, so
+    # every tile writes past the staged escape records; every request's
+    # container is compared with the oracle's
+    import hashlib
     b = kvgen.paged_batch(adversarial=True)
     plan = paged_run(b)
     sizes = plan.sizes.cpu().numpy()
     for r in range(b.n_requests):
         n = int(b.lengths[r]) * kvgen.HEADS * kvgen.HEAD_DIM
         assert sizes[r] <= sz.max_bytes(n)
-    sample = list(range(0, b.n_requests, 16))
     host = plan.container.cpu().numpy()
-    for r in sample:
+    want = oracle_digests([b.request_stream(r) for r in range(b.n_requests)])
+    for r in range(b.n_requests):
         off = int(plan.out_offset[r])
-        assert host[off: off + int(sizes[r])].tobytes() == oracle.encode(b.request_stream(r))
+        got = hashlib.sha256(host[off: off + int(sizes[r])].tobytes()).hexdigest()
+        assert got == want[r], "request %d differs from the oracle" % r
 
 
 @pytest.mark.parametrize("page", [39936, 150016])
