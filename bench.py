@@ -58,7 +58,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
-    p.add_argument("--no-one-pass", action="store_true")
+    p.add_argument("--no-one-pass", action="store_true", help="skip the read-once and codebook-reuse encodes")
+    p.add_argument("--no-workloads", action="store_true", help="skip the compact lines of the other workloads")
     p.add_argument("--tensors", type=int, default=0,
                    help="time only the first T (layer, K/V) tensors (a smaller case for profiling)")
     p.add_argument("--sweep", action="store_true",
@@ -522,6 +523,259 @@ def run_transfer(args):
 
 
 # ------------------------------------------------------------------ our arm
+def host_facts():
+    """Cores and CPU model of the host the CPU baseline runs on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
+def job_config(cfg, world):
+    """The workload's config plus how the job is spread over `world` GPUs:
+    every rank codes its own copy of the workload (units are independent;
+    no collective touches the data path)."""
+    out = dict(cfg)
+    if world == 1:
+        out["parallelism"] = "1 GPU"
+    else:
+        out["parallelism"] = ("replicas x%d: each rank codes its own copy of the workload; the only "
+                              "collectives are the timing barrier and a max all-reduce" % world)
+    return out
+
+
+def accumulate_chunks(inp, sz, dev, chunk_tokens=4096, page_chunks=4):
+    """The workload's cache as it is written during prefill, one plan per
+    prefill chunk for sz_histogram_accumulate_batched.  Contiguous
+    workloads: every chunk of `chunk_tokens` tokens adds, for every (layer,
+    K/V) tensor and head, its token slice (a contiguous run) to the tensor's
+    histogram.  Paged: every request's pages arrive in `page_chunks` runs.
+    Returns [(plan, page pointers, histogram row of each segment)]."""
+    import torch
+    out = []
+    if inp.contiguous:
+        S, n = inp.d_in.shape
+        T = n // (kvgen.HEADS * kvgen.HEAD_DIM)
+        base = inp.d_in.data_ptr()
+        for c0 in range(0, T, chunk_tokens):
+            t = min(chunk_tokens, T - c0)
+            ptrs = [base + 2 * (k * n + (h * T + c0) * kvgen.HEAD_DIM) for k in range(S) for h in range(kvgen.HEADS)]
+            rows = [k for k in range(S) for _ in range(kvgen.HEADS)]
+            p = sz.BatchPlan([t * kvgen.HEAD_DIM] * len(ptrs), t * kvgen.HEAD_DIM, device=dev, buffers=False)
+            out.append((p, torch.tensor(ptrs, dtype=torch.int64, device=dev),
+                        torch.tensor(rows, dtype=torch.int32, device=dev)))
+    else:
+        b, P = inp.batch, kvgen.PAGE_ELEMS
+        base = inp.pool_in.data_ptr()
+        for c in range(page_chunks):
+            lens, ptrs, rows = [], [], []
+            for r in range(b.n_requests):
+                slots = np.array_split(b.page_table[r], page_chunks)[c]
+                if slots.size:
+                    lens.append(int(slots.size) * P)
+                    ptrs.extend(int(base + 2 * P * s_) for s_ in slots)
+                    rows.append(r)
+            p = sz.BatchPlan(lens, P, device=dev, buffers=False)
+            out.append((p, torch.tensor(ptrs, dtype=torch.int64, device=dev),
+                        torch.tensor(rows, dtype=torch.int32, device=dev)))
+    return out
+
+
+def time_events(fn, k, stream):
+    """Mean device time (s) of fn() over k calls, CUDA events on `stream`."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k)]
+    for a0, a1 in ev:
+        a0.record(stream)
+        fn()
+        a1.record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([a0.elapsed_time(a1) for a0, a1 in ev])) / 1e3
+
+
+def read_once_phase(inp, plan, sz, dev, stream, steps, peak):
+    """The read-once encode: histograms accumulated while the cache is
+    written (timed per prefill chunk), then per step the select of the exact
+    codebooks and the one-pass encode.  Its containers must be the two-pass
+    path's bytes.  Returns (dict, the one-pass plan, codebooks)."""
+    import torch
+    chunks = accumulate_chunks(inp, sz, dev)
+    hists = torch.zeros((plan.n_segs, 256), dtype=torch.int32, device=dev)
+
+    def accumulate():
+        hists.zero_()
+        for p, ptrs, rows in chunks:
+            p.accumulate(ptrs, hists, rows, stream)
+
+    accumulate()
+    torch.cuda.synchronize()
+    acc_ok = all(int(p.acc_status.abs().sum()) == 0 for p, _, _ in chunks)
+    # per chunk: device time of each chunk's call, averaged
+    t_acc = []
+    for _ in range(3):
+        for p, ptrs, rows in chunks:
+            t_acc.append(time_events(lambda: p.accumulate(ptrs, hists, rows, stream), 1, stream))
+    accumulate()  # the histograms again (the timing loop added the cache three more times)
+    plan1 = sz.BatchPlan(plan.seg_elems, plan.page_elems, device=dev)
+    cbs = torch.empty((plan.n_segs, 16), dtype=torch.uint8, device=dev)
+
+    def step():
+        sz.sz_select_codebook_batched(plan.n_segs, hists, cbs, None, stream)
+        plan1.encode_one_pass(inp.in_ptrs, cbs, stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    same = bool(torch.equal(plan1.sizes, plan.sizes)) and int(plan1.enc_status.abs().sum()) == 0 and acc_ok
+    same = same and bool(torch.equal(cbs, plan.codebooks[: plan.n_segs]))
+    sizes = plan.sizes.cpu().numpy()
+    for k in range(plan.n_segs):
+        o, z = int(plan.out_offset[k]), int(sizes[k])
+        same = same and bool(torch.equal(plan1.container[o: o + z], plan.container[o: o + z]))
+    t1 = time_events(step, steps, stream)
+    U, comp = inp.U, int(sizes.sum())
+    chunk_bytes = U / len(chunks)
+    ta = float(np.mean(t_acc))
+    res = {"ms": round(t1 * 1e3, 4), "encode_gbs": round(U / t1 / 1e9, 2),
+           "roofline_frac": round((U + comp) / t1 / 1e9 / peak, 4),
+           "roofline_frac_of_spec": round((U + comp) / t1 / 1e9 / SPEC_HBM_GBS, 4),
+           "same_containers_as_two_pass": same, "steps": steps,
+           "launches": "select (1 block per codebook), one-pass encode, escape placement, overflow rescan",
+           "accumulate": {"chunks": len(chunks), "ms_per_chunk": round(ta * 1e3, 4),
+                          "chunk_bytes": int(chunk_bytes), "gbs": round(chunk_bytes / ta / 1e9, 1),
+                          "roofline_frac": round(chunk_bytes / ta / 1e9 / peak, 4),
+                          "what": ("per prefill chunk of 4096 tokens: every (layer, K/V) tensor's 8 head slices "
+                                   "added to its histogram, one launch" if inp.contiguous else
+                                   "per prefill chunk: a quarter of every request's pages added to its "
+                                   "request's histogram, one launch")}}
+    return res, plan1, cbs
+
+
+def reuse_phase(inp, plan, plan1, cbs, stream, steps, peak):
+    """Codebook reuse across layers: layer L's K and V tensors encoded with
+    layer L-1's K and V codebooks (layer 0 keeps its own), one pass.
+    Escapes, ratio and time beside the tensors' own codebooks."""
+    import torch
+    S = plan.n_segs
+    prev = cbs.clone()
+    prev[2:] = cbs[: S - 2]
+    plan1.encode_one_pass(inp.in_ptrs, prev, stream)
+    torch.cuda.synchronize()
+    ok = int(plan1.enc_status.abs().sum()) == 0
+    t = time_events(lambda: plan1.encode_one_pass(inp.in_ptrs, prev, stream), steps, stream)
+    seg_n = np.array(plan.seg_elems, dtype=np.int64)
+    sizes = plan1.sizes.cpu().numpy().astype(np.int64)
+    esc = int(((sizes - (HEADER + seg_n + (seg_n + 1) // 2)) // 5).sum())
+    comp = int(sizes.sum())
+    return {"codebooks": "layer L-1's (K for K, V for V); layer 0 its own", "status_ok": ok,
+            "escape_frac": round(esc / (inp.U // 2), 6), "ratio": round(inp.U / comp, 5),
+            "ms": round(t * 1e3, 4), "encode_gbs": round(inp.U / t / 1e9, 2),
+            "roofline_frac": round((inp.U + comp) / t / 1e9 / peak, 4)}
+
+
+def two_pass_steps(inp, plan, stream, steps, warmup, flush=None, clocks=None, barrier=None):
+    """Warm-up, then `steps` timed steps of histogram + select, encode and
+    decode.  Returns per-step phase times (s) and the clock record."""
+    import torch
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+
+    def step(ev=None):
+        if flush is not None:  # an input that fits L2 is flushed out of it before every step
+            flush.fill_(1)
+        if ev is not None:
+            ev[0].record(stream)
+        plan.histogram(inp.in_ptrs, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        plan.encode_only(inp.in_ptrs, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        plan.decode(inp.out_ptrs, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(plan.enc_status.abs().sum()) or int(plan.dec_status.abs().sum()):
+        raise RuntimeError("device status: encode %s decode %s" % (plan.enc_status.tolist(), plan.dec_status.tolist()))
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.25)  # let the sampler take its first reading
+    for k in range(steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    clock_info = clocks.stop() if clocks else None
+    if barrier:
+        barrier()
+    t_hist = np.array([e[0].elapsed_time(e[1]) for e in evs]) / 1e3
+    t_enc = np.array([e[1].elapsed_time(e[2]) for e in evs]) / 1e3
+    t_dec = np.array([e[2].elapsed_time(e[3]) for e in evs]) / 1e3
+    total_s = evs[0][0].elapsed_time(evs[-1][3]) / 1e3
+    return t_hist, t_enc, t_dec, total_s, clock_info
+
+
+def phase_fracs(U, comp, th, te, td, peak):
+    return {"histogram+select": round(U / th / 1e9 / peak, 4),
+            "encode_kernel": round((U + comp) / te / 1e9 / peak, 4),
+            "encode_end_to_end": round((U + comp) / (th + te) / 1e9 / peak, 4),
+            "decode": round((U + comp) / td / 1e9 / peak, 4)}
+
+
+def other_workload(w, dev, sz, stream, steps, peak):
+    """A compact line for another workload: ratio, escapes, phase fractions
+    of the measured peak, the read-once encode, and for the paged batch the
+    adversarial pass's worst-case bound."""
+    import types
+
+    import torch
+    inp = Inputs(types.SimpleNamespace(workload=w, tensors=0), dev, sz)
+    plan = inp.plan
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if inp.flush_l2 else None
+    th, te, td, _, _ = two_pass_steps(inp, plan, stream, steps, 3, flush)
+    th, te, td = float(th.mean()), float(te.mean()), float(td.mean())
+    seg_n = np.array(plan.seg_elems, dtype=np.int64)
+    sizes = plan.sizes.cpu().numpy().astype(np.int64)
+    comp = int(sizes.sum())
+    esc = int(((sizes - (HEADER + seg_n + (seg_n + 1) // 2)) // 5).sum())
+    U = inp.U
+    res = {"config": inp.cfg["workload"], "bytes": U, "ratio": round(U / comp, 5),
+           "escape_frac": round(esc / (U // 2), 6), "round_trip": inp.round_trip_ok(), "steps": steps,
+           "ms": {"histogram+select": round(th * 1e3, 4), "encode_kernel": round(te * 1e3, 4),
+                  "decode": round(td * 1e3, 4)},
+           "frac": phase_fracs(U, comp, th, te, td, peak)}
+    ro, plan1, cbs = read_once_phase(inp, plan, sz, dev, stream, steps, peak)
+    res["encode_read_once"] = {k: ro[k] for k in ("ms", "roofline_frac", "same_containers_as_two_pass")}
+    res["encode_read_once"]["accumulate_frac"] = ro["accumulate"]["roofline_frac"]
+    if inp.contiguous and w == 3:
+        res["codebook_reuse"] = reuse_phase(inp, plan, plan1, cbs, stream, steps, peak)
+    del plan1
+    if w == 4:  # adversarial pass: uniform random 16-bit patterns in the same pages
+        b = kvgen.paged_batch(adversarial=True)
+        for r in range(b.n_requests):
+            inp.pool_in[torch.from_numpy(b.page_table[r]).to(dev)] = torch.from_numpy(b.pages[r].view(np.int16)).to(dev)
+        plan.encode(inp.in_ptrs, stream)
+        torch.cuda.synchronize()
+        sz_adv = plan.sizes.cpu().numpy().astype(np.int64)
+        bound = HEADER + seg_n + (seg_n + 1) // 2 + 5 * (seg_n - (seg_n + 15) // 16)
+        res["adversarial"] = {"status_ok": int(plan.enc_status.abs().sum()) == 0,
+                              "within_bound": bool((sz_adv <= bound).all()),
+                              "max_size_over_bound": round(float((sz_adv / bound).max()), 6),
+                              "ratio": round(U / int(sz_adv.sum()), 5)}
+    del inp, plan, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -555,51 +809,17 @@ def main():
             dist.barrier(device_ids=[local])
 
     inp = Inputs(args, dev, sz)
-    cfg, plan, in_ptrs, out_ptrs = inp.cfg, inp.plan, inp.in_ptrs, inp.out_ptrs
+    cfg, plan, in_ptrs = inp.cfg, inp.plan, inp.in_ptrs
     U = inp.U  # uncompressed bytes per step on this rank
     seg_n = np.array(plan.seg_elems, dtype=np.int64)
     S = plan.n_segs
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if inp.flush_l2 else None
-
-    def step(ev=None):
-        if flush is not None:  # an input that fits L2 is flushed out of it before every step
-            flush.fill_(1)
-        if ev is not None:
-            ev[0].record(stream)
-        plan.histogram(in_ptrs, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        plan.encode_only(in_ptrs, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        plan.decode(out_ptrs, stream)
-        if ev is not None:
-            ev[3].record(stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize(dev)
-    if int(plan.enc_status.abs().sum()) or int(plan.dec_status.abs().sum()):
-        raise RuntimeError("device status: encode %s decode %s" % (plan.enc_status.tolist(), plan.dec_status.tolist()))
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
     clocks = ClockSampler(vis.split(",")[local] if vis else str(local))
-    barrier()
-    torch.cuda.synchronize(dev)
-    clocks.start()
-    time.sleep(0.25)  # let the sampler take its first reading
-    for k in range(args.steps):
-        step(evs[k])
-    torch.cuda.synchronize(dev)
-    clock_info = clocks.stop()
-    barrier()
 
-    t_hist = np.array([e[0].elapsed_time(e[1]) for e in evs]) / 1e3
-    t_enc = np.array([e[1].elapsed_time(e[2]) for e in evs]) / 1e3
-    t_dec = np.array([e[2].elapsed_time(e[3]) for e in evs]) / 1e3
-    total_s = evs[0][0].elapsed_time(evs[-1][3]) / 1e3
+    t_hist, t_enc, t_dec, total_s, clock_info = two_pass_steps(inp, plan, stream, args.steps, args.warmup, flush,
+                                                               clocks, barrier)
     ms_step = total_s / args.steps * 1e3
     if flush is not None:  # the flushes between steps are not the codec's time
         ms_step = float(np.mean(t_hist + t_enc + t_dec)) * 1e3
@@ -653,34 +873,16 @@ def main():
                 "spec_peak": SPEC_HBM_GBS, "frac_of_spec": roof[dom]["frac_of_spec"],
                 "peak_kind": peak_kind + " (copy, MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"}
 
-    # ---- one pass with the codebooks kept from the timed steps (codebook
-    # reuse): the input is read once; the containers must be the same bytes
-    one_pass = None
+    # ---- the read-once encode (histograms kept while the cache is written,
+    # exact codebooks, one pass) and the cost of reusing the previous
+    # layer's codebooks instead
+    read_once = reuse = None
+    k1 = max(1, min(args.steps, 50))
     if not args.no_one_pass:
-        plan1 = sz.BatchPlan(plan.seg_elems, plan.page_elems, device=dev)
-        cbs = plan.codebooks.clone()
-        for _ in range(3):
-            plan1.encode_one_pass(in_ptrs, cbs, stream)
-        torch.cuda.synchronize(dev)
-        same = bool(torch.equal(plan1.sizes, plan.sizes)) and int(plan1.enc_status.abs().sum()) == 0
-        for k in range(S):
-            o, z = int(plan.out_offset[k]), int(sizes[k])
-            same = same and bool(torch.equal(plan1.container[o: o + z], plan.container[o: o + z]))
-        k1 = max(1, min(args.steps, 50))
-        ev1 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(k1)]
-        for a0, a1 in ev1:
-            a0.record(stream)
-            plan1.encode_one_pass(in_ptrs, cbs, stream)
-            a1.record(stream)
-        torch.cuda.synchronize(dev)
-        t1 = float(np.mean([a0.elapsed_time(a1) for a0, a1 in ev1])) / 1e3
-        one_pass = {"encode_gbs": round(U / t1 / 1e9, 2), "ms": round(t1 * 1e3, 4),
-                    "roofline_frac": round((U + comp) / t1 / 1e9 / peak, 4),
-                    "roofline_frac_of_spec": round((U + comp) / t1 / 1e9 / SPEC_HBM_GBS, 4),
-                    "same_containers_as_two_pass": same, "steps": k1,
-                    "codebooks": "kept from the two-pass encode of the same tensors",
-                    "launches": "one-pass encode, escape placement, overflow rescan"}
-        del plan1
+        read_once, plan1, cbs = read_once_phase(inp, plan, sz, dev, stream, k1, peak)
+        if inp.contiguous and S > 2:
+            reuse = reuse_phase(inp, plan, plan1, cbs, stream, k1, peak)
+        del plan1, cbs
 
     # ---- end to end: pinned host buffers, copies inside the timed region.
     # The cache goes up, is encoded, its containers come down and go up
@@ -721,23 +923,34 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(inp, args.cpu_seconds)
+        cpu.update(host_facts())
+
+    # ---- the other workloads, fewer steps each (rank 0, one GPU)
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads and args.tensors <= 0:
+        del inp, plan, flush
+        torch.cuda.empty_cache()
+        workloads = {}
+        for w in (1, 3, 4):
+            if w != args.workload:
+                workloads[WORKLOAD_NAMES[w]] = other_workload(w, dev, sz, stream, min(args.steps, 10), peak)
 
     if rank == 0:
         value = world * U / (ms_step / 1e3) / 1e9
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "u16", "data": "synthetic", "config": cfg,
+            "vs_baseline": None, "dtype": "u16", "data": "synthetic", "config": job_config(cfg, world),
             "encode_gbs": round(U / encode_s / 1e9, 2), "decode_gbs": round(U / td / 1e9, 2),
             "encode_roofline_frac": round(enc_e2e_bytes / encode_s / 1e9 / peak, 4),
             "decode_roofline_frac": roof["decode"]["frac"],
             "encode_roofline_frac_of_spec": round(enc_e2e_bytes / encode_s / 1e9 / SPEC_HBM_GBS, 4),
             "decode_roofline_frac_of_spec": roof["decode"]["frac_of_spec"],
-            "encode_one_pass": one_pass,
+            "encode_read_once": read_once, "codebook_reuse": reuse,
             "ratio": round(U / comp, 5), "escape_frac": round(esc / (U // 2), 6),
             "roofline": roofline, "roofline_phases": roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * args.steps,  # hist, encode, esc_index, decode
-            "clocks": clock_info, "parity": parity,
+            "clocks": clock_info, "parity": parity, "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

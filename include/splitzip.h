@@ -346,6 +346,63 @@ sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, 
                                      uint64_t *d_out_bytes, int32_t *d_status, void *d_ws, uint64_t ws_bytes,
                                      void *stream);
 
+/* ------------------------- histogram kept while the cache is written */
+/*
+ * The codebook is each tensor's own top 16 (explainer section 3), so the
+ * two-call path reads the input twice: once to count exponents, once to
+ * encode.  A serving engine can instead count each chunk of KV as it is
+ * written during prefill, into a running histogram per tensor or request;
+ * at transfer time sz_select_codebook(_batched) turns the histograms into
+ * the exact codebooks and sz_encode_one_pass(_batched) reads the cache
+ * once.  The containers are byte for byte those of the two-call path
+ * (explainer, "Le probleme des methodes d'envoi actuelles": the compressor
+ * must keep pace with the prefill team producing the notes).
+ *
+ * sz_histogram_accumulate -- add the exponent counts of d_in[0..n) to the
+ * caller's uint32[256] histogram (zero it before the first chunk, e.g.
+ * with cudaMemsetAsync).  No workspace; n = 0 enqueues nothing.  The caller
+ * keeps each histogram's total below 2^32 (the container's element limit).
+ *   d_in            n BF16 values, 16-byte aligned
+ *   d_hist256       in/out uint32[256], 4-byte aligned
+ */
+sz_status sz_histogram_accumulate(const uint16_t *d_in, uint64_t n, uint32_t *d_hist256, void *stream);
+
+/*
+ * sz_histogram_accumulate_batched -- add the exponent counts of every
+ * segment of a batch (newly written pages or chunks, laid out as for
+ * sz_plan_batched: d_segs from a plan of the new data's lengths) to the
+ * caller's histograms, one launch.
+ *   d_hist_index_or_null  uint32[n_segs]: segment k adds to histogram
+ *                   d_hist_index[k] (several segments may share one, e.g.
+ *                   the eight heads' slices of one tensor's new tokens);
+ *                   NULL: segment k adds to histogram k
+ *   d_hists         in/out uint32[rows][256], 4-byte aligned
+ *   d_status        out int32[n_segs]: SZ_ERR_ALIGN for a misaligned page
+ *                   (that segment's counts are then incomplete); set to
+ *                   SZ_OK first
+ */
+sz_status sz_histogram_accumulate_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                                          const uint16_t *const *d_pages, uint64_t page_elems,
+                                          const uint32_t *d_hist_index_or_null, uint32_t *d_hists,
+                                          int32_t *d_status, void *stream);
+
+/*
+ * sz_select_codebook -- the codebook of a histogram: the 16 exponents
+ * first in (count descending, exponent ascending) order, code k = the k-th
+ * (explainer section 3), the same choice sz_histogram_codebook makes.
+ *   d_hist256          uint32[256]
+ *   d_codebook16       out: 16 bytes
+ *   d_escapes_or_null  optional out: uint64 escape count (total - the 16
+ *                      codebook counts), 8-byte aligned
+ * sz_select_codebook_batched does the same for n_hists histograms
+ * (uint32[n_hists][256] -> uint8[n_hists][16], uint64[n_hists]), one
+ * block per histogram.
+ */
+sz_status sz_select_codebook(const uint32_t *d_hist256, uint8_t *d_codebook16, uint64_t *d_escapes_or_null,
+                             void *stream);
+sz_status sz_select_codebook_batched(uint32_t n_hists, const uint32_t *d_hists, uint8_t *d_codebooks,
+                                     uint64_t *d_escapes_or_null, void *stream);
+
 /* ------------------------------------------------------- no-allocation path */
 /*
  * sz_encode_static -- the whole compression of one tensor (histogram,

@@ -26,7 +26,8 @@ __all__ = [
     "SzError", "sz_segment", "sz_plan", "sz_histogram_codebook", "sz_encode", "sz_compress", "sz_decode",
     "sz_plan_batched", "sz_histogram_codebook_batched", "sz_encode_batched", "sz_decode_batched",
     "sz_encode_static", "sz_plan_one_pass", "sz_encode_one_pass", "sz_workspace_one_pass_batched",
-    "sz_encode_one_pass_batched", "sz_set_wait_limit_ns", "sz_debug_set_flags", "sz_tile_elems",
+    "sz_encode_one_pass_batched", "sz_histogram_accumulate", "sz_histogram_accumulate_batched",
+    "sz_select_codebook", "sz_select_codebook_batched", "select_codebooks", "sz_set_wait_limit_ns", "sz_debug_set_flags", "sz_tile_elems",
     "sz_version", "encode", "compress", "encode_one_pass", "decode", "BatchPlan", "lib",
     "HEADER_BYTES", "max_bytes", "STATUS",
 ]
@@ -79,6 +80,10 @@ def lib():
             "sz_encode_one_pass": [vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
             "sz_workspace_one_pass_batched": [u32, u64, pu64],
             "sz_encode_one_pass_batched": [u32, vp, u64, vp, u64, vp, vp, u64, vp, vp, vp, u64, vp],
+            "sz_histogram_accumulate": [vp, u64, vp, vp],
+            "sz_histogram_accumulate_batched": [u32, vp, u64, vp, u64, vp, vp, vp, vp],
+            "sz_select_codebook": [vp, vp, vp, vp],
+            "sz_select_codebook_batched": [u32, vp, vp, vp, vp],
             "sz_set_wait_limit_ns": [u64],
             "sz_debug_set_flags": [u32],
         }
@@ -219,6 +224,27 @@ def sz_encode_one_pass_batched(n_segs, d_segs, n_tiles, d_pages, page_elems, d_c
                                             _s(stream)), "sz_encode_one_pass_batched")
 
 
+def sz_histogram_accumulate(d_in, n, d_hist256, stream=None):
+    _check(lib().sz_histogram_accumulate(_p(d_in), n, _p(d_hist256), _s(stream)), "sz_histogram_accumulate")
+
+
+def sz_histogram_accumulate_batched(n_segs, d_segs, n_tiles, d_pages, page_elems, d_hist_index, d_hists, d_status,
+                                    stream=None):
+    _check(lib().sz_histogram_accumulate_batched(n_segs, _p(d_segs), n_tiles, _p(d_pages), page_elems,
+                                                 _p(d_hist_index), _p(d_hists), _p(d_status), _s(stream)),
+           "sz_histogram_accumulate_batched")
+
+
+def sz_select_codebook(d_hist256, d_codebook16, d_escapes=None, stream=None):
+    _check(lib().sz_select_codebook(_p(d_hist256), _p(d_codebook16), _p(d_escapes), _s(stream)),
+           "sz_select_codebook")
+
+
+def sz_select_codebook_batched(n_hists, d_hists, d_codebooks, d_escapes=None, stream=None):
+    _check(lib().sz_select_codebook_batched(n_hists, _p(d_hists), _p(d_codebooks), _p(d_escapes), _s(stream)),
+           "sz_select_codebook_batched")
+
+
 def sz_set_wait_limit_ns(limit_ns: int):
     _check(lib().sz_set_wait_limit_ns(limit_ns), "sz_set_wait_limit_ns")
 
@@ -326,6 +352,20 @@ def encode_one_pass(x, codebook, stream=None, workspace=None):
     return out, size, status
 
 
+def select_codebooks(hists, stream=None, escapes=True):
+    """Codebooks of caller histograms (uint32/int32 CUDA tensor [rows, 256]
+    or [256]).  Returns (codebooks uint8 [rows, 16], escape counts int64
+    [rows] or None)."""
+    torch = _torch()
+    if not hists.is_contiguous() or hists.element_size() != 4 or hists.numel() % 256:
+        raise ValueError("hists must be a contiguous 32-bit tensor of rows of 256 counts")
+    rows = hists.numel() // 256
+    cbs = torch.empty((max(rows, 1), 16), dtype=torch.uint8, device=hists.device)
+    esc = torch.empty(max(rows, 1), dtype=torch.int64, device=hists.device) if escapes else None
+    sz_select_codebook_batched(rows, hists, cbs, esc, stream)
+    return cbs[:rows], (esc[:rows] if esc is not None else None)
+
+
 def decode(container, n, out=None, stream=None, workspace=None):
     """Decode a container (uint8 CUDA tensor) of n elements into an int16
     tensor (bit patterns).  Returns (out, status int32 tensor [1])."""
@@ -348,8 +388,12 @@ class BatchPlan:
     """Buffers of one batched encode/decode: the segment table (host and
     device), container buffer, workspace, per-segment sizes and statuses."""
 
-    def __init__(self, seg_elems, page_elems, device="cuda"):
+    def __init__(self, seg_elems, page_elems, device="cuda", buffers=True):
+        """buffers=False: only the segment table and the statuses (a plan
+        of newly written data for ``accumulate``, which needs no container
+        buffer or workspace)."""
         torch = _torch()
+        self.device = torch.device(device)
         self.seg_elems = [int(v) for v in seg_elems]
         self.page_elems = int(page_elems)
         segs, self.total_pages, self.n_tiles, self.out_bytes, self.ws_bytes = sz_plan_batched(
@@ -361,8 +405,10 @@ class BatchPlan:
         self.tile_begin = raw[:, 3].copy()
         self.page_begin = raw[:, 1].copy()
         self.d_segs = torch.from_numpy(raw.copy().view(np.int64)).to(device)
-        self.container = torch.empty(max(self.out_bytes, 16), dtype=torch.uint8, device=device)
-        self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
+        self.container = self.ws = None
+        if buffers:
+            self.container = torch.empty(max(self.out_bytes, 16), dtype=torch.uint8, device=device)
+            self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device)
         self.sizes = torch.zeros(max(self.n_segs, 1), dtype=torch.int64, device=device)
         self.codebooks = torch.zeros((max(self.n_segs, 1), 16), dtype=torch.uint8, device=device)
         self.enc_status = torch.zeros(max(self.n_segs, 1), dtype=torch.int32, device=device)
@@ -387,10 +433,23 @@ class BatchPlan:
         torch = _torch()
         if getattr(self, "ws1", None) is None:
             wb = sz_workspace_one_pass_batched(self.n_segs, self.n_tiles)
-            self.ws1 = torch.empty(max(wb, 256), dtype=torch.uint8, device=self.container.device)
+            self.ws1 = torch.empty(max(wb, 256), dtype=torch.uint8, device=self.device)
         sz_encode_one_pass_batched(self.n_segs, self.d_segs, self.n_tiles, d_page_ptrs, self.page_elems, d_codebooks,
                                    self.container, self.container.numel(), self.sizes, self.enc_status, self.ws1,
                                    self.ws1.numel(), stream)
+
+    def accumulate(self, d_page_ptrs, d_hists, d_hist_index=None, stream=None):
+        """Add every segment's exponent counts (the plan describes newly
+        written data) to the caller's histograms d_hists (32-bit [rows, 256]
+        on the device), segment k into row d_hist_index[k] (uint32/int32
+        [n_segs]) or row k.  Per-segment status in self.acc_status."""
+        torch = _torch()
+        if getattr(self, "acc_status", None) is None:
+            self.acc_status = torch.zeros(max(self.n_segs, 1), dtype=torch.int32, device=self.device)
+        if not d_hists.is_contiguous() or d_hists.element_size() != 4:
+            raise ValueError("d_hists must be a contiguous 32-bit tensor")
+        sz_histogram_accumulate_batched(self.n_segs, self.d_segs, self.n_tiles, d_page_ptrs, self.page_elems,
+                                        d_hist_index, d_hists, self.acc_status, stream)
 
     def decode(self, d_page_ptrs, stream=None, container=None):
         """Decode every segment into the pages d_page_ptrs lists.  container:

@@ -8,6 +8,8 @@
 
 namespace sz {
 cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s);
+cudaError_t launch_select(const uint32_t *hists, uint32_t n_hists, uint8_t *codebooks, uint64_t *escapes,
+                          cudaStream_t s);
 cudaError_t launch_reselect(const ReselectArgs &a, cudaStream_t s);
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s);
 cudaError_t launch_encode_one_pass(const EncodeArgs &a, bool batched, cudaStream_t s);
@@ -570,6 +572,60 @@ sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, 
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     return one_pass(make_batch(n_segs, d_segs, n_tiles, page_elems), d_pages, nullptr, d_codebooks, d_out, out_cap,
                     d_out_bytes, d_status, d_ws, w, static_cast<cudaStream_t>(stream));
+}
+
+sz_status sz_histogram_accumulate(const uint16_t *d_in, uint64_t n, uint32_t *d_hist256, void *stream) {
+    if (!d_hist256 || (n > 0 && !d_in)) return SZ_ERR_NULL;
+    if (n > kMaxElems) return SZ_ERR_TOO_LARGE;
+    if ((n > 0 && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_hist256) & 3) != 0) return SZ_ERR_ALIGN;
+    if (n == 0) return SZ_OK;
+    DeviceInfo dev;
+    if (const sz_status st = device_info(dev)) return st;
+    HistArgs h{};
+    h.sel.batch = single_batch(n);
+    h.sel.range_tiles = plan_ranges(h.sel.batch.n_tiles, (uint64_t)dev.sms).tiles;
+    h.base = d_in;
+    h.accum = d_hist256;
+    return cuda_status(launch_hist(h, false, static_cast<cudaStream_t>(stream)));
+}
+
+sz_status sz_histogram_accumulate_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles,
+                                          const uint16_t *const *d_pages, uint64_t page_elems,
+                                          const uint32_t *d_hist_index_or_null, uint32_t *d_hists,
+                                          int32_t *d_status, void *stream) {
+    if (n_segs == 0) return SZ_OK;
+    if (!d_segs || !d_hists || !d_status || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
+    if (page_elems == 0) return SZ_ERR_INVALID;
+    if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
+    if ((reinterpret_cast<uintptr_t>(d_hists) & 3) != 0) return SZ_ERR_ALIGN;
+    DeviceInfo dev;
+    if (const sz_status st = device_info(dev)) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
+    if (n_tiles == 0) return SZ_OK;
+    HistArgs h{};
+    h.sel.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
+    h.sel.range_tiles = plan_ranges(n_tiles, (uint64_t)dev.sms).tiles;
+    h.pages = d_pages;
+    h.status = d_status;
+    h.accum = d_hists;
+    h.accum_index = d_hist_index_or_null;
+    return cuda_status(launch_hist(h, true, s));
+}
+
+sz_status sz_select_codebook(const uint32_t *d_hist256, uint8_t *d_codebook16, uint64_t *d_escapes_or_null,
+                             void *stream) {
+    return sz_select_codebook_batched(1, d_hist256, d_codebook16, d_escapes_or_null, stream);
+}
+
+sz_status sz_select_codebook_batched(uint32_t n_hists, const uint32_t *d_hists, uint8_t *d_codebooks,
+                                     uint64_t *d_escapes_or_null, void *stream) {
+    if (n_hists == 0) return SZ_OK;
+    if (!d_hists || !d_codebooks) return SZ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(d_hists) & 3) != 0 || (reinterpret_cast<uintptr_t>(d_escapes_or_null) & 7) != 0)
+        return SZ_ERR_ALIGN;
+    return cuda_status(launch_select(d_hists, n_hists, d_codebooks, d_escapes_or_null,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 sz_status sz_set_wait_limit_ns(uint64_t limit_ns) {

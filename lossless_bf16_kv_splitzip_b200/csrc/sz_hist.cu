@@ -56,6 +56,19 @@ struct SelShared {
     uint8_t cb[16];
 };
 
+// Rank of exponent `tid` (count c) among the 256 counts in cnt[] in the
+// order (count descending, exponent ascending): the number of exponents
+// before it.  Ranks 0..15 are the codebook.
+__device__ __forceinline__ uint32_t exponent_rank(const uint32_t *cnt, uint32_t c, uint32_t tid) {
+    uint32_t rank = 0;
+#pragma unroll 8
+    for (uint32_t u = 0; u < 256; ++u) {
+        const uint32_t cu = cnt[u];
+        rank += (cu > c) || (cu == c && u < tid);
+    }
+    return rank;
+}
+
 // Codebook, escape count and range records of segment k, by the kThreads
 // threads of one block (every one of them must call it).  Thread t holds
 // exponent t: its rank is the number of exponents before it in (count
@@ -76,12 +89,7 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
     ss.cnt[tid] = c;
     __syncthreads();
     if (codebook_in == nullptr) {
-        uint32_t rank = 0;
-#pragma unroll 8
-        for (uint32_t u = 0; u < 256; ++u) {
-            const uint32_t cu = ss.cnt[u];
-            rank += (cu > c) || (cu == c && u < tid);
-        }
+        const uint32_t rank = exponent_rank(ss.cnt, c, tid);
         if (rank < 16) ss.cb[rank] = (uint8_t)tid;
     } else if (tid < 16) {
         ss.cb[tid] = codebook_in[tid];
@@ -215,7 +223,10 @@ __device__ void empty_segments(const HistArgs &h) {
 // elements); that build is given registers for 3 blocks per SM -- measured
 // 0.70 -> 0.86 of the copy bandwidth on 16-token pages, while the same
 // bound costs 8 % on 65,536-element tiles, which keep the default build.
-template <bool kBatched, bool kSmallTiles>
+// kAccum: the accumulate mode -- each piece's counts are added to the
+// caller's histogram of its segment (a.accum, row a.accum_index[k] or k);
+// no range records, no completion count, no select.
+template <bool kBatched, bool kSmallTiles, bool kAccum>
 __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(const HistArgs a) {
     extern __shared__ __align__(128) uint32_t s_hist[];  // kHistWords
     __shared__ SegCache s_segc;
@@ -225,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
 
     for (uint32_t i = threadIdx.x; i < kHistWords; i += kThreads) s_hist[i] = 0;
     seg_cache_fill(s_segc, batch);  // ends with __syncthreads
-    if (blockIdx.x == 0) empty_segments(a);
+    if (!kAccum && blockIdx.x == 0) empty_segments(a);
 
     const uint32_t tid = threadIdx.x;
     const uint32_t col = smem_u32(s_hist) + (tid & 31) * 4;
@@ -284,6 +295,12 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
         for (uint32_t i = 0; i < 32; ++i) sum += s_hist[tid * 32 + ((i + tid) & 31)];
         const uint32_t acc = sum - prev;
         prev = sum;
+        if (kAccum) {
+            const size_t row = a.accum_index ? a.accum_index[k] : k;
+            if (acc) atomicAdd(&a.accum[row * 256 + tid], acc);
+            __syncthreads();  // folds done before the next piece's counts land
+            continue;
+        }
         if (ps == t_begin) a.rhist[(blockIdx.x * 2ull) * 256 + tid] = acc;
         else if (pe == t_end) a.rhist[(blockIdx.x * 2ull + 1) * 256 + tid] = acc;
         if (acc) atomicAdd(&a.seg_hist[(size_t)k * 256 + tid], acc);
@@ -320,19 +337,70 @@ __global__ void __launch_bounds__(kThreads) reselect_kernel(const ReselectArgs a
     select_segment(a.sel, 0, a.codebook_in, s_sel);
 }
 
+// Codebook of each of a list of caller histograms (one block per
+// histogram): the 16 exponents of rank 0..15 and, optionally, the escape
+// count = the histogram's total - the codebook's counts.
+__global__ void __launch_bounds__(kThreads) select_kernel(const uint32_t *hists, uint8_t *codebooks,
+                                                          uint64_t *escapes) {
+    __shared__ uint32_t s_cnt[256];
+    __shared__ unsigned long long s_sum[2][kWarps];  // [0]: all counts, [1]: codebook counts
+    const uint32_t tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const uint32_t c = hists[(size_t)blockIdx.x * 256 + tid];
+    s_cnt[tid] = c;
+    __syncthreads();
+    const uint32_t rank = exponent_rank(s_cnt, c, tid);
+    if (rank < 16) codebooks[(size_t)blockIdx.x * 16 + rank] = (uint8_t)tid;
+    if (escapes == nullptr) return;
+    unsigned long long all = c, top = rank < 16 ? c : 0u;
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) {
+        all += __shfl_down_sync(0xFFFFFFFFu, all, d);
+        top += __shfl_down_sync(0xFFFFFFFFu, top, d);
+    }
+    if (lane == 0) {
+        s_sum[0][wid] = all;
+        s_sum[1][wid] = top;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        unsigned long long ta = 0, tt = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            ta += s_sum[0][w];
+            tt += s_sum[1][w];
+        }
+        escapes[blockIdx.x] = ta - tt;
+    }
+}
+
 // ------------------------------------------------------------ launchers
+template <bool kAccum>
+void launch_hist_t(const HistArgs &a, bool batched, int grid, size_t smem, cudaStream_t s) {
+    const bool small = a.sel.batch.page_elems <= kSub;
+    if (batched && small)
+        hist_kernel<true, true, kAccum><<<grid, kThreads, smem, s>>>(a);
+    else if (batched)
+        hist_kernel<true, false, kAccum><<<grid, kThreads, smem, s>>>(a);
+    else if (small)
+        hist_kernel<false, true, kAccum><<<grid, kThreads, smem, s>>>(a);
+    else
+        hist_kernel<false, false, kAccum><<<grid, kThreads, smem, s>>>(a);
+}
+
+// a.accum set: the accumulate mode
 cudaError_t launch_hist(const HistArgs &a, bool batched, cudaStream_t s) {
     const int grid = (int)umax64(1, div_up(a.sel.batch.n_tiles, a.sel.range_tiles));
     const size_t smem = kHistWords * sizeof(uint32_t);
-    const bool small = a.sel.batch.page_elems <= kSub;
-    if (batched && small)
-        hist_kernel<true, true><<<grid, kThreads, smem, s>>>(a);
-    else if (batched)
-        hist_kernel<true, false><<<grid, kThreads, smem, s>>>(a);
-    else if (small)
-        hist_kernel<false, true><<<grid, kThreads, smem, s>>>(a);
+    if (a.accum != nullptr)
+        launch_hist_t<true>(a, batched, grid, smem, s);
     else
-        hist_kernel<false, false><<<grid, kThreads, smem, s>>>(a);
+        launch_hist_t<false>(a, batched, grid, smem, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select(const uint32_t *hists, uint32_t n_hists, uint8_t *codebooks, uint64_t *escapes,
+                          cudaStream_t s) {
+    if (n_hists == 0) return cudaSuccess;
+    select_kernel<<<n_hists, kThreads, 0, s>>>(hists, codebooks, escapes);
     return cudaGetLastError();
 }
 

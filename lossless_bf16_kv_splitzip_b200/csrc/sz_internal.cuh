@@ -338,6 +338,8 @@ struct HistArgs {
     uint32_t *seg_done;            // [n_segs] tiles counted so far, zero on entry
     uint32_t *rhist;               // [ranges][2][256]
     int32_t *status;               // [n_segs] or nullptr
+    uint32_t *accum;               // accumulate mode: caller histograms [rows][256] (else nullptr)
+    const uint32_t *accum_index;   // accumulate mode: row of segment k (nullptr: row k)
 };
 
 // Select with a caller codebook (single tensor), ahead of the encode.

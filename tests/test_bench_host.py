@@ -105,3 +105,18 @@ def test_committed_summaries_parse(phase):
     assert int(fields["traffic_per_full_launch_bytes"]) > 0
     sha = fields["kernel_source_sha256"].split(" ")[0]
     assert len(sha) == 16 and int(sha, 16) >= 0
+
+
+def test_job_config_states_the_spread_over_gpus():
+    cfg = {"workload": "llama3-8b-kv-32k", "bytes": 4}
+    one = bench.job_config(cfg, 1)
+    assert one["parallelism"] == "1 GPU" and one["workload"] == cfg["workload"]
+    eight = bench.job_config(cfg, 8)
+    assert "replicas x8" in eight["parallelism"] and "each rank codes its own copy" in eight["parallelism"]
+    assert "parallelism" not in cfg  # the workload's own config is left as it was
+
+
+def test_host_facts_name_cores_and_model():
+    f = bench.host_facts()
+    assert f["host_cores"] == os.cpu_count()
+    assert f["cpu_model"] is None or isinstance(f["cpu_model"], str)
