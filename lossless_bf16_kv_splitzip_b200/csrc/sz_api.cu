@@ -49,11 +49,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 //   meta       SegMeta[S]      codebook and escape count per segment
 //   rhist      u32[G][2][256]  counts of each range's first and last piece
 //   rrec       RangeRec[G]     escape placement of each range's pieces
-//   sub_start  u32[4T + S]     first escape index of each sub-tile (decode; 4 = sub-tiles per tile)
+//   sub_start  u32[ST + S]     first escape index of each sub-tile (decode; S = sub-tiles per tile)
 struct Ws {
     uint64_t seg_hist, seg_done, enc_done, meta, rhist, rrec, sub_start, total;
 };
-Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
+Ws ws_layout(uint64_t n_segs, uint64_t n_tiles, uint64_t tile_subs) {
     const uint64_t g = umin64(n_tiles, kMaxRanges);
     Ws w;
     w.seg_hist = 0;
@@ -63,7 +63,7 @@ Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
     w.rhist = round_up(w.meta + sizeof(SegMeta) * n_segs, kAlign);
     w.rrec = round_up(w.rhist + 2048 * g, kAlign);
     w.sub_start = round_up(w.rrec + sizeof(RangeRec) * g, kAlign);
-    w.total = round_up(w.sub_start + 4 * (kSubsPerTile * n_tiles + n_segs), kAlign);
+    w.total = round_up(w.sub_start + 4 * (tile_subs * n_tiles + n_segs), kAlign);
     return w;
 }
 
@@ -75,11 +75,11 @@ Ws ws_layout(uint64_t n_segs, uint64_t n_tiles) {
 //   seg_e     u32[S]              escape count of each segment
 //   tile_cnt  u32[T]              escapes of each tile
 //   ovf       OvfItem[T]          tiles whose records overflowed their slot
-//   slots     u32[T][kSlotCap]    each tile's first kSlotCap escape records
+//   slots     u32[T][C]           each tile's first C = tile / 16 escape records
 struct Ws1 {
     uint64_t ovf_count, blocks_done, rcnt, seg_e, tile_cnt, ovf, slots, total;
 };
-Ws1 ws1_layout(uint64_t n_segs, uint64_t n_tiles) {
+Ws1 ws1_layout(uint64_t n_segs, uint64_t n_tiles, uint64_t slot_cap) {
     const uint64_t g = umin64(n_tiles, kMaxRanges);
     Ws1 w;
     w.ovf_count = 0;
@@ -89,7 +89,7 @@ Ws1 ws1_layout(uint64_t n_segs, uint64_t n_tiles) {
     w.tile_cnt = round_up(w.seg_e + 4 * n_segs, kAlign);
     w.ovf = round_up(w.tile_cnt + 4 * n_tiles, kAlign);
     w.slots = round_up(w.ovf + sizeof(OvfItem) * n_tiles, kAlign);
-    w.total = round_up(w.slots + 4ull * kSlotCap * n_tiles, kAlign);
+    w.total = round_up(w.slots + 4ull * slot_cap * n_tiles, kAlign);
     return w;
 }
 
@@ -120,8 +120,10 @@ Batch single_batch(uint64_t n) {
     b.segs = nullptr;
     b.n_segs = 1;
     b.page_elems = n > 0 ? n : 1;
-    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems);
-    b.n_tiles = segment_tiles(n, b.page_elems);
+    b.tile_subs = n < kSmallTileBelow ? 1u : kSubsPerTile;
+    b.tile_elems = kSub * b.tile_subs;
+    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems, b.tile_elems);
+    b.n_tiles = segment_tiles(n, b.page_elems, b.tile_elems);
     b.single.n_elems = n;
     b.single.page_begin = 0;
     b.single.out_offset = 0;
@@ -138,7 +140,9 @@ Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, ui
     b.segs = d_segs;
     b.n_segs = n_segs;
     b.page_elems = page_elems;
-    b.tiles_per_page = (uint32_t)tiles_per_page(page_elems);
+    b.tile_subs = kSubsPerTile;
+    b.tile_elems = kTile;
+    b.tiles_per_page = (uint32_t)tiles_per_page(page_elems, kTile);
     b.n_tiles = n_tiles;
     return b;
 }
@@ -161,7 +165,8 @@ WsSmall small_layout(uint64_t n) {
 }
 
 Ws single_ws(uint64_t n) {
-    Ws w = ws_layout(1, single_batch(n).n_tiles);
+    const Batch b = single_batch(n);
+    Ws w = ws_layout(1, b.n_tiles, b.tile_subs);
     if (n <= kSmallEncodeMax) w.total = umax64(w.total, small_layout(n).total);
     return w;
 }
@@ -255,8 +260,6 @@ sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, u
                              uint64_t *d_out_bytes, uint8_t *d_codebook16_or_null, int32_t *d_status,
                              const CompressScratch &w, const DeviceInfo &dev, cudaStream_t s) {
     SZ_TRY_CUDA(cudaMemsetAsync(w.zero, 0, w.zero_bytes, s));  // seg_hist, seg_done, enc_done
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
-    SZ_TRY_CUDA(cudaMemsetAsync(d_out_bytes, 0, sizeof(uint64_t), s));
     SelectCtx c{};
     c.batch = single_batch(n);
     c.seg_hist = w.seg_hist;
@@ -271,6 +274,8 @@ sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, u
     h.seg_hist = w.seg_hist;
     h.seg_done = w.seg_done;
     h.rhist = w.rhist;
+    h.reset_status = d_status;  // the histogram kernel sets no status on a single stream
+    h.reset_size = d_out_bytes;
     SZ_TRY_CUDA(launch_hist(h, false, s));
     EncodeArgs a{};  // the codebook the histogram kernel chose: no reselect
     a.batch = c.batch;
@@ -365,8 +370,10 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     const Ws w = single_ws(n);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
-    if (n <= kSmallDecodeMax) return cuda_status(launch_small_decode(d_in, in_bytes, d_out, n, d_status, s));
+    if (n <= kSmallDecodeMax) {
+        SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, sizeof(int32_t), s));
+        return cuda_status(launch_small_decode(d_in, in_bytes, d_out, n, d_status, s));
+    }
     DeviceInfo dev;
     if (const sz_status st = device_info(dev)) return st;
     DecodeArgs a{};
@@ -435,7 +442,7 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
         h_segs[k].out_offset = out;
         h_segs[k].tile_begin = tiles;
         pages += div_up(n, page_elems);
-        tiles += segment_tiles(n, page_elems);
+        tiles += segment_tiles(n, page_elems, kTile);
         out += round_up(SZ_MAX_BYTES(n), kAlign);
     }
     if (multi_page && page_elems % 64 != 0) return SZ_ERR_ALIGN;
@@ -443,7 +450,7 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
     *total_pages = pages;
     *n_tiles = tiles;
     *out_bytes = out;
-    *workspace_bytes = ws_layout(n_segs, tiles).total;
+    *workspace_bytes = ws_layout(n_segs, tiles, kSubsPerTile).total;
     return SZ_OK;
 }
 
@@ -455,7 +462,7 @@ sz_status sz_histogram_codebook_batched(uint32_t n_segs, const sz_segment *d_seg
     if (!d_segs || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const Ws w = ws_layout(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles, kSubsPerTile);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (const sz_status st = device_info(dev)) return st;
@@ -478,7 +485,7 @@ sz_status sz_encode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     if (!d_segs || !d_out || !d_out_bytes || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const Ws w = ws_layout(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles, kSubsPerTile);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (const sz_status st = device_info(dev)) return st;
@@ -509,13 +516,12 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     if (!d_segs || !d_in || !d_status || !d_ws || (n_tiles > 0 && !d_pages)) return SZ_ERR_NULL;
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (!aligned16(d_in) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const Ws w = ws_layout(n_segs, n_tiles);
+    const Ws w = ws_layout(n_segs, n_tiles, kSubsPerTile);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     DeviceInfo dev;
     if (const sz_status st = device_info(dev)) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    SZ_TRY_CUDA(cudaMemsetAsync(d_status, 0, 4 * (uint64_t)n_segs, s));
-    DecodeArgs a{};
+    DecodeArgs a{};  // the index kernel writes every segment's status
     a.batch = make_batch(n_segs, d_segs, n_tiles, page_elems);
     a.pages = d_pages;
     a.in = d_in;
@@ -532,7 +538,8 @@ sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uin
     if (!max_compressed_bytes || !workspace_bytes) return SZ_ERR_NULL;
     if (n_elems > kMaxElems) return SZ_ERR_TOO_LARGE;
     *max_compressed_bytes = container_size(n_elems, n_elems);
-    *workspace_bytes = ws1_layout(1, single_batch(n_elems).n_tiles).total;
+    const Batch b = single_batch(n_elems);
+    *workspace_bytes = ws1_layout(1, b.n_tiles, slot_cap(b)).total;
     return SZ_OK;
 }
 
@@ -544,7 +551,7 @@ sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
     if (out_cap < container_size(n, 0)) return SZ_ERR_CAPACITY;
     const Batch b = single_batch(n);
-    const Ws1 w = ws1_layout(1, b.n_tiles);
+    const Ws1 w = ws1_layout(1, b.n_tiles, slot_cap(b));
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     return one_pass(b, nullptr, d_in, d_codebook16, d_out, out_cap, d_out_bytes, d_status, d_ws, w,
                     static_cast<cudaStream_t>(stream));
@@ -553,7 +560,7 @@ sz_status sz_encode_one_pass(const uint16_t *d_in, uint64_t n, const uint8_t *d_
 sz_status sz_workspace_one_pass_batched(uint32_t n_segs, uint64_t n_tiles, uint64_t *workspace_bytes) {
     if (!workspace_bytes) return SZ_ERR_NULL;
     if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
-    *workspace_bytes = ws1_layout(n_segs, n_tiles).total;
+    *workspace_bytes = ws1_layout(n_segs, n_tiles, kTile / kSlotDiv).total;
     return SZ_OK;
 }
 
@@ -568,7 +575,7 @@ sz_status sz_encode_one_pass_batched(uint32_t n_segs, const sz_segment *d_segs, 
     if (page_elems == 0) return SZ_ERR_INVALID;
     if (n_tiles > 0xFFFFFFFFull) return SZ_ERR_TOO_LARGE;
     if (!aligned16(d_out) || !aligned16(d_ws)) return SZ_ERR_ALIGN;
-    const Ws1 w = ws1_layout(n_segs, n_tiles);
+    const Ws1 w = ws1_layout(n_segs, n_tiles, kTile / kSlotDiv);
     if (ws_bytes < w.total) return SZ_ERR_WORKSPACE;
     return one_pass(make_batch(n_segs, d_segs, n_tiles, page_elems), d_pages, nullptr, d_codebooks, d_out, out_cap,
                     d_out_bytes, d_status, d_ws, w, static_cast<cudaStream_t>(stream));
@@ -638,7 +645,7 @@ sz_status sz_debug_set_flags(uint32_t flags) {
     return SZ_OK;
 }
 
-uint64_t sz_tile_elems(void) { return kTile; }
+uint64_t sz_tile_elems(void) { return kTile; }  // batched calls and single streams of 2^27 elements or more
 
 const char *sz_version(void) { return "splitzip-b200 1.1 sm_100a"; }
 

@@ -66,59 +66,83 @@ __device__ inline Header read_header(const uint8_t *c, uint64_t cap, uint64_t n)
 }
 
 // ------------------------------------------------- per-sub-tile escape index
-// Entry j of segment k (j = S*tile + sub, S = kSubsPerTile, j = 0..S*tiles_k)
-// = index of the first escape whose position is >= the first element of that
-// sub-tile (sub-tiles past a short tile's end start at the tile's end); entry
-// S*tiles_k = e.  Entries of segment k start at S*tile_begin_k + k.
+// Entry j of segment k (j = S*tile + sub, S = sub-tiles per tile, j =
+// 0..S*tiles_k) = index of the first escape whose position is >= the first
+// element of that sub-tile (sub-tiles past a short tile's end start at the
+// tile's end); entry S*tiles_k = e.  Entries of segment k start at
+// S*tile_begin_k + k.  One warp per entry: a 32-way search over the
+// ascending position stream (each round probes 32 evenly spaced records and
+// keeps the interval where the positions reach the target, so about log32 e
+// dependent loads).  On a corrupt stream the search still ends, on some
+// index; the decode's per-sub-tile checks reject the records.  The entry of
+// the segment's sentinel also writes the segment's status (SZ_OK, or the
+// header's error): the decode kernel after it only ever sets errors.
+__device__ inline uint64_t warp_first_at_least(const uint8_t *pos, uint64_t e, uint64_t target, uint32_t lane) {
+    uint64_t lo = 0, hi = e;  // the answer is in [lo, hi]
+    while (lo < hi) {
+        const uint64_t step = (hi - lo + 31) / 32;
+        const uint64_t p = lo + (uint64_t)(lane + 1) * step - 1;
+        bool ge = true;  // probes past the interval count as reaching the target
+        if (p < hi) ge = load_u32_any(pos + 4 * p) >= target;
+        const uint32_t b = __ballot_sync(0xFFFFFFFFu, ge);
+        if (b == 0) return hi;  // every probe is below: the answer is hi
+        const uint64_t f = (uint64_t)(__ffs(b) - 1);
+        const uint64_t nhi = umin64(hi, lo + (f + 1) * step - 1);
+        lo = f == 0 ? lo : lo + f * step;
+        hi = nhi;
+    }
+    return lo;
+}
+
 template <bool kBatched>
 __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint64_t n_entries) {
     __shared__ uint64_t s_entry_begin[kMaxSmemSegs + 1];
+    allow_dependents();      // the decode kernel may start its prologue
+    grid_dependency_wait();  // the kernel that wrote the containers has finished
+    const uint32_t S = a.batch.tile_subs;
     const uint32_t ns = kBatched ? a.batch.n_segs : 1u;
     const bool cached = kBatched && ns <= kMaxSmemSegs;
     if (cached) {
         for (uint32_t i = threadIdx.x; i < ns; i += blockDim.x)
-            s_entry_begin[i] = kSubsPerTile * a.batch.segs[i].tile_begin + i;
+            s_entry_begin[i] = S * a.batch.segs[i].tile_begin + i;
     }
     __syncthreads();
-    const uint64_t j_glob = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint32_t lane = threadIdx.x & 31;
+    const uint64_t j_glob = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // one warp per entry
     if (j_glob >= n_entries) return;
     uint32_t k = 0;
-    if (kBatched) {  // largest k with 4*tile_begin_k + k <= j_glob
+    if (kBatched) {  // largest k with S*tile_begin_k + k <= j_glob
         uint32_t lo = 0, hi = ns;
         while (hi - lo > 1) {
             const uint32_t mid = (lo + hi) >> 1;
-            const uint64_t b = cached ? s_entry_begin[mid] : kSubsPerTile * a.batch.segs[mid].tile_begin + mid;
+            const uint64_t b = cached ? s_entry_begin[mid] : S * a.batch.segs[mid].tile_begin + mid;
             if (b <= j_glob) lo = mid; else hi = mid;
         }
         k = lo;
     }
     const sz_segment seg = load_segment(a.batch, k);
-    const uint64_t j = j_glob - (kSubsPerTile * seg.tile_begin + k);
-    const uint64_t tiles = segment_tiles(seg.n_elems, a.batch.page_elems);
-    uint32_t *ts = a.sub_start + kSubsPerTile * seg.tile_begin + k;
-    if (j > kSubsPerTile * tiles) return;
+    const uint64_t j = j_glob - (S * seg.tile_begin + k);
+    const uint64_t tiles = seg_tiles(a.batch, seg.n_elems);
+    uint32_t *ts = a.sub_start + S * seg.tile_begin + k;
+    if (j > S * tiles) return;
     const uint64_t cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
     const uint8_t *c = a.in + seg.out_offset;
     const Header h = read_header(c, cap, seg.n_elems);
-    if (j == kSubsPerTile * tiles) {  // the sentinel thread reports the header of its segment
-        if (!h.ok) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
-        ts[j] = h.ok ? (uint32_t)h.e : 0u;
+    if (j == S * tiles) {  // the sentinel entry: the segment's status and its escape count
+        if (lane == 0) {
+            a.status[k] = h.ok ? SZ_OK : (h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
+            ts[j] = h.ok ? (uint32_t)h.e : 0u;
+        }
         return;
     }
-    if (!h.ok) {
-        ts[j] = 0;
-        return;
+    uint64_t idx = 0;
+    if (h.ok) {
+        const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / S);
+        const uint64_t first = r.elem0 + umin32((uint32_t)(j % S) * kSub, r.len);
+        const uint64_t n = h.n;
+        idx = warp_first_at_least(c + kHeader + n + (n + 1) / 2, h.e, first, lane);
     }
-    const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / kSubsPerTile);
-    const uint64_t first = r.elem0 + umin32((uint32_t)(j % kSubsPerTile) * kSub, r.len);
-    const uint64_t n = h.n, e = h.e;
-    const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
-    uint64_t lo = 0, hi = e;  // first index with pos >= first
-    while (lo < hi) {
-        const uint64_t mid = (lo + hi) >> 1;
-        if (load_u32_any(pos + 4 * mid) < first) lo = mid + 1; else hi = mid;
-    }
-    ts[j] = (uint32_t)lo;
+    if (lane == 0) ts[j] = (uint32_t)idx;
 }
 
 // -------------------------------------------------------------- decode
@@ -189,6 +213,7 @@ constexpr uint32_t kEscCap = 1024;  // escape records bulk-copied per sub-tile; 
 
 constexpr uint32_t kDFlagEnd = 1u;
 constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
+constexpr uint32_t kDFlagTileEnd = 4u;  // last sub-tile of its tile
 constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage
 
 struct DecMeta {
@@ -197,6 +222,7 @@ struct DecMeta {
     uint64_t elem0;     // first element of the sub-tile in the segment stream
     uint64_t n, e;
     uint64_t cb_lo, cb_hi;
+    uint64_t tile;      // global tile of the sub-tile
     uint32_t seg, len, flags, lo, cnt;
     uint32_t pos_skew;  // byte offset of record lo's position inside the staged copy
     uint32_t raw_skew;  // byte offset of record lo's exponent inside the staged copy
@@ -225,6 +251,24 @@ __host__ __device__ inline uint64_t tiles_per_group(const Batch &b) {
     return g > 0 ? g : 1;
 }
 
+// The tile a CTA of `grid` decodes after tile t.
+__device__ __forceinline__ uint64_t next_dealt_tile(uint64_t t, uint64_t group, uint32_t grid) {
+    return (t + 1) % group == 0 ? t + 1 + (uint64_t)(grid - 1) * group : t + 1;
+}
+
+// A stage wait of this CTA ran out.  Its tiles before `from` (in the order
+// it decodes them) are complete; every segment with a tile at or after
+// `from` gets SZ_ERR_DEVICE_TIMEOUT.
+__device__ void decode_timeout_from(const DecodeArgs &a, const SegCache &c, uint64_t from) {
+    const uint64_t group = tiles_per_group(a.batch);
+    uint32_t last = 0xFFFFFFFFu;
+    for (uint64_t t = from; t < a.batch.n_tiles; t = next_dealt_tile(t, group, gridDim.x)) {
+        const uint32_t k = find_segment(c, a.batch, t);
+        if (k != last) set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
+        last = k;
+    }
+}
+
 // ------------------------------------------------------------ producer
 // One thread: per sub-tile, wait for the stage to be free, then bulk-copy
 // the sm bytes, the codes and (when they fit and stay inside the buffer) a
@@ -240,8 +284,7 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     uint64_t cap = 0;
     bool tma_ok = false;
     const uint64_t group = tiles_per_group(a.batch);
-    for (uint64_t t = (uint64_t)blockIdx.x * group; t < a.batch.n_tiles;
-         t = (t + 1) % group == 0 ? t + 1 + (uint64_t)(gridDim.x - 1) * group : t + 1) {
+    for (uint64_t t = (uint64_t)blockIdx.x * group; t < a.batch.n_tiles; t = next_dealt_tile(t, group, gridDim.x)) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
             cur = k;
@@ -260,10 +303,11 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
         // the tile's five sub-tile starts; the last sub-tile of a tile ends
         // where the next tile starts (the segment's last: at e), so the
         // ranges cover every escape record
-        const uint32_t *ts = a.sub_start + kSubsPerTile * (seg.tile_begin + r.local) + k;
+        const uint32_t S = a.batch.tile_subs;
+        const uint32_t *ts = a.sub_start + S * (seg.tile_begin + r.local) + k;
         uint32_t tsv[kSubsPerTile + 1];
 #pragma unroll
-        for (uint32_t q = 0; q <= kSubsPerTile; ++q) tsv[q] = ts[q];
+        for (uint32_t q = 0; q <= kSubsPerTile; ++q) tsv[q] = q <= S ? ts[q] : 0u;
         const uint64_t pos_off = kHeader + h.n + (h.n + 1) / 2;
         const uint64_t raw_off = pos_off + 4 * h.e;
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
@@ -274,7 +318,10 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
             }
             const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
             const uint32_t len = umin32(kSub, r.len - sub * kSub);
-            uint32_t lo = tsv[0], hi = tsv[kSubsPerTile];
+            uint32_t lo = tsv[0], hi = tsv[0];
+#pragma unroll
+            for (uint32_t q = 0; q <= kSubsPerTile; ++q)
+                if (q == S) hi = tsv[q];
 #pragma unroll
             for (uint32_t q = 0; q < kSubsPerTile; ++q) {
                 if (q == sub) {
@@ -299,8 +346,9 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
             m.len = len;
             m.lo = lo;
             m.cnt = cnt;
+            m.tile = t;
             const bool tma = tma_ok && len == kSub;
-            uint32_t bytes = 0, f = 0;
+            uint32_t bytes = 0, f = sub + 1 == r.n_subs ? kDFlagTileEnd : 0u;
             // escape records: aligned supersets [ps & ~15, ceil16(pe)) that
             // must lie inside the caller's buffer
             uint64_t p0 = 0, p1 = 0, r0 = 0, r1 = 0;
@@ -394,15 +442,15 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
     uint32_t cur = 0xFFFFFFFFu;
     DecTables T{};
     uint32_t cbset[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    // thread 0: this CTA's first tile not yet decoded completely (every
+    // consumer has passed the barrier below when it is read)
+    uint64_t next_tile = (uint64_t)blockIdx.x * tiles_per_group(a.batch);
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kDecStages);
         if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
         consumer_sync();
         if (!sh.go) {  // the same decision in every consumer thread
-            if (tid == 0 && a.batch.n_tiles > 0) {
-                const uint64_t t0 = umin64((uint64_t)blockIdx.x * tiles_per_group(a.batch), a.batch.n_tiles - 1);
-                set_status(a.status + find_segment(sh.segc, a.batch, t0), SZ_ERR_DEVICE_TIMEOUT);
-            }
+            if (tid == 0) decode_timeout_from(a, sh.segc, next_tile);
             return;
         }
         const DecMeta m = sh.meta[s];
@@ -459,6 +507,8 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
                 if (bad) set_status(status, SZ_ERR_CORRUPT);
             }
         }
+        if (tid == 0 && (m.flags & kDFlagTileEnd))
+            next_tile = next_dealt_tile(m.tile, tiles_per_group(a.batch), gridDim.x);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.empty[s]);
     }
@@ -476,6 +526,7 @@ __global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArg
         }
         fence_mbar_init();
     }
+    grid_dependency_wait();  // the index kernel before it has finished
     seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
     if (tid >= kThreads) {
         if (tid == kThreads) decode_producer<kBatched>(a, sh);
@@ -585,14 +636,13 @@ cudaError_t launch_small_decode(const uint8_t *c, uint64_t cap, uint16_t *out, u
     return cudaGetLastError();
 }
 
+// Also writes every segment's status word (no memset before it).
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {
-    const uint64_t entries = kSubsPerTile * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
-    const uint64_t grid = div_up(entries, 256);
-    if (batched)
-        esc_index_kernel<true><<<(unsigned)grid, 256, 0, s>>>(a, entries);
-    else
-        esc_index_kernel<false><<<(unsigned)grid, 256, 0, s>>>(a, entries);
-    return cudaGetLastError();
+    const uint64_t entries = (uint64_t)a.batch.tile_subs * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
+    const uint64_t grid = div_up(entries, 256 / 32);  // one warp per entry
+    const cudaError_t e = batched ? launch_after(esc_index_kernel<true>, dim3((unsigned)grid), dim3(256), 0, s, a, entries)
+                                  : launch_after(esc_index_kernel<false>, dim3((unsigned)grid), dim3(256), 0, s, a, entries);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStream_t s) {
@@ -605,13 +655,13 @@ cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStre
     if (batched) {
         e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_kernel<true><<<grid, kPipeThreads, smem, s>>>(a);
+        e = launch_after(decode_kernel<true>, dim3(grid), dim3(kPipeThreads), smem, s, a);
     } else {
         e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        decode_kernel<false><<<grid, kPipeThreads, smem, s>>>(a);
+        e = launch_after(decode_kernel<false>, dim3(grid), dim3(kPipeThreads), smem, s, a);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 int decode_blocks_per_sm() {

@@ -178,7 +178,7 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             if (!valid) set_status(a.status + k, SZ_ERR_INVALID);
             else if (!fits) set_status(a.status + k, SZ_ERR_CAPACITY);
             else if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
-            seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
+            seg_end = seg.tile_begin + seg_tiles(a.batch, seg.n_elems);
             p_first = t;
             p_last = umin64(seg_end, t_end) - 1;
             if (t == t_begin) {  // opens the range
@@ -199,6 +199,16 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
         if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
             const int s = (int)(j % kEncStages);
+            // the next sub-tile into L2 ahead of its bulk copy: in this tile,
+            // or -- a single stream, where tiles follow in memory -- the next
+            // tile's first
+            {
+                uint64_t rest = 0;
+                if (sub + 1 < r.n_subs) rest = r.len - (sub + 1) * kSub;
+                else if (!kBatched && t + 1 < t_end) rest = r.n - (r.elem0 + r.len);
+                const uint32_t next = aligned ? ((uint32_t)umin64(kSub, rest) * 2u) & ~15u : 0u;
+                if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src + (sub + 1) * kSub), "r"(next) : "memory");
+            }
             if (j >= (uint32_t)kEncStages && !mbar_wait(&sh.empty[s], ((j / kEncStages) - 1) & 1u, a.wait_limit_ns)) {
                 set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
                 return;
@@ -262,13 +272,13 @@ struct PendingEsc {
 
 // Every consumer thread takes records tid, tid + 256, ...: consecutive
 // threads write consecutive positions and exponents (one-pass: consecutive
-// slot entries, the first kSlotCap records of the tile).
+// slot entries, the first slot_cap records of the tile; lim = slot_cap).
 template <bool kOnePass>
 __device__ __forceinline__ void copy_out_escapes(const uint32_t *stg, const PendingEsc &p, int tid) {
     if constexpr (kOnePass) {
         for (uint32_t i = tid; i < p.cnt; i += kThreads) {
             const uint64_t g = p.first + i;
-            if (g >= kSlotCap) break;
+            if (g >= p.lim) break;
             const uint32_t rec = stg[i];
             p.slot[g] = (rec & 0xFF0000u) | (p.tile_off + (rec & 0xFFFFu));
         }
@@ -334,7 +344,7 @@ __device__ void timeout_from(const EncodeArgs &a, const SegCache &c, uint64_t fr
         const uint32_t k = find_segment(c, a.batch, t);  // the segment that holds tile t
         set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
         const sz_segment sk = load_segment(a.batch, k);
-        t = sk.tile_begin + segment_tiles(sk.n_elems, a.batch.page_elems);
+        t = sk.tile_begin + seg_tiles(a.batch, sk.n_elems);
     }
 }
 
@@ -481,8 +491,9 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             // the records this sub-tile may write: [first, last) of the segment
             // (one-pass: of the tile's slot)
             const uint64_t first = kOnePass ? (uint64_t)running : (uint64_t)m.esc_base + running;
-            const uint64_t lim = kOnePass ? (uint64_t)kSlotCap : umin64(e_total, (uint64_t)m.esc_base + m.esc_count);
-            uint32_t *slot = kOnePass ? a.slots + (size_t)m.esc_base * kSlotCap : nullptr;
+            const uint32_t cap = slot_cap(a.batch);
+            const uint64_t lim = kOnePass ? (uint64_t)cap : umin64(e_total, (uint64_t)m.esc_base + m.esc_count);
+            uint32_t *slot = kOnePass ? a.slots + (size_t)m.esc_base * cap : nullptr;
             const uint32_t tile_off = m.sub_in_tile * kSub;
             const bool staged = sub_total <= kEscStage;
             uint32_t *stg = sh.esc[j & 1];
@@ -589,6 +600,7 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
     extern __shared__ __align__(128) uint8_t smem_raw[];
     EncShared &sh = *reinterpret_cast<EncShared *>(smem_raw);
     const int tid = threadIdx.x;
+    allow_dependents();  // the escape placement (one-pass) may start its prologue
     if (tid == 0) {
         for (int s = 0; s < kEncStages; ++s) {
             mbar_init(&sh.full[s], 1);
@@ -596,6 +608,7 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
         }
         fence_mbar_init();
     }
+    grid_dependency_wait();  // the histogram kernel before it has finished
     seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
 
     // Segments with no elements have no tiles: CTA 0 writes their header
@@ -649,7 +662,7 @@ __global__ void __launch_bounds__(kThreads) small_hist_kernel(const uint16_t *in
                                                               uint8_t *codebook_out, int32_t *status,
                                                               uint64_t *out_bytes) {
     extern __shared__ __align__(16) uint32_t s_col[];  // kTinyColWords
-    __shared__ uint32_t s_cnt[256];
+    __shared__ RankShared s_rank;
     __shared__ uint32_t s_warp[kWarps];
     __shared__ uint32_t s_carry;
     __shared__ uint8_t s_cb[16];
@@ -698,14 +711,7 @@ __global__ void __launch_bounds__(kThreads) small_hist_kernel(const uint16_t *in
     // ---- the last block: select, escape count, first escape index per slice
     __threadfence();
     c = __ldcg(w.seg_hist + tid);
-    s_cnt[tid] = c;
-    __syncthreads();
-    uint32_t rank = 0;
-#pragma unroll 8
-    for (uint32_t u = 0; u < 256; ++u) {
-        const uint32_t cu = s_cnt[u];
-        rank += (cu > c) || (cu == c && u < tid);
-    }
+    const uint32_t rank = exponent_rank(c, tid, s_rank);
     if (rank < 16) {
         s_cb[rank] = (uint8_t)tid;
         atomicAdd(&s_top, (unsigned long long)c);
@@ -878,11 +884,11 @@ template <bool kBatched, bool kOnePass>
 cudaError_t launch_encode_t(const EncodeArgs &a, cudaStream_t s) {
     const size_t smem = sizeof(EncShared);
     const int grid = (int)umax64(1, div_up(a.batch.n_tiles, a.range_tiles));
-    const cudaError_t e =
+    cudaError_t e =
         cudaFuncSetAttribute(encode_kernel<kBatched, kOnePass>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    encode_kernel<kBatched, kOnePass><<<grid, kPipeThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    e = launch_after(encode_kernel<kBatched, kOnePass>, dim3(grid), dim3(kPipeThreads), smem, s, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_encode(const EncodeArgs &a, bool batched, cudaStream_t s) {

@@ -47,6 +47,7 @@ __device__ __forceinline__ void count_v4(uint4 v, uint32_t col) {
 // ---------------------------------------------------------- top-16 select
 // Shared state of one segment's select (256 threads).
 struct SelShared {
+    RankShared rank;
     uint32_t cnt[256];
     uint32_t warp[kWarps];
     unsigned long long top;
@@ -55,19 +56,6 @@ struct SelShared {
     int flag;
     uint8_t cb[16];
 };
-
-// Rank of exponent `tid` (count c) among the 256 counts in cnt[] in the
-// order (count descending, exponent ascending): the number of exponents
-// before it.  Ranks 0..15 are the codebook.
-__device__ __forceinline__ uint32_t exponent_rank(const uint32_t *cnt, uint32_t c, uint32_t tid) {
-    uint32_t rank = 0;
-#pragma unroll 8
-    for (uint32_t u = 0; u < 256; ++u) {
-        const uint32_t cu = cnt[u];
-        rank += (cu > c) || (cu == c && u < tid);
-    }
-    return rank;
-}
 
 // Codebook, escape count and range records of segment k, by the kThreads
 // threads of one block (every one of them must call it).  Thread t holds
@@ -89,7 +77,7 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
     ss.cnt[tid] = c;
     __syncthreads();
     if (codebook_in == nullptr) {
-        const uint32_t rank = exponent_rank(ss.cnt, c, tid);
+        const uint32_t rank = exponent_rank(c, tid, ss.rank);
         if (rank < 16) ss.cb[rank] = (uint8_t)tid;
     } else if (tid < 16) {
         ss.cb[tid] = codebook_in[tid];
@@ -130,7 +118,7 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
     // ---- the segment's pieces: one per range it reaches
     const uint64_t R = a.range_tiles;
     const uint64_t t_first = seg.tile_begin;
-    const uint64_t t_last = t_first + segment_tiles(n, a.batch.page_elems) - 1;
+    const uint64_t t_last = t_first + seg_tiles(a.batch, n) - 1;
     const uint64_t b_first = t_first / R, b_last = t_last / R;
     if (b_first == b_last) {  // inside one range: only a range-opening segment has a record
         if (tid == 0 && t_first == b_first * R) {
@@ -220,9 +208,10 @@ __device__ void empty_segments(const HistArgs &h) {
 // counts, and kept when the piece opens or closes the range.  The block
 // that completes a segment's tile count runs that segment's select.
 // kSmallTiles: every tile is a single sub-tile (pages of at most 16,384
-// elements); that build is given registers for 3 blocks per SM -- measured
-// 0.70 -> 0.86 of the copy bandwidth on 16-token pages, while the same
-// bound costs 8 % on 65,536-element tiles, which keep the default build.
+// elements, or the one-sub-tile tiles of a short single stream); that
+// build is given registers for 3 blocks per SM -- measured 0.70 -> 0.86 of
+// the copy bandwidth on 16-token pages, while the same bound costs 8 % on
+// 65,536-element tiles, which keep the default build.
 // kAccum: the accumulate mode -- each piece's counts are added to the
 // caller's histogram of its segment (a.accum, row a.accum_index[k] or k);
 // no range records, no completion count, no select.
@@ -234,6 +223,11 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
     static_assert(kThreads == 256, "one thread per bin");
     const Batch &batch = a.sel.batch;
 
+    allow_dependents();  // the encode kernel may start its prologue
+    if (blockIdx.x == 0 && threadIdx.x == 0) {  // words only the next kernel reads
+        if (a.reset_status) *a.reset_status = SZ_OK;
+        if (a.reset_size) *a.reset_size = 0;
+    }
     for (uint32_t i = threadIdx.x; i < kHistWords; i += kThreads) s_hist[i] = 0;
     seg_cache_fill(s_segc, batch);  // ends with __syncthreads
     if (!kAccum && blockIdx.x == 0) empty_segments(a);
@@ -249,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
     while (t < t_end) {
         const uint32_t k = find_segment(s_segc, batch, t);
         const sz_segment seg = load_segment(batch, k);
-        const uint64_t seg_tiles = segment_tiles(seg.n_elems, batch.page_elems);
-        const uint64_t ps = t, pe = umin64(seg.tile_begin + seg_tiles, t_end);  // the piece [ps, pe)
+        const uint64_t n_seg_tiles = seg_tiles(batch, seg.n_elems);
+        const uint64_t ps = t, pe = umin64(seg.tile_begin + n_seg_tiles, t_end);  // the piece [ps, pe)
         for (; t < pe; ++t) {
             const TileRef r = resolve_tile(batch, seg, k, t);
             const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
@@ -259,9 +253,14 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
             for (uint32_t sub = 0; ok && sub < r.n_subs; ++sub) {
                 const uint16_t *p = src + sub * kSub;
                 const uint32_t len = umin32(kSub, r.len - sub * kSub);
-                // bulk prefetch of the next sub-tile into L2 while this one is counted
-                if (tid == 0 && sub + 1 < r.n_subs) {
-                    const uint32_t next = (umin32(kSub, r.len - (sub + 1) * kSub) * 2u) & ~15u;
+                // bulk prefetch of the next sub-tile into L2 while this one is
+                // counted: inside the tile, or -- a single stream of one-sub-tile
+                // tiles, where the next tile follows in memory -- the next tile's
+                if (tid == 0) {
+                    uint64_t rest = 0;
+                    if (sub + 1 < r.n_subs) rest = r.len - (sub + 1) * kSub;
+                    else if (!kBatched && batch.tile_subs == 1 && t + 1 < t_end) rest = r.n - (r.elem0 + r.len);
+                    const uint32_t next = ((uint32_t)umin64(kSub, rest) * 2u) & ~15u;
                     if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p + kSub), "r"(next) : "memory");
                 }
                 if (len == kSub) {
@@ -308,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
         __syncthreads();  // folds done before the next piece's counts land
         if (tid == 0) {
             const uint32_t add = (uint32_t)(pe - ps);
-            s_sel.flag = atomicAdd(&a.seg_done[k], add) + add == (uint32_t)seg_tiles;
+            s_sel.flag = atomicAdd(&a.seg_done[k], add) + add == (uint32_t)n_seg_tiles;
         }
         __syncthreads();
         if (s_sel.flag) {  // every other piece of segment k is counted and published
@@ -342,13 +341,11 @@ __global__ void __launch_bounds__(kThreads) reselect_kernel(const ReselectArgs a
 // count = the histogram's total - the codebook's counts.
 __global__ void __launch_bounds__(kThreads) select_kernel(const uint32_t *hists, uint8_t *codebooks,
                                                           uint64_t *escapes) {
-    __shared__ uint32_t s_cnt[256];
+    __shared__ RankShared s_rank;
     __shared__ unsigned long long s_sum[2][kWarps];  // [0]: all counts, [1]: codebook counts
     const uint32_t tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const uint32_t c = hists[(size_t)blockIdx.x * 256 + tid];
-    s_cnt[tid] = c;
-    __syncthreads();
-    const uint32_t rank = exponent_rank(s_cnt, c, tid);
+    const uint32_t rank = exponent_rank(c, tid, s_rank);
     if (rank < 16) codebooks[(size_t)blockIdx.x * 16 + rank] = (uint8_t)tid;
     if (escapes == nullptr) return;
     unsigned long long all = c, top = rank < 16 ? c : 0u;
@@ -375,7 +372,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const uint32_t *hists,
 // ------------------------------------------------------------ launchers
 template <bool kAccum>
 void launch_hist_t(const HistArgs &a, bool batched, int grid, size_t smem, cudaStream_t s) {
-    const bool small = a.sel.batch.page_elems <= kSub;
+    const bool small = a.sel.batch.page_elems <= kSub || a.sel.batch.tile_elems <= kSub;
     if (batched && small)
         hist_kernel<true, true, kAccum><<<grid, kThreads, smem, s>>>(a);
     else if (batched)

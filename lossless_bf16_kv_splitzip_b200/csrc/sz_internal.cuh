@@ -19,7 +19,9 @@ namespace sz {
 // each.  Chunk c of thread t covers sub-tile elements [(c*256 + t)*16, +16),
 // so a warp-wide 16-byte access is 512 contiguous bytes.
 // Tile: 4 sub-tiles (65,536 elements) inside one page; the unit of work
-// scheduling.
+// scheduling.  Single-stream calls on streams shorter than
+// kSmallTileBelow elements use tiles of one sub-tile (16,384 elements)
+// instead, so that a mid-size stream still spreads over every CTA slot.
 // Range: a run of consecutive tiles of the batch, one CTA's share in both
 // the histogram and the encode kernel (the two use the same partition).  A
 // range cut by segment boundaries holds several pieces; the histogram kernel
@@ -31,13 +33,14 @@ constexpr int kPipeThreads = kThreads + 32;   // + one producer warp
 constexpr int kChunk = 16;
 constexpr int kChunks = 4;
 constexpr uint32_t kSub = kThreads * kChunk * kChunks;  // 16,384 elements
-constexpr uint32_t kSubsPerTile = 4;
-constexpr uint32_t kTile = kSub * kSubsPerTile;         // 65,536 elements
+constexpr uint32_t kSubsPerTile = 4;                    // the most sub-tiles in a tile
+constexpr uint32_t kTile = kSub * kSubsPerTile;         // 65,536 elements: batched calls, long streams
+constexpr uint64_t kSmallTileBelow = 1ull << 27;        // single streams shorter than this: kSub tiles
 constexpr uint64_t kHeader = 48;
 constexpr uint32_t kMaxSmemSegs = 256;  // segment starts cached in shared memory
 constexpr uint64_t kMaxRanges = 1024;   // ranges of one call (workspace bound)
 constexpr uint64_t kRangesPerSM = 3;    // encode CTAs resident per SM
-constexpr uint32_t kSlotCap = 4096;     // one-pass encode: escape records staged per tile (6.25 %)
+constexpr uint32_t kSlotDiv = 16;       // one-pass encode: escape records staged per tile = tile / 16 (6.25 %)
 
 // Per-segment record kept in the workspace between kernels (32 bytes).
 struct SegMeta {
@@ -88,12 +91,14 @@ __host__ __device__ inline uint64_t umax64(uint64_t a, uint64_t b) { return a > 
 __host__ __device__ inline uint32_t umin32(uint32_t a, uint32_t b) { return a < b ? a : b; }
 
 // Tiles of a segment of n elements in pages of page_elems: every page is cut
-// into tiles of kTile elements (its last tile may be short).
-__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems) { return div_up(page_elems, kTile); }
-__host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems) {
+// into tiles of tile_elems elements (its last tile may be short).
+__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems, uint64_t tile_elems) {
+    return div_up(page_elems, tile_elems);
+}
+__host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems, uint64_t tile_elems) {
     if (n == 0) return 0;
     const uint64_t full = n / page_elems, rem = n % page_elems;
-    return full * tiles_per_page(page_elems) + div_up(rem, kTile);
+    return full * tiles_per_page(page_elems, tile_elems) + div_up(rem, tile_elems);
 }
 
 // ------------------------------------------------------------ tile lookup
@@ -103,10 +108,18 @@ struct Batch {
     const sz_segment *segs;  // nullptr for a single tensor
     uint32_t n_segs;
     uint64_t page_elems;
-    uint32_t tiles_per_page;  // ceil(page_elems / kTile), precomputed on the host
+    uint32_t tiles_per_page;  // ceil(page_elems / tile_elems), precomputed on the host
+    uint32_t tile_subs;       // sub-tiles per tile: kSubsPerTile, or 1 for short single streams
+    uint32_t tile_elems;      // kSub * tile_subs
     uint64_t n_tiles;
     sz_segment single;        // the implicit segment of a single-tensor call
 };
+
+__host__ __device__ inline uint64_t seg_tiles(const Batch &b, uint64_t n) {
+    return segment_tiles(n, b.page_elems, b.tile_elems);
+}
+// one-pass encode: escape records a tile's workspace slot holds
+__host__ __device__ inline uint32_t slot_cap(const Batch &b) { return b.tile_elems / kSlotDiv; }
 
 struct TileRef {
     uint32_t seg;
@@ -177,15 +190,16 @@ __device__ inline TileRef resolve_tile(const Batch &b, const sz_segment &s, uint
     r.local = (uint32_t)(tile - s.tile_begin);
     r.n = s.n_elems;
     const uint32_t tpp = b.tiles_per_page;
+    const uint32_t te = b.tile_elems;
     r.page = r.local / tpp;
-    r.in_page = (r.local - r.page * tpp) * kTile;
+    r.in_page = (r.local - r.page * tpp) * te;
     r.elem0 = (uint64_t)r.page * b.page_elems + r.in_page;
     const uint64_t page_len = umin64(b.page_elems, r.n - (uint64_t)r.page * b.page_elems);
-    r.len = (uint32_t)umin64(kTile, page_len - r.in_page);
+    r.len = (uint32_t)umin64(te, page_len - r.in_page);
     r.n_subs = (r.len + kSub - 1) / kSub;
     const uint64_t full = r.n / b.page_elems;
     const uint64_t rem = r.n - full * b.page_elems;
-    r.tiles = (uint32_t)(full * tpp + (rem + kTile - 1) / kTile);
+    r.tiles = (uint32_t)(full * tpp + (rem + te - 1) / te);
     return r;
 }
 
@@ -225,6 +239,45 @@ __device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligne
         p[2] = (uint8_t)(v >> 16);
         p[3] = (uint8_t)(v >> 24);
     }
+}
+
+// Rank of exponent `tid` (count c) in the order (count descending, exponent
+// ascending): the number of exponents before it; ranks 0..15 are the
+// codebook.  Every one of the 256 threads calls it (thread t = exponent t).
+// Only the exponents that occur are compared: they are compacted, in
+// ascending order, as keys count << 8 | (255 - exponent) -- one key is
+// greater than another exactly when it comes first -- and an exponent that
+// does not occur ranks after all that do, in ascending order (its rank is
+// the number of occurring exponents plus the absent ones below it).
+struct RankShared {
+    unsigned long long key[256];
+    uint32_t warp[kWarps];
+};
+__device__ inline uint32_t exponent_rank(uint32_t c, uint32_t tid, RankShared &rs) {
+    const uint32_t lane = tid & 31, wid = tid >> 5;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, c != 0);
+    if (lane == 0) rs.warp[wid] = __popc(m);
+    __syncthreads();
+    uint32_t before = 0, nnz = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t x = rs.warp[w];
+        before += (uint32_t)w < wid ? x : 0u;
+        nnz += x;
+    }
+    const uint32_t pos = before + __popc(m & ((1u << lane) - 1u));  // occurring exponents below tid
+    const unsigned long long mine = ((unsigned long long)c << 8) | (255u - tid);
+    if (c) rs.key[pos] = mine;
+    __syncthreads();
+    uint32_t rank = 0;
+    if (c == 0) {
+        rank = nnz + (tid - pos);
+    } else {
+#pragma unroll 4
+        for (uint32_t u = 0; u < nnz; ++u) rank += rs.key[u] > mine;
+    }
+    __syncthreads();  // the scratch may be reused
+    return rank;
 }
 
 // ------------------------------------------------------------ status words
@@ -270,6 +323,32 @@ __device__ __forceinline__ uint32_t load_u32_any(const uint8_t *p) {
 // the producer warp.
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with launch_after() may start while the kernel before
+// it in the stream is still running; it calls grid_dependency_wait() before
+// it reads anything that kernel wrote (the wait returns once that kernel has
+// finished and its memory operations are visible; without a prerequisite
+// kernel it returns at once).  A kernel calls allow_dependents() to let the
+// next launch_after() kernel start early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_after(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                         Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
 
 // ------------------------------------------------- mbarrier + 1-D TMA copy
@@ -340,6 +419,8 @@ struct HistArgs {
     int32_t *status;               // [n_segs] or nullptr
     uint32_t *accum;               // accumulate mode: caller histograms [rows][256] (else nullptr)
     const uint32_t *accum_index;   // accumulate mode: row of segment k (nullptr: row k)
+    int32_t *reset_status;         // optional: set to SZ_OK by block 0 (the encode's status, single stream)
+    uint64_t *reset_size;          // optional: set to 0 by block 0 (the encode's size word)
 };
 
 // Select with a caller codebook (single tensor), ahead of the encode.
@@ -368,7 +449,7 @@ struct EncodeArgs {
     // one-pass mode (caller codebooks, no histogram pass)
     const uint8_t *codebooks_in;  // [n_segs][16]
     uint32_t *tile_cnt;           // [n_tiles] escapes of each tile
-    uint32_t *slots;              // [n_tiles][kSlotCap] records: raw << 16 | offset in the tile
+    uint32_t *slots;              // [n_tiles][slot_cap] records: raw << 16 | offset in the tile
     RangeRec *rcnt;               // [ranges] first_cnt / last_cnt: escapes of the first / last piece
 };
 
@@ -402,7 +483,7 @@ struct PlaceArgs {
     uint64_t *out_bytes;          // [n_segs]
     int32_t *status;              // [n_segs]
     const uint32_t *tile_cnt;     // [n_tiles]
-    const uint32_t *slots;        // [n_tiles][kSlotCap]
+    const uint32_t *slots;        // [n_tiles][slot_cap]
     const RangeRec *rcnt;         // [ranges]
     uint64_t range_tiles;
     uint32_t *ovf_count;          // overflowed tiles listed so far (zero on entry)

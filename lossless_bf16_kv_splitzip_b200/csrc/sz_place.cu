@@ -181,6 +181,8 @@ __device__ void place_empty_segments(const PlaceArgs &a) {
 template <bool kBatched>
 __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
     __shared__ PlaceShared sh;
+    allow_dependents();      // the rescan kernel may start its prologue
+    grid_dependency_wait();  // the one-pass encode before it has finished
     seg_cache_fill(sh.segc, a.batch);  // ends with __syncthreads
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     if (blockIdx.x == 0) place_empty_segments(a);
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
     while (t < t_end) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         const sz_segment seg = load_segment(a.batch, k);
-        const uint64_t seg_end = seg.tile_begin + segment_tiles(seg.n_elems, a.batch.page_elems);
+        const uint64_t seg_end = seg.tile_begin + seg_tiles(a.batch, seg.n_elems);
         const uint64_t ps = t, pe = umin64(seg_end, t_end);  // this range's piece of segment k
         t = pe;
         // the encode refused the segment: skip it.  Thread 0 reads the word
@@ -249,10 +251,11 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
             sh.elem0[tid] = tt < pe ? resolve_tile(a.batch, seg, k, tt).elem0 : 0;
             __syncthreads();
             const uint32_t nt = (uint32_t)umin64(kThreads, pe - c0);
+            const uint32_t cap = slot_cap(a.batch);
             for (uint32_t i = wid; i < nt; i += kWarps) {
                 const uint32_t ci = sh.cnt[i];
-                if (ci > kSlotCap) continue;
-                const uint32_t *slot = a.slots + (c0 + i) * kSlotCap;
+                if (ci > cap) continue;
+                const uint32_t *slot = a.slots + (c0 + i) * cap;
                 const uint64_t bi = sh.base[i], e0 = sh.elem0[i];
                 for (uint32_t j0 = lane; j0 < ci; j0 += 128) {
                     uint32_t rec[4];
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const PlaceArgs a) {
                     }
                 }
             }
-            if (tid < nt && cnt > kSlotCap) {  // left for the rescan kernel
+            if (tid < nt && cnt > cap) {  // left for the rescan kernel
                 OvfItem it;
                 it.tile = tt;
                 it.base = sh.base[tid];
@@ -293,6 +296,7 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const PlaceArgs a) {
     __shared__ PlaceShared sh;
     __shared__ uint8_t s_esc[256];
     __shared__ int s_last;
+    grid_dependency_wait();  // the placement before it has finished
     const uint32_t count = *a.ovf_count;
     uint32_t cur = 0xFFFFFFFFu;
     for (uint32_t i = blockIdx.x; i < count; i += gridDim.x) {
@@ -325,14 +329,15 @@ __global__ void __launch_bounds__(kThreads) rescan_kernel(const PlaceArgs a) {
 cudaError_t launch_place(const PlaceArgs &a, bool batched, int sms, cudaStream_t s) {
     const int grid = (int)umax64(1, div_up(a.batch.n_tiles, a.range_tiles));
     const int rgrid = (int)umax64(1, umin64(a.batch.n_tiles, 2ull * (uint64_t)sms));
+    cudaError_t e;
     if (batched) {
-        place_kernel<true><<<grid, kThreads, 0, s>>>(a);
-        rescan_kernel<true><<<rgrid, kThreads, 0, s>>>(a);
+        e = launch_after(place_kernel<true>, dim3(grid), dim3(kThreads), 0, s, a);
+        if (e == cudaSuccess) e = launch_after(rescan_kernel<true>, dim3(rgrid), dim3(kThreads), 0, s, a);
     } else {
-        place_kernel<false><<<grid, kThreads, 0, s>>>(a);
-        rescan_kernel<false><<<rgrid, kThreads, 0, s>>>(a);
+        e = launch_after(place_kernel<false>, dim3(grid), dim3(kThreads), 0, s, a);
+        if (e == cudaSuccess) e = launch_after(rescan_kernel<false>, dim3(rgrid), dim3(kThreads), 0, s, a);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sz

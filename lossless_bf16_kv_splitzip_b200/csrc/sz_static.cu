@@ -18,15 +18,15 @@ using namespace sz;
 namespace {
 
 // Scratch layout for one tensor of at most SZ_STATIC_MAX_ELEMS elements
-// (4096 tiles, so at most kMaxRanges = 1024 ranges):
+// (at most kMaxRanges = 1024 ranges, whatever the tile size):
 //   [0, 1024)      exponent counts of the tensor, u32[256]      } cleared
 //   [1024, 1028)   tiles counted so far                         } by every
 //   [1028, 1032)   tiles of complete encode pieces              } call
 //   [1280, 1312)   SegMeta (codebook, escape count)
 //   [1536, ...)    counts of each range's first and last piece, u32[1024][2][256]
 //   then           escape placement of each range, RangeRec[1024]
-constexpr uint64_t kMaxTiles = (SZ_STATIC_MAX_ELEMS + kTile - 1) / kTile;
-constexpr uint64_t kRanges = kMaxTiles < kMaxRanges ? kMaxTiles : kMaxRanges;
+constexpr uint64_t kRanges = kMaxRanges;
+static_assert(SZ_STATIC_MAX_ELEMS / kTile >= kMaxRanges, "a stream at the limit may use every range");
 constexpr uint64_t kOffSegHist = 0;
 constexpr uint64_t kOffSegDone = 1024;
 constexpr uint64_t kOffEncDone = 1028;

@@ -43,15 +43,20 @@ def test_library_is_built_for_sm100a():
     assert "sm_100a" in sz.sz_version()
 
 
-@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 65536, 65537, 1 << 25, (1 << 32) - 2, (1 << 32) - 1])
+@pytest.mark.parametrize("n", [0, 1, 2, 17, 16384, 65536, 65537, 1 << 25, (1 << 27) - 1, 1 << 27, (1 << 32) - 2,
+                               (1 << 32) - 1])
 def test_plan_worst_case_bound(n):
     cap, ws = sz.sz_plan(n)
     assert cap == 48 + n + (n + 1) // 2 + 5 * (n - (n + 15) // 16)
-    tiles = -(-n // 65536)
+    # streams below 2^27 elements are cut into 16,384-element tiles (one
+    # sub-tile each), longer ones into 65,536-element tiles (four)
+    tile = 16384 if n < 1 << 27 else 65536
+    tiles = -(-n // tile)
     ranges = min(tiles, 1024)
-    # segment histogram, tile count and record; the first- and last-piece
-    # histograms and the record of every range; sub-tile escape starts
-    need = 1024 + 4 + 32 + 2048 * ranges + 16 * ranges + 4 * (4 * tiles + 1)
+    # segment histogram, tile count, completion count and record; the first-
+    # and last-piece histograms and the record of every range; sub-tile
+    # escape starts
+    need = 1024 + 4 + 4 + 32 + 2048 * ranges + 16 * ranges + 4 * ((tile // 16384) * tiles + 1)
     assert need <= ws
     if n <= 1 << 21:  # also the one-call compression's scratch: counts of every 4,096-element slice
         nb = max(1, -(-n // 4096))

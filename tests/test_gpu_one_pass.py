@@ -193,3 +193,32 @@ def test_batched_workload1_reuses_codebooks_bit_exactly():
     k = 2 * layers - 1
     o = int(one.out_offset[k])
     assert one.container[o: o + int(one.sizes[k])].cpu().numpy().tobytes() == oracle.encode(host[k])
+
+
+@pytest.mark.parametrize("workload,tokens", [(1, 1024), (3, 512)])
+def test_previous_layer_codebooks_equal_oracle(workload, tokens):
+    """Codebook reuse across layers, as the bench measures it: layer L's K
+    and V tensors encoded in one pass with layer L-1's K and V codebooks
+    (layer 0 with its own).  Every container is the oracle's container for
+    that codebook, and decodes back."""
+    layers = 4
+    cache = kvgen.contiguous_cache(workload, layers=layers, tokens=tokens)
+    S, n = cache.shape
+    own = np.stack([own_codebook(x) for x in cache])
+    prev = own.copy()
+    prev[2:] = own[:-2]
+    d = torch.from_numpy(cache.view(np.int16)).to(DEV)
+    ptrs = torch.tensor([d.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=DEV)
+    plan = sz.BatchPlan([n] * S, n, device=DEV)
+    plan.encode_one_pass(ptrs, torch.from_numpy(prev).to(DEV))
+    torch.cuda.synchronize()
+    assert plan.enc_status.abs().sum().item() == 0
+    sizes = plan.sizes.cpu().numpy()
+    host = plan.container.cpu().numpy()
+    for k in range(S):
+        o = int(plan.out_offset[k])
+        assert host[o: o + int(sizes[k])].tobytes() == oracle.encode(cache[k], codebook=prev[k]), k
+    out = torch.zeros_like(d)
+    plan.decode(torch.tensor([out.data_ptr() + 2 * n * k for k in range(S)], dtype=torch.int64, device=DEV))
+    torch.cuda.synchronize()
+    assert plan.dec_status.abs().sum().item() == 0 and torch.equal(out, d)

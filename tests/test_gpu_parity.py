@@ -247,10 +247,11 @@ def test_stale_workspace_histogram_is_reported():
 
 @pytest.mark.parametrize("tile", [0, 4, 8])
 def test_stale_workspace_on_several_ranges_keeps_size_zero(tile):
-    """A stream of 9 tiles is encoded by 9 CTAs, one tile each.  Its input
-    changes after the histogram in one tile only, so that tile's CTA finds
-    more escapes than the workspace counted: the status is SZ_ERR_CORRUPT
-    and the size stays 0, whichever CTA finishes the stream last."""
+    """A stream of 8 x 65,536 + 5 elements is encoded by several CTAs, each
+    a range of tiles.  Its input changes after the histogram in one 65,536-
+    element stretch only, so the CTAs there find more escapes than the
+    workspace counted: the status is SZ_ERR_CORRUPT and the size stays 0,
+    whichever CTA finishes the stream last."""
     n = 8 * 65536 + 5
     a = kvgen.mixed_small(n, seed=13)
     cap, wsb = sz.sz_plan(n)
@@ -386,9 +387,9 @@ def test_stage_wait_times_out_cleanly():
 
 
 def test_stage_wait_timeout_on_several_ranges_and_one_pass():
-    """Every stage wait runs out on a stream of 9 CTA ranges (two-pass and
-    one-pass encode) and on a batch of several segments: every status is
-    SZ_ERR_DEVICE_TIMEOUT and every size 0."""
+    """Every stage wait runs out on a stream of several CTA ranges (two-pass
+    and one-pass encode) and on a batch of several segments (encode and
+    decode): every status is SZ_ERR_DEVICE_TIMEOUT and every size 0."""
     n = 8 * 65536 + 5
     x = kvgen.mixed_small(n, seed=33)
     lens = [3 * 65536 + 7, 16384, 5 * 65536]
@@ -420,6 +421,21 @@ def test_stage_wait_timeout_on_several_ranges_and_one_pass():
     plan.encode(ptrs)
     torch.cuda.synchronize()
     assert plan.enc_status.abs().sum().item() == 0
+    dst = torch.zeros_like(pool)
+    dptrs = torch.from_numpy((np.array(starts) * 2 + dst.data_ptr()).astype(np.int64)).to(DEV)
+    try:
+        sz.sz_set_wait_limit_ns(2_000_000)
+        sz.sz_debug_set_flags(1)
+        plan.decode(dptrs)
+        torch.cuda.synchronize()
+        assert plan.dec_status.cpu().tolist() == [sz.SZ_ERR_DEVICE_TIMEOUT] * 3
+    finally:
+        sz.sz_debug_set_flags(0)
+        sz.sz_set_wait_limit_ns(1_000_000_000)
+    plan.decode(dptrs)
+    torch.cuda.synchronize()
+    assert plan.dec_status.abs().sum().item() == 0
+    assert torch.equal(dst, pool)
     for k, s_ in enumerate(streams):
         off, z = int(plan.out_offset[k]), int(plan.sizes[k].item())
         assert plan.container[off: off + z].cpu().numpy().tobytes() == oracle.encode(s_)
