@@ -274,9 +274,6 @@ sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, u
     h.seg_hist = w.seg_hist;
     h.seg_done = w.seg_done;
     h.rhist = w.rhist;
-    h.reset_status = d_status;  // the histogram kernel sets no status on a single stream
-    h.reset_size = d_out_bytes;
-    SZ_TRY_CUDA(launch_hist(h, false, s));
     EncodeArgs a{};  // the codebook the histogram kernel chose: no reselect
     a.batch = c.batch;
     a.base = d_in;
@@ -290,6 +287,9 @@ sz_status compress_pipelined(const uint16_t *d_in, uint64_t n, uint8_t *d_out, u
     a.enc_done = w.enc_done;
     a.wait_limit_ns = wait_limit_ns();
     a.debug_flags = debug_flags();
+    h.reset_status = d_status;  // the histogram kernel sets no status on a single stream
+    h.reset_size = d_out_bytes;
+    SZ_TRY_CUDA(launch_hist(h, false, s));
     return cuda_status(launch_encode(a, false, s));
 }
 

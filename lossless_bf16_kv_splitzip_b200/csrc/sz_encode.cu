@@ -63,41 +63,38 @@ struct __align__(128) EncShared {
     uint32_t esc[2][kEscStage];
 };
 
-// exponent -> code (0..15) or 0x80 (escape); static so that lookups address
-// it as [index + constant]
-__shared__ __align__(16) uint8_t s_lut[256];
+// Four lookup tables, one per position k of an element in its quad of 4:
+// entry e = code(e) << 4k for a codebook exponent, 1 << (16 + k) for an
+// escape (placeholder code 0).  OR-ing a quad's four entries gives its four
+// code nibbles in bits 0..15 and its escape flags in bits 16..19.  Static, so
+// that a lookup addresses it as [byte offset + constant].
+__shared__ __align__(16) uint32_t s_lut[4][256];
+
+__device__ __forceinline__ uint32_t lut_at(int k, uint32_t byte_off) {
+    return *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(s_lut[k]) + byte_off);
+}
 
 // ---------------------------------------------------------- chunk encode
 // 16 consecutive BF16 values (two uint4) -> 16 sm bytes, 8 code bytes and an
-// escape mask.  The LUT maps exponent -> code (0..15) or 0x80 (escape; its
-// low nibble 0 is the placeholder code).  Escape mask layout: element j of
-// the chunk is bit 8*(j%4) + j/4.
+// escape mask.  Escape mask layout: element j = 4q + k of the chunk is bit
+// k + 16 (q & 1) + 4 (q >> 1).
 __device__ __forceinline__ void encode_chunk(const uint4 v0, const uint4 v1, uint4 &sm, uint64_t &codes,
                                              uint32_t &esc) {
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint32_t smw[4], P[4];
-    esc = 0;
+    uint32_t smw[4], B[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint32_t a = w[2 * q], b = w[2 * q + 1];
         const uint32_t hi = prmt(a, b, 0x7531u);  // high bytes of the 4 values: sign | exp >> 1
         const uint32_t lo = prmt(a, b, 0x6420u);  // low bytes: exp & 1 | mantissa
         smw[q] = (hi & 0x80808080u) | (lo & 0x7F7F7F7Fu);
-        // the 4 exponents, one per byte: (hi << 1) supplies bits 7..1, lo's
-        // bit 7 supplies bit 0
-        const uint32_t e4 = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
-        uint32_t c[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) c[k] = s_lut[prmt(e4, 0u, 0x4440u | (uint32_t)k)];  // byte k, zero-extended
-        const uint32_t B = prmt(prmt(c[0], c[1], 0x5140u), prmt(c[2], c[3], 0x5140u), 0x5410u);
-        esc |= (B >> (7 - q)) & (0x01010101u << q);
-        // byte 0 = n0 | n1 << 4, byte 2 = n2 | n3 << 4 (the escape bits drop out)
-        P[q] = (B & 0x0F0F0F0Fu) | ((B >> 4) & 0xF0F0F0F0u);
+        // byte offset 4 * exponent of each value (exponent in bits 7..14 of its half)
+        B[q] = lut_at(0, (a >> 5) & 0x3FCu) | lut_at(1, (a >> 21) & 0x3FCu) | lut_at(2, (b >> 5) & 0x3FCu) |
+               lut_at(3, (b >> 21) & 0x3FCu);
     }
     sm = make_uint4(smw[0], smw[1], smw[2], smw[3]);
-    const uint32_t lo32 = prmt(P[0], P[1], 0x6420u);
-    const uint32_t hi32 = prmt(P[2], P[3], 0x6420u);
-    codes = (uint64_t)lo32 | ((uint64_t)hi32 << 32);
+    codes = (uint64_t)prmt(B[0], B[1], 0x5410u) | ((uint64_t)prmt(B[2], B[3], 0x5410u) << 32);
+    esc = prmt(B[0], B[1], 0x7632u) | (prmt(B[2], B[3], 0x7632u) << 4);
 }
 
 __device__ __forceinline__ uint32_t byte_of(uint4 v, int b) {  // b is a compile-time constant
@@ -105,18 +102,18 @@ __device__ __forceinline__ uint32_t byte_of(uint4 v, int b) {  // b is a compile
     return (w >> (8 * (b & 3))) & 0xFFu;
 }
 
-// Escape mask in element order (bit j = element j), from the interleaved
-// layout above: for each quad q, bits 8b + q (b = 0..3) are gathered by one
-// multiply -- the four products of 1 + 2^7 + 2^14 + 2^21 do not overlap, and
-// bits 21..24 receive b = 0..3 in order.
+// Escape mask in element order (bit j = element j), from the layout above.
 __device__ __forceinline__ uint32_t esc_in_element_order(uint32_t m) {
-    uint32_t r = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) r |= ((((m >> q) & 0x01010101u) * 0x00204081u) >> 21 & 0xFu) << (4 * q);
-    return r;
+    return (m & 0xFu) | ((m >> 12) & 0xF0u) | ((m << 4) & 0xF00u) | ((m >> 8) & 0xF000u);
 }
 
-__device__ __forceinline__ uint32_t esc_bit_of_elem(int j) { return 1u << (8 * (j & 3) + (j >> 2)); }
+__device__ __forceinline__ uint32_t esc_bit_of_elem(int j) {
+    return 1u << ((j & 3) | (((j >> 2) & 1) << 4) | ((j >> 3) << 2));
+}
+
+// Element of the chunk whose escape flag is bit b of the mask.
+__device__ __forceinline__ int elem_of_esc_bit(int b) { return (b & 3) | (((b >> 4) & 1) << 2) | (((b >> 2) & 1) << 3); }
+
 
 __device__ __forceinline__ uint32_t field16(uint64_t v, int c) { return (uint32_t)(v >> (16 * c)) & 0xFFFFu; }
 
@@ -199,16 +196,6 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
         if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
         for (uint32_t sub = 0; sub < r.n_subs; ++sub, ++j) {
             const int s = (int)(j % kEncStages);
-            // the next sub-tile into L2 ahead of its bulk copy: in this tile,
-            // or -- a single stream, where tiles follow in memory -- the next
-            // tile's first
-            {
-                uint64_t rest = 0;
-                if (sub + 1 < r.n_subs) rest = r.len - (sub + 1) * kSub;
-                else if (!kBatched && t + 1 < t_end) rest = r.n - (r.elem0 + r.len);
-                const uint32_t next = aligned ? ((uint32_t)umin64(kSub, rest) * 2u) & ~15u : 0u;
-                if (next) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src + (sub + 1) * kSub), "r"(next) : "memory");
-            }
             if (j >= (uint32_t)kEncStages && !mbar_wait(&sh.empty[s], ((j / kEncStages) - 1) & 1u, a.wait_limit_ns)) {
                 set_status(a.status + k, SZ_ERR_DEVICE_TIMEOUT);
                 return;
@@ -379,10 +366,15 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
             return;
         }
         if (m.seg != cur) {  // every consumer is past the previous sub-tile's compute
-            s_lut[tid] = 0x80;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s_lut[k][tid] = 1u << (16 + k);
             consumer_sync();
             const uint8_t *cbk = kOnePass ? a.codebooks_in + 16 * (size_t)m.seg : a.meta[m.seg].codebook;
-            if (tid < 16) s_lut[cbk[tid]] = (uint8_t)tid;
+            if (tid < 16) {
+                const uint32_t x = cbk[tid];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) s_lut[k][x] = (uint32_t)tid << (4 * k);
+            }
             const sz_segment seg = load_segment(a.batch, m.seg);
             out = a.out + seg.out_offset;
             n = seg.n_elems;
@@ -508,8 +500,7 @@ __device__ void encode_consumers(const EncodeArgs &a, EncShared &sh) {
                 uint32_t msk = multi ? esc_in_element_order(esc[c]) : 0u;
                 int q = 0;
                 if (!multi) {
-                    const int bit = __ffs(esc[c]) - 1;
-                    q = 4 * (bit & 7) + (bit >> 3);
+                    q = elem_of_esc_bit(__ffs(esc[c]) - 1);
                 } else {
                     q = __ffs(msk) - 1;
                     msk &= msk - 1;
@@ -768,9 +759,14 @@ __global__ void __launch_bounds__(kThreads) small_encode_kernel(const uint16_t *
     __shared__ int s_last;
     const uint32_t tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const uint32_t nb = (uint32_t)umax64(1, div_up(n, kSlice));  // an empty stream: one block
-    s_lut[tid] = 0x80;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s_lut[k][tid] = 1u << (16 + k);
     __syncthreads();
-    if (tid < 16) s_lut[w.meta->codebook[tid]] = (uint8_t)tid;
+    if (tid < 16) {
+        const uint32_t x = w.meta->codebook[tid];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s_lut[k][x] = (uint32_t)tid << (4 * k);
+    }
     const uint64_t e_total = w.meta->n_escapes;
     if (container_size(n, e_total) > out_cap) {  // the same decision in every block
         if (tid == 0 && blockIdx.x == 0) set_status(status, SZ_ERR_CAPACITY);

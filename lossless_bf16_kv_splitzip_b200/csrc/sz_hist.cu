@@ -183,10 +183,10 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
 
 // Segments with no elements have no tiles, so no range completes them:
 // their codebook is exponents 0..15 (all counts zero) and e = 0.
-__device__ void empty_segments(const HistArgs &h) {
+__device__ inline void empty_segments(const HistArgs &h) {
     const SelectCtx &a = h.sel;
     const uint32_t ns = a.batch.segs ? a.batch.n_segs : 1u;
-    for (uint32_t k = threadIdx.x; k < ns; k += blockDim.x) {
+    for (uint32_t k = threadIdx.x; k < ns; k += kThreads) {
         if (load_segment(a.batch, k).n_elems != 0) continue;
         SegMeta &m = a.meta[k];
         for (int q = 0; q < 16; ++q) {
@@ -198,40 +198,22 @@ __device__ void empty_segments(const HistArgs &h) {
         m.pad = 0;
     }
     if (a.hist_out && a.batch.segs == nullptr && a.batch.single.n_elems == 0)
-        for (uint32_t i = threadIdx.x; i < 256; i += blockDim.x) a.hist_out[i] = 0;
+        for (uint32_t i = threadIdx.x; i < 256; i += kThreads) a.hist_out[i] = 0;
 }
 
 // ------------------------------------------------------------- histogram
-// One block per range.  The tiles of a range are counted piece by piece (a
-// piece = the range's tiles of one segment); at the end of a piece its 256
-// counts are the difference of the column sums, added to the segment's
-// counts, and kept when the piece opens or closes the range.  The block
-// that completes a segment's tile count runs that segment's select.
-// kSmallTiles: every tile is a single sub-tile (pages of at most 16,384
-// elements, or the one-sub-tile tiles of a short single stream); that
-// build is given registers for 3 blocks per SM -- measured 0.70 -> 0.86 of
-// the copy bandwidth on 16-token pages, while the same bound costs 8 % on
-// 65,536-element tiles, which keep the default build.
-// kAccum: the accumulate mode -- each piece's counts are added to the
-// caller's histogram of its segment (a.accum, row a.accum_index[k] or k);
-// no range records, no completion count, no select.
-template <bool kBatched, bool kSmallTiles, bool kAccum>
-__global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(const HistArgs a) {
-    extern __shared__ __align__(128) uint32_t s_hist[];  // kHistWords
-    __shared__ SegCache s_segc;
-    __shared__ SelShared s_sel;
-    static_assert(kThreads == 256, "one thread per bin");
+// The tiles of range blockIdx.x counted piece by piece (a piece = the
+// range's tiles of one segment) by the block's kThreads threads, into the
+// 256 x 32 lane columns s_hist (zeroed, and seg_cache filled, before);
+// at the end of a piece its 256 counts are the difference of the column
+// sums, added to the segment's counts, and kept when the piece opens or
+// closes the range.  The block that completes a segment's tile count runs
+// that segment's select.
+// kAccum: the piece counts go to the caller's histograms instead (no range
+// records, no completion count, no select).
+template <bool kBatched, bool kAccum>
+__device__ void count_range(const HistArgs &a, uint32_t *s_hist, const SegCache &s_segc, SelShared &s_sel) {
     const Batch &batch = a.sel.batch;
-
-    allow_dependents();  // the encode kernel may start its prologue
-    if (blockIdx.x == 0 && threadIdx.x == 0) {  // words only the next kernel reads
-        if (a.reset_status) *a.reset_status = SZ_OK;
-        if (a.reset_size) *a.reset_size = 0;
-    }
-    for (uint32_t i = threadIdx.x; i < kHistWords; i += kThreads) s_hist[i] = 0;
-    seg_cache_fill(s_segc, batch);  // ends with __syncthreads
-    if (!kAccum && blockIdx.x == 0) empty_segments(a);
-
     const uint32_t tid = threadIdx.x;
     const uint32_t col = smem_u32(s_hist) + (tid & 31) * 4;
     const uint64_t R = a.sel.range_tiles;
@@ -315,6 +297,31 @@ __global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(con
             select_segment(a.sel, k, nullptr, s_sel);
         }
     }
+}
+
+
+// ------------------------------------------------------------- histogram
+// One block per range (count_range).  kSmallTiles: every tile is a single
+// sub-tile (pages of at most 16,384 elements, or the one-sub-tile tiles of
+// a short single stream); that build is given registers for 3 blocks per
+// SM -- measured 0.70 -> 0.86 of the copy bandwidth on 16-token pages,
+// while the same bound costs 8 % on 65,536-element tiles, which keep the
+// default build.
+template <bool kBatched, bool kSmallTiles, bool kAccum>
+__global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(const HistArgs a) {
+    extern __shared__ __align__(128) uint32_t s_hist[];  // kHistWords
+    __shared__ SegCache s_segc;
+    __shared__ SelShared s_sel;
+    static_assert(kThreads == 256, "one thread per bin");
+    allow_dependents();  // the encode kernel may start its prologue
+    if (blockIdx.x == 0 && threadIdx.x == 0) {  // words only the next kernel reads
+        if (a.reset_status) *a.reset_status = SZ_OK;
+        if (a.reset_size) *a.reset_size = 0;
+    }
+    for (uint32_t i = threadIdx.x; i < kHistWords; i += kThreads) s_hist[i] = 0;
+    seg_cache_fill(s_segc, a.sel.batch);  // ends with __syncthreads
+    if (!kAccum && blockIdx.x == 0) empty_segments(a);
+    count_range<kBatched, kAccum>(a, s_hist, s_segc, s_sel);
 }
 
 // Caller codebook for a single tensor: the select again with that codebook,

@@ -241,45 +241,6 @@ __device__ __forceinline__ void store_u32_le(uint8_t *p, uint32_t v, bool aligne
     }
 }
 
-// Rank of exponent `tid` (count c) in the order (count descending, exponent
-// ascending): the number of exponents before it; ranks 0..15 are the
-// codebook.  Every one of the 256 threads calls it (thread t = exponent t).
-// Only the exponents that occur are compared: they are compacted, in
-// ascending order, as keys count << 8 | (255 - exponent) -- one key is
-// greater than another exactly when it comes first -- and an exponent that
-// does not occur ranks after all that do, in ascending order (its rank is
-// the number of occurring exponents plus the absent ones below it).
-struct RankShared {
-    unsigned long long key[256];
-    uint32_t warp[kWarps];
-};
-__device__ inline uint32_t exponent_rank(uint32_t c, uint32_t tid, RankShared &rs) {
-    const uint32_t lane = tid & 31, wid = tid >> 5;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, c != 0);
-    if (lane == 0) rs.warp[wid] = __popc(m);
-    __syncthreads();
-    uint32_t before = 0, nnz = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        const uint32_t x = rs.warp[w];
-        before += (uint32_t)w < wid ? x : 0u;
-        nnz += x;
-    }
-    const uint32_t pos = before + __popc(m & ((1u << lane) - 1u));  // occurring exponents below tid
-    const unsigned long long mine = ((unsigned long long)c << 8) | (255u - tid);
-    if (c) rs.key[pos] = mine;
-    __syncthreads();
-    uint32_t rank = 0;
-    if (c == 0) {
-        rank = nnz + (tid - pos);
-    } else {
-#pragma unroll 4
-        for (uint32_t u = 0; u < nnz; ++u) rank += rs.key[u] > mine;
-    }
-    __syncthreads();  // the scratch may be reused
-    return rank;
-}
-
 // ------------------------------------------------------------ status words
 __device__ inline void set_status(int32_t *status, int32_t code) {
     if (status != nullptr) atomicCAS(reinterpret_cast<int *>(status), 0, code);
@@ -349,6 +310,46 @@ cudaError_t launch_after(void (*kernel)(Params...), dim3 grid, dim3 block, size_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
+// Rank of exponent `tid` (count c) in the order (count descending, exponent
+// ascending): the number of exponents before it; ranks 0..15 are the
+// codebook.  Every one of the 256 threads of the block calls it (thread t =
+// exponent t).
+// Only the exponents that occur are compared: they are compacted, in
+// ascending order, as keys count << 8 | (255 - exponent) -- one key is
+// greater than another exactly when it comes first -- and an exponent that
+// does not occur ranks after all that do, in ascending order (its rank is
+// the number of occurring exponents plus the absent ones below it).
+struct RankShared {
+    unsigned long long key[256];
+    uint32_t warp[kWarps];
+};
+__device__ inline uint32_t exponent_rank(uint32_t c, uint32_t tid, RankShared &rs) {
+    const uint32_t lane = tid & 31, wid = tid >> 5;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, c != 0);
+    if (lane == 0) rs.warp[wid] = __popc(m);
+    __syncthreads();
+    uint32_t before = 0, nnz = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t x = rs.warp[w];
+        before += (uint32_t)w < wid ? x : 0u;
+        nnz += x;
+    }
+    const uint32_t pos = before + __popc(m & ((1u << lane) - 1u));  // occurring exponents below tid
+    const unsigned long long mine = ((unsigned long long)c << 8) | (255u - tid);
+    if (c) rs.key[pos] = mine;
+    __syncthreads();
+    uint32_t rank = 0;
+    if (c == 0) {
+        rank = nnz + (tid - pos);
+    } else {
+#pragma unroll 4
+        for (uint32_t u = 0; u < nnz; ++u) rank += rs.key[u] > mine;
+    }
+    __syncthreads();  // the scratch may be reused
+    return rank;
 }
 
 // ------------------------------------------------- mbarrier + 1-D TMA copy

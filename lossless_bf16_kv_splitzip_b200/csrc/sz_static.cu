@@ -72,8 +72,8 @@ extern "C" sz_status sz_encode_static(const uint16_t *d_in, uint64_t n, uint8_t 
     DeviceInfo dev;
     if (const sz_status st = device_info(dev)) return st;
     // The array keeps the previous call's contents: the tensor counts and
-    // the two completion counts are accumulated with atomics and are
-    // cleared first; everything else is overwritten before it is read.
+    // the two completion counts are cleared first; everything else is
+    // overwritten before it is read.
     CompressScratch cs;
     cs.zero = ws + kOffSegHist;
     cs.zero_bytes = kOffEncDone + 4;

@@ -336,11 +336,13 @@ def test_odd_tail_nibble_rejected():
 
 
 # -------------------------------------------------- one-call compression
-@pytest.mark.parametrize("n", [0, 1, 17, 4095, 4096, 4097, 32769, 65537, 3 * 65536 + 100, SHORT, SHORT + 1])
+@pytest.mark.parametrize("n", [0, 1, 17, 4095, 4096, 4097, 32769, 65537, 3 * 65536 + 100, SHORT, SHORT + 1,
+                               (1 << 23) + 7, (1 << 25) + 12345, (1 << 26) + 33, (1 << 27) - 5, (1 << 27) + 16])
 def test_compress_one_call_equals_oracle(n):
     """sz_compress: short streams by 4,096-element blocks in two launches,
-    longer ones by the histogram and encode kernels; the same bytes as the
-    oracle (and as the two-call path), and the codebook it reports is the
+    longer ones by the histogram and encode kernels (16,384-element tiles
+    below 2^27 elements, 65,536 from there); the same bytes as the oracle
+    (and as the two-call path), and the codebook it reports is the
     header's."""
     x = kvgen.mixed_small(n, seed=300 + n % 101)
     cb = torch.zeros(16, dtype=torch.uint8, device=DEV)
@@ -439,6 +441,27 @@ def test_stage_wait_timeout_on_several_ranges_and_one_pass():
     for k, s_ in enumerate(streams):
         off, z = int(plan.out_offset[k]), int(plan.sizes[k].item())
         assert plan.container[off: off + z].cpu().numpy().tobytes() == oracle.encode(s_)
+
+
+@pytest.mark.parametrize("n", [SHORT + 5, (1 << 24) + 3])
+def test_compress_wait_times_out_cleanly(n):
+    """sz_compress of a stream past the short-stream limit: every stage wait
+    of its encode kernel runs out; status SZ_ERR_DEVICE_TIMEOUT, size 0, and
+    the next call is bit-exact."""
+    x = kvgen.mixed_small(n, seed=36)
+    try:
+        sz.sz_set_wait_limit_ns(2_000_000)
+        sz.sz_debug_set_flags(1)
+        out, size, status = sz.compress(to_dev(x))
+        torch.cuda.synchronize()
+        assert int(status.item()) == sz.SZ_ERR_DEVICE_TIMEOUT and int(size.item()) == 0
+    finally:
+        sz.sz_debug_set_flags(0)
+        sz.sz_set_wait_limit_ns(1_000_000_000)
+    out, size, status = sz.compress(to_dev(x))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert out[: int(size.item())].cpu().numpy().tobytes() == oracle.encode(x)
 
 
 def test_decode_stage_wait_times_out_cleanly():
