@@ -120,10 +120,8 @@ Batch single_batch(uint64_t n) {
     b.segs = nullptr;
     b.n_segs = 1;
     b.page_elems = n > 0 ? n : 1;
-    b.tile_subs = n < kSmallTileBelow ? 1u : kSubsPerTile;
-    b.tile_elems = kSub * b.tile_subs;
-    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems, b.tile_elems);
-    b.n_tiles = segment_tiles(n, b.page_elems, b.tile_elems);
+    set_tiles(b, n < kSmallTileBelow ? 1u : kSubsPerTile);
+    b.n_tiles = segment_tiles(n, b.page_elems, b.tile_shift);
     b.single.n_elems = n;
     b.single.page_begin = 0;
     b.single.out_offset = 0;
@@ -140,9 +138,7 @@ Batch make_batch(uint32_t n_segs, const sz_segment *d_segs, uint64_t n_tiles, ui
     b.segs = d_segs;
     b.n_segs = n_segs;
     b.page_elems = page_elems;
-    b.tile_subs = kSubsPerTile;
-    b.tile_elems = kTile;
-    b.tiles_per_page = (uint32_t)tiles_per_page(page_elems, kTile);
+    set_tiles(b, kSubsPerTile);
     b.n_tiles = n_tiles;
     return b;
 }
@@ -442,7 +438,7 @@ sz_status sz_plan_batched(uint32_t n_segs, const uint64_t *h_seg_elems, uint64_t
         h_segs[k].out_offset = out;
         h_segs[k].tile_begin = tiles;
         pages += div_up(n, page_elems);
-        tiles += segment_tiles(n, page_elems, kTile);
+        tiles += segment_tiles(n, page_elems, 16);
         out += round_up(SZ_MAX_BYTES(n), kAlign);
     }
     if (multi_page && page_elems % 64 != 0) return SZ_ERR_ALIGN;

@@ -70,13 +70,15 @@ __device__ inline Header read_header(const uint8_t *c, uint64_t cap, uint64_t n)
 // 0..S*tiles_k) = index of the first escape whose position is >= the first
 // element of that sub-tile (sub-tiles past a short tile's end start at the
 // tile's end); entry S*tiles_k = e.  Entries of segment k start at
-// S*tile_begin_k + k.  One warp per entry: a 32-way search over the
-// ascending position stream (each round probes 32 evenly spaced records and
-// keeps the interval where the positions reach the target, so about log32 e
-// dependent loads).  On a corrupt stream the search still ends, on some
-// index; the decode's per-sub-tile checks reject the records.  The entry of
-// the segment's sentinel also writes the segment's status (SZ_OK, or the
-// header's error): the decode kernel after it only ever sets errors.
+// S*tile_begin_k + k.  kWarp (few entries, where latency rules): one warp per
+// entry, a 32-way search over the ascending position stream (each round
+// probes 32 evenly spaced records and keeps the interval where the positions
+// reach the target, so about log32 e dependent loads); else one thread per
+// entry and a binary search (log2 e dependent loads, 32x fewer threads).
+// On a corrupt stream either search still ends, on some index; the decode's
+// per-sub-tile checks reject the records.  The entry of the segment's
+// sentinel also writes the segment's status (SZ_OK, or the header's error):
+// the decode kernel after it only ever sets errors.
 __device__ inline uint64_t warp_first_at_least(const uint8_t *pos, uint64_t e, uint64_t target, uint32_t lane) {
     uint64_t lo = 0, hi = e;  // the answer is in [lo, hi]
     while (lo < hi) {
@@ -94,7 +96,7 @@ __device__ inline uint64_t warp_first_at_least(const uint8_t *pos, uint64_t e, u
     return lo;
 }
 
-template <bool kBatched>
+template <bool kBatched, bool kWarp>
 __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint64_t n_entries) {
     __shared__ uint64_t s_entry_begin[kMaxSmemSegs + 1];
     allow_dependents();      // the decode kernel may start its prologue
@@ -107,8 +109,8 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
             s_entry_begin[i] = S * a.batch.segs[i].tile_begin + i;
     }
     __syncthreads();
-    const uint32_t lane = threadIdx.x & 31;
-    const uint64_t j_glob = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // one warp per entry
+    const uint32_t lane = kWarp ? threadIdx.x & 31 : 0u;
+    const uint64_t j_glob = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> (kWarp ? 5 : 0);
     if (j_glob >= n_entries) return;
     uint32_t k = 0;
     if (kBatched) {  // largest k with S*tile_begin_k + k <= j_glob
@@ -140,7 +142,17 @@ __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint
         const TileRef r = resolve_tile(a.batch, seg, k, seg.tile_begin + j / S);
         const uint64_t first = r.elem0 + umin32((uint32_t)(j % S) * kSub, r.len);
         const uint64_t n = h.n;
-        idx = warp_first_at_least(c + kHeader + n + (n + 1) / 2, h.e, first, lane);
+        const uint8_t *pos = c + kHeader + n + (n + 1) / 2;
+        if (kWarp) {
+            idx = warp_first_at_least(pos, h.e, first, lane);
+        } else {  // first index with pos >= first
+            uint64_t lo = 0, hi = h.e;
+            while (lo < hi) {
+                const uint64_t mid = (lo + hi) >> 1;
+                if (load_u32_any(pos + 4 * mid) < first) lo = mid + 1; else hi = mid;
+            }
+            idx = lo;
+        }
     }
     if (lane == 0) ts[j] = (uint32_t)idx;
 }
@@ -245,14 +257,11 @@ struct __align__(128) DecShared {
 // of a contiguous tensor, several when pages are smaller than a tile, so
 // that a CTA meets a new segment (header, codebook tables) at most once per
 // group.  Group g holds tiles [g * group, (g + 1) * group).
-__host__ __device__ inline uint64_t tiles_per_group(const Batch &b) {
-    const uint64_t tile_elems = b.page_elems < (uint64_t)kTile ? b.page_elems : (uint64_t)kTile;
-    const uint64_t g = (uint64_t)kTile / (tile_elems > 0 ? tile_elems : 1);
-    return g > 0 ? g : 1;
-}
+__host__ __device__ inline uint64_t tiles_per_group(const Batch &b) { return b.group_tiles; }
 
 // The tile a CTA of `grid` decodes after tile t.
 __device__ __forceinline__ uint64_t next_dealt_tile(uint64_t t, uint64_t group, uint32_t grid) {
+    if (group == 1) return t + grid;
     return (t + 1) % group == 0 ? t + 1 + (uint64_t)(grid - 1) * group : t + 1;
 }
 
@@ -636,12 +645,21 @@ cudaError_t launch_small_decode(const uint8_t *c, uint64_t cap, uint16_t *out, u
     return cudaGetLastError();
 }
 
-// Also writes every segment's status word (no memset before it).
+// Also writes every segment's status word (no memset before it).  A warp
+// per entry while the warps fit about one wave of the GPU, a thread per
+// entry beyond.
+constexpr uint64_t kWarpIndexMax = 8192;
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) {
     const uint64_t entries = (uint64_t)a.batch.tile_subs * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
-    const uint64_t grid = div_up(entries, 256 / 32);  // one warp per entry
-    const cudaError_t e = batched ? launch_after(esc_index_kernel<true>, dim3((unsigned)grid), dim3(256), 0, s, a, entries)
-                                  : launch_after(esc_index_kernel<false>, dim3((unsigned)grid), dim3(256), 0, s, a, entries);
+    const bool warp = entries <= kWarpIndexMax;
+    const dim3 grid((unsigned)div_up(entries, warp ? 256 / 32 : 256)), block(256);
+    cudaError_t e;
+    if (batched)
+        e = warp ? launch_after(esc_index_kernel<true, true>, grid, block, 0, s, a, entries)
+                 : launch_after(esc_index_kernel<true, false>, grid, block, 0, s, a, entries);
+    else
+        e = warp ? launch_after(esc_index_kernel<false, true>, grid, block, 0, s, a, entries)
+                 : launch_after(esc_index_kernel<false, false>, grid, block, 0, s, a, entries);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

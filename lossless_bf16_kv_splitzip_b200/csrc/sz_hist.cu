@@ -212,7 +212,7 @@ __device__ inline void empty_segments(const HistArgs &h) {
 // kAccum: the piece counts go to the caller's histograms instead (no range
 // records, no completion count, no select).
 template <bool kBatched, bool kAccum>
-__device__ void count_range(const HistArgs &a, uint32_t *s_hist, const SegCache &s_segc, SelShared &s_sel) {
+__device__ __forceinline__ void count_range(const HistArgs &a, uint32_t *s_hist, const SegCache &s_segc, SelShared &s_sel) {
     const Batch &batch = a.sel.batch;
     const uint32_t tid = threadIdx.x;
     const uint32_t col = smem_u32(s_hist) + (tid & 31) * 4;

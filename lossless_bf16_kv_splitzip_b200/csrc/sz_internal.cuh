@@ -91,14 +91,14 @@ __host__ __device__ inline uint64_t umax64(uint64_t a, uint64_t b) { return a > 
 __host__ __device__ inline uint32_t umin32(uint32_t a, uint32_t b) { return a < b ? a : b; }
 
 // Tiles of a segment of n elements in pages of page_elems: every page is cut
-// into tiles of tile_elems elements (its last tile may be short).
-__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems, uint64_t tile_elems) {
-    return div_up(page_elems, tile_elems);
+// into tiles of 2^tile_shift elements (its last tile may be short).
+__host__ __device__ inline uint64_t tiles_per_page(uint64_t page_elems, uint32_t tile_shift) {
+    return (page_elems + (1ull << tile_shift) - 1) >> tile_shift;
 }
-__host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems, uint64_t tile_elems) {
+__host__ __device__ inline uint64_t segment_tiles(uint64_t n, uint64_t page_elems, uint32_t tile_shift) {
     if (n == 0) return 0;
-    const uint64_t full = n / page_elems, rem = n % page_elems;
-    return full * tiles_per_page(page_elems, tile_elems) + div_up(rem, tile_elems);
+    const uint64_t full = n / page_elems, rem = n - full * page_elems;
+    return full * tiles_per_page(page_elems, tile_shift) + ((rem + (1ull << tile_shift) - 1) >> tile_shift);
 }
 
 // ------------------------------------------------------------ tile lookup
@@ -111,12 +111,28 @@ struct Batch {
     uint32_t tiles_per_page;  // ceil(page_elems / tile_elems), precomputed on the host
     uint32_t tile_subs;       // sub-tiles per tile: kSubsPerTile, or 1 for short single streams
     uint32_t tile_elems;      // kSub * tile_subs
+    uint32_t tile_shift;      // log2(tile_elems)
+    uint32_t group_tiles;     // the decode deals tiles round robin in groups of this many
     uint64_t n_tiles;
     sz_segment single;        // the implicit segment of a single-tensor call
 };
 
 __host__ __device__ inline uint64_t seg_tiles(const Batch &b, uint64_t n) {
-    return segment_tiles(n, b.page_elems, b.tile_elems);
+    return segment_tiles(n, b.page_elems, b.tile_shift);
+}
+
+// Tile size of a batch: tile_subs sub-tiles of kSub elements.  The decode
+// deals tiles round robin in groups of about kTile elements -- one tile, or
+// several pages shorter than a tile -- so that a CTA meets a new segment at
+// most once per group.
+__host__ __device__ inline void set_tiles(Batch &b, uint32_t tile_subs) {
+    b.tile_subs = tile_subs;
+    b.tile_elems = kSub * tile_subs;
+    b.tile_shift = tile_subs == 1 ? 14u : 16u;
+    b.tiles_per_page = (uint32_t)tiles_per_page(b.page_elems, b.tile_shift);
+    const uint64_t te = b.page_elems < (uint64_t)kTile ? b.page_elems : (uint64_t)kTile;
+    const uint64_t g = (uint64_t)kTile / (te > 0 ? te : 1);
+    b.group_tiles = g > 0 ? (uint32_t)g : 1u;
 }
 // one-pass encode: escape records a tile's workspace slot holds
 __host__ __device__ inline uint32_t slot_cap(const Batch &b) { return b.tile_elems / kSlotDiv; }
@@ -191,15 +207,15 @@ __device__ inline TileRef resolve_tile(const Batch &b, const sz_segment &s, uint
     r.n = s.n_elems;
     const uint32_t tpp = b.tiles_per_page;
     const uint32_t te = b.tile_elems;
-    r.page = r.local / tpp;
-    r.in_page = (r.local - r.page * tpp) * te;
+    r.page = tpp == 1 ? r.local : r.local / tpp;
+    r.in_page = (r.local - r.page * tpp) << b.tile_shift;
     r.elem0 = (uint64_t)r.page * b.page_elems + r.in_page;
     const uint64_t page_len = umin64(b.page_elems, r.n - (uint64_t)r.page * b.page_elems);
     r.len = (uint32_t)umin64(te, page_len - r.in_page);
     r.n_subs = (r.len + kSub - 1) / kSub;
     const uint64_t full = r.n / b.page_elems;
     const uint64_t rem = r.n - full * b.page_elems;
-    r.tiles = (uint32_t)(full * tpp + (rem + te - 1) / te);
+    r.tiles = (uint32_t)(full * tpp + ((rem + te - 1) >> b.tile_shift));
     return r;
 }
 
