@@ -16,10 +16,12 @@
 //                    escape positions and exponents into a 2-stage ring;
 //   8 consumer warps turn codes + sm bytes into BF16 with register-only
 //                    PRMT lookups and write 16-byte stores (the escaped
-//                    places get codebook[0]); then, after one barrier, one
-//                    thread per escape checks its record (inside the
-//                    sub-tile, strictly ascending, raw exponent outside the
-//                    codebook, placeholder code 0) and overwrites the value.
+//                    places get codebook[0]); then, after one barrier per
+//                    sub-tile -- into which the wait for the next stage's
+//                    data is folded -- one thread per escape checks its
+//                    record (inside the sub-tile, strictly ascending, raw
+//                    exponent outside the codebook, placeholder code 0) and
+//                    overwrites the value.
 // Monotone sub-tile starts plus in-sub-tile checks prove the whole escape
 // stream well formed.  Every mbarrier wait is bounded.
 //
@@ -250,7 +252,7 @@ struct __align__(128) DecShared {
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
     SegCache segc;
-    int go;
+    int go[2];  // stage j's data arrived (slot j & 1)
 };
 
 // Tiles are dealt round robin in groups of about kTile elements: one tile
@@ -454,11 +456,14 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
     // thread 0: this CTA's first tile not yet decoded completely (every
     // consumer has passed the barrier below when it is read)
     uint64_t next_tile = (uint64_t)blockIdx.x * tiles_per_group(a.batch);
+    // One consumer barrier per sub-tile: after its values are stored, thread
+    // 0 waits for the next stage's data, then the barrier orders every store
+    // before the escape patches and hands the next stage's arrival to all.
+    if (tid == 0) sh.go[0] = mbar_wait(&sh.full[0], 0u, a.wait_limit_ns) ? 1 : 0;
+    consumer_sync();
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kDecStages);
-        if (tid == 0) sh.go = mbar_wait(&sh.full[s], (j / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
-        consumer_sync();
-        if (!sh.go) {  // the same decision in every consumer thread
+        if (!sh.go[j & 1]) {  // the same decision in every consumer thread
             if (tid == 0) decode_timeout_from(a, sh.segc, next_tile);
             return;
         }
@@ -482,11 +487,13 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
 #pragma unroll
         for (int q = 0; q < kChunks; ++q) decode_store_chunk(m, sh, s, T, q, tid, status);
 
+        const int s_next = (int)((j + 1) % kDecStages);
+        if (tid == 0) sh.go[(j + 1) & 1] = mbar_wait(&sh.full[s_next], ((j + 1) / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
+        consumer_sync();
+
         // ---- escapes, one per thread, after every chunk store of the
-        // sub-tile (the barrier orders the two writes of an escaped place):
-        // check the record and overwrite its value's exponent
+        // sub-tile: check the record and overwrite its value's exponent
         if (m.cnt) {
-            consumer_sync();
             const bool es = (m.flags & kDFlagEscSmem) != 0;
             const bool ss = (m.flags & kDFlagInSmem) != 0;
             const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
