@@ -294,17 +294,17 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
  * codebook.
  *
  * Three kernels: the encode writes the sign+mantissa and code streams in
- * place and parks each 65,536-element tile's escape records (up to 4,096 per
- * tile, 6.25 %) in the workspace; a placement kernel then counts each
- * segment's escapes, writes the header and moves the records into place; a
- * third kernel reads again the input of every tile with more than 4,096
- * escapes (spread over the GPU), and its last block writes every segment's
- * size (0 for a segment with an error).
+ * place and parks each tile's escape records (up to 1/16 of the tile,
+ * 4,096 per 65,536-element tile) in the workspace; a placement kernel then
+ * counts each segment's escapes, writes the header and moves the records
+ * into place; a third kernel reads again the input of every tile with more
+ * escapes than its slot holds (spread over the GPU), and its last block
+ * writes every segment's size (0 for a segment with an error).
  *
  * sz_plan_one_pass -- worst-case container (every element an escape:
- * 48 + n + ceil(n/2) + 5n) and workspace bytes (16,420 bytes per tile,
- * about 1/8 of the input's bytes, plus 16 bytes per range and 4 per
- * segment).  Host only.
+ * 48 + n + ceil(n/2) + 5n) and workspace bytes (16,420 bytes per 65,536
+ * elements, about 1/8 of the input's bytes, plus 16 bytes per range and 4
+ * per segment).  Host only.
  */
 sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes);
 
@@ -451,8 +451,11 @@ sz_status sz_set_wait_limit_ns(uint64_t limit_ns);
  */
 sz_status sz_debug_set_flags(uint32_t flags);
 
-/* Tile size in elements used by every kernel (65536; a tile never crosses
- * a page, so the last tile of a page may be shorter). */
+/* Tile size in elements of the batched calls and of single streams of 2^27
+ * elements or more: 65536 (a tile never crosses a page, so the last tile of
+ * a page may be shorter).  Single-stream calls on shorter streams cut them
+ * into tiles of 16384 elements, so that a mid-size stream still spreads over
+ * every CTA; the containers do not depend on the tile size. */
 uint64_t sz_tile_elems(void);
 
 /* Library version string, e.g. "splitzip-b200 1.0 sm_100a". */
