@@ -47,7 +47,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 //   seg_done   u32[S]          tiles counted so far per segment } by the histogram call
 //   enc_done   u32[S]          tiles of complete encode pieces  } (and by the encode call)
 //   meta       SegMeta[S]      codebook and escape count per segment
-//   rhist      u32[G][2][256]  counts of each range's first and last piece
+//   rhist      u32[2][256][G]  counts of each range's first and last piece (range-minor)
 //   rrec       RangeRec[G]     escape placement of each range's pieces
 //   sub_start  u32[ST + S]     first escape index of each sub-tile (decode; S = sub-tiles per tile)
 struct Ws {

@@ -101,8 +101,11 @@ __device__ inline uint64_t warp_first_at_least(const uint8_t *pos, uint64_t e, u
 template <bool kBatched, bool kWarp>
 __global__ void __launch_bounds__(256) esc_index_kernel(const DecodeArgs a, uint64_t n_entries) {
     __shared__ uint64_t s_entry_begin[kMaxSmemSegs + 1];
-    allow_dependents();      // the decode kernel may start its prologue
     grid_dependency_wait();  // the kernel that wrote the containers has finished
+    // The decode kernel may start now: every container is complete, so it
+    // may read headers, sm bytes and codes before its own wait (only the
+    // index entries and status words written here need that wait).
+    allow_dependents();
     const uint32_t S = a.batch.tile_subs;
     const uint32_t ns = kBatched ? a.batch.n_segs : 1u;
     const bool cached = kBatched && ns <= kMaxSmemSegs;
@@ -230,6 +233,14 @@ constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
 constexpr uint32_t kDFlagTileEnd = 4u;  // last sub-tile of its tile
 constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage
 
+// What the producer read and copied before the grid dependency wait.
+struct DecEarly {
+    uint32_t n;  // leading sub-tiles whose sm + code copies were issued
+    uint32_t k;  // segment whose header was read (0xFFFFFFFF: none)
+    sz_segment seg;
+    Header h;
+};
+
 struct DecMeta {
     uint16_t *dst;      // global destination of the sub-tile's first element
     const uint8_t *c;   // the segment's container
@@ -252,6 +263,7 @@ struct __align__(128) DecShared {
     uint64_t full[kDecStages];
     uint64_t empty[kDecStages];
     SegCache segc;
+    DecEarly early;  // producer only: what it read and copied before the grid dependency wait
     int go[2];  // stage j's data arrived (slot j & 1)
 };
 
@@ -281,12 +293,55 @@ __device__ void decode_timeout_from(const DecodeArgs &a, const SegCache &c, uint
 }
 
 // ------------------------------------------------------------ producer
+// Before the grid dependency wait (the index kernel's end): the header of
+// the CTA's first segment and the sm + code copies of its first kDecStages
+// sub-tiles -- what the containers alone give, not the index entries or
+// status words the index kernel writes.  The containers are complete here:
+// the index kernel lets this kernel start only after its own wait for the
+// kernel that wrote them.  Stops at the first sub-tile that is short, in
+// another segment, or whose header or alignment rules out bulk copies; the
+// issued stages have their transaction count set, and the producer arrives
+// on them after the wait.  Sets no status (the index kernel writes it).
+template <bool kBatched>
+__device__ void decode_prefetch(const DecodeArgs &a, DecShared &sh) {
+    DecEarly &p = sh.early;  // the producer thread's own (shared memory: no registers held over the wait)
+    p.n = 0;
+    p.k = 0xFFFFFFFFu;
+    if ((a.debug_flags & kDebugNoSignal) != 0) return;
+    const uint64_t group = tiles_per_group(a.batch);
+    for (uint64_t t = (uint64_t)blockIdx.x * group; t < a.batch.n_tiles && p.n < (uint32_t)kDecStages;
+         t = next_dealt_tile(t, group, gridDim.x)) {
+        const uint32_t k = find_segment(sh.segc, a.batch, t);
+        if (k != p.k) {
+            if (p.k != 0xFFFFFFFFu) return;
+            p.k = k;
+            p.seg = load_segment(a.batch, k);
+            const uint64_t cap = p.seg.out_offset <= a.in_cap ? a.in_cap - p.seg.out_offset : 0;
+            p.h = read_header(a.in + p.seg.out_offset, cap, p.seg.n_elems);
+        }
+        if (!p.h.ok || (p.seg.n_elems % 16) != 0) return;
+        const TileRef r = resolve_tile(a.batch, p.seg, k, t);
+        const uint8_t *c = a.in + p.seg.out_offset;
+        for (uint32_t sub = 0; sub < r.n_subs && p.n < (uint32_t)kDecStages; ++sub) {
+            if (r.len - sub * kSub < kSub) return;
+            const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
+            mbar_expect_tx(&sh.full[p.n], kSub + kSub / 2);
+            tma_load_1d(sh.sm[p.n], c + kHeader + elem0, kSub, &sh.full[p.n]);
+            tma_load_1d(sh.codes[p.n], c + kHeader + p.h.n + elem0 / 2, kSub / 2, &sh.full[p.n]);
+            ++p.n;
+        }
+    }
+}
+
 // One thread: per sub-tile, wait for the stage to be free, then bulk-copy
 // the sm bytes, the codes and (when they fit and stay inside the buffer) a
-// 16-byte aligned superset of the sub-tile's escape positions and exponents.
+// 16-byte aligned superset of the sub-tile's escape positions and exponents
+// (the first sh.early.n sub-tiles: only the escape records, the rest was
+// copied before the wait).
 template <bool kBatched>
 __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
+    const DecEarly &pf = sh.early;
     uint32_t j = 0;
     uint32_t cur = 0xFFFFFFFFu;
     sz_segment seg{};
@@ -299,10 +354,10 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
         const uint32_t k = find_segment(sh.segc, a.batch, t);
         if (k != cur) {
             cur = k;
-            seg = load_segment(a.batch, k);
+            seg = k == pf.k ? pf.seg : load_segment(a.batch, k);
             cap = seg.out_offset <= a.in_cap ? a.in_cap - seg.out_offset : 0;
             c = a.in + seg.out_offset;
-            h = read_header(c, cap, seg.n_elems);
+            h = k == pf.k ? pf.h : read_header(c, cap, seg.n_elems);
             tma_ok = (seg.n_elems % 16) == 0;  // code and position streams 16-byte aligned
             if (!h.ok) set_status(a.status + k, h.misaligned ? SZ_ERR_ALIGN : SZ_ERR_CORRUPT);
         }
@@ -375,15 +430,18 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                     bytes += (uint32_t)(p1 - p0) + (uint32_t)(r1 - r0);
                 }
             }
+            const bool early = j < pf.n;  // sm + codes copied before the wait (then tma holds)
             if (tma) {
                 f |= kDFlagInSmem;
-                bytes += kSub + kSub / 2;
+                if (!early) bytes += kSub + kSub / 2;
             }
             m.flags = f;
             if (bytes) {
                 mbar_arrive_expect_tx(&sh.full[s], bytes);
-                tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
-                tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
+                if (!early) {
+                    tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
+                    tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
+                }
                 if (f & kDFlagEscSmem) {
                     tma_load_1d(sh.pos[s], c + p0, (uint32_t)(p1 - p0), &sh.full[s]);
                     tma_load_1d(sh.raw[s], c + r0, (uint32_t)(r1 - r0), &sh.full[s]);
@@ -542,8 +600,9 @@ __global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArg
         }
         fence_mbar_init();
     }
+    seg_cache_fill(sh.segc, a.batch);  // all threads (the caller's table); ends with __syncthreads
+    if (tid == kThreads) decode_prefetch<kBatched>(a, sh);
     grid_dependency_wait();  // the index kernel before it has finished
-    seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
     if (tid >= kThreads) {
         if (tid == kThreads) decode_producer<kBatched>(a, sh);
     } else {

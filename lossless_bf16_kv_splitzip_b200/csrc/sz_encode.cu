@@ -140,8 +140,38 @@ __device__ __forceinline__ void read_chunk_global(const uint16_t *p, uint32_t cn
 }
 
 // ------------------------------------------------------------ producer
+// Before the grid dependency wait: the bulk copies of the CTA's first
+// kEncStages sub-tiles, which need only the caller's input and the batch
+// geometry, not what the kernel before this one writes (codebooks, escape
+// counts) -- the copies then overlap that kernel's end.  Stops at the first
+// sub-tile that is short or misaligned.  Returns how many leading sub-tiles
+// were issued: their stages have the transaction count set, and the
+// producer arrives on them once their descriptions are written.  The input
+// is complete here: the kernel before this one in the stream started only
+// after the input's writers finished (it is a plain launch or a memset).
+template <bool kBatched>
+__device__ uint32_t encode_prefetch(const EncodeArgs &a, EncShared &sh) {
+    if ((a.debug_flags & kDebugNoSignal) != 0) return 0;
+    const uint64_t t_begin = (uint64_t)blockIdx.x * a.range_tiles;
+    const uint64_t t_end = umin64(t_begin + a.range_tiles, a.batch.n_tiles);
+    uint32_t j = 0;
+    for (uint64_t t = t_begin; t < t_end && j < (uint32_t)kEncStages; ++t) {
+        const uint32_t k = find_segment(sh.segc, a.batch, t);
+        const sz_segment seg = load_segment(a.batch, k);
+        const TileRef r = resolve_tile(a.batch, seg, k, t);
+        const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
+        if ((reinterpret_cast<uintptr_t>(src) & 15) != 0) return j;
+        for (uint32_t sub = 0; sub < r.n_subs && j < (uint32_t)kEncStages; ++sub, ++j) {
+            if (r.len - sub * kSub < kSub) return j;
+            mbar_expect_tx(&sh.full[j], kSub * 2);
+            tma_load_1d(sh.stage[j], src + sub * kSub, kSub * 2, &sh.full[j]);
+        }
+    }
+    return j;
+}
+
 template <bool kBatched, bool kOnePass>
-__device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
+__device__ void encode_producer(const EncodeArgs &a, EncShared &sh, uint32_t n_early) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
     const uint64_t t_begin = (uint64_t)blockIdx.x * a.range_tiles;
     const uint64_t t_end = umin64(t_begin + a.range_tiles, a.batch.n_tiles);
@@ -189,8 +219,17 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
                 p_count = (uint32_t)e_total;
             }
         }
-        if (!seg_ok) continue;  // every tile of the segment is skipped
         const TileRef r = resolve_tile(a.batch, seg, k, t);
+        if (!seg_ok) {  // every tile of the segment is skipped
+            // sub-tiles of it copied before the wait go out as empty ones
+            for (uint32_t sub = 0; sub < r.n_subs && j < n_early; ++sub, ++j) {
+                EncMeta &m = sh.meta[j % kEncStages];
+                m = EncMeta{};
+                m.seg = k;
+                mbar_arrive(&sh.full[j % kEncStages]);
+            }
+            continue;
+        }
         const uint16_t *src = kBatched ? a.pages[seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
         const bool aligned = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
         if (!aligned) set_status(a.status + k, SZ_ERR_ALIGN);
@@ -228,7 +267,9 @@ __device__ void encode_producer(const EncodeArgs &a, EncShared &sh) {
             const bool tma = m.len == kSub;
             if (tma) f |= kFlagInSmem;
             m.flags = f;
-            if (tma) {
+            if (j < n_early) {  // copied before the wait (same source, a full sub-tile)
+                mbar_arrive(&sh.full[s]);
+            } else if (tma) {
                 mbar_arrive_expect_tx(&sh.full[s], kSub * 2);
                 tma_load_1d(sh.stage[s], m.src, kSub * 2, &sh.full[s]);
             } else {
@@ -599,8 +640,10 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
         }
         fence_mbar_init();
     }
-    grid_dependency_wait();  // the histogram kernel before it has finished
-    seg_cache_fill(sh.segc, a.batch);  // all threads; ends with __syncthreads
+    seg_cache_fill(sh.segc, a.batch);  // all threads (the caller's table); ends with __syncthreads
+    uint32_t n_early = 0;
+    if (tid == kThreads) n_early = encode_prefetch<kBatched>(a, sh);
+    grid_dependency_wait();  // the kernel before it (histogram, select) has finished
 
     // Segments with no elements have no tiles: CTA 0 writes their header
     // (one-pass: the escape placement does).
@@ -630,7 +673,7 @@ __global__ void __launch_bounds__(kPipeThreads, 3) encode_kernel(const EncodeArg
     }
 
     if (tid >= kThreads) {
-        if (tid == kThreads) encode_producer<kBatched, kOnePass>(a, sh);
+        if (tid == kThreads) encode_producer<kBatched, kOnePass>(a, sh, n_early);
     } else {
         encode_consumers<kBatched, kOnePass>(a, sh);
     }

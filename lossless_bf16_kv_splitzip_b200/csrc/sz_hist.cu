@@ -117,6 +117,7 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
 
     // ---- the segment's pieces: one per range it reaches
     const uint64_t R = a.range_tiles;
+    const uint64_t G = range_count(a.batch.n_tiles, R);
     const uint64_t t_first = seg.tile_begin;
     const uint64_t t_last = t_first + seg_tiles(a.batch, n) - 1;
     const uint64_t b_first = t_first / R, b_last = t_last / R;
@@ -137,10 +138,9 @@ __device__ void select_segment(const SelectCtx &a, uint32_t k, const uint8_t *co
         if (b <= b_last) {
             const uint64_t ps = umax64(t_first, b * R), pe = umin64(t_last + 1, (b + 1) * R);
             opens = ps == b * R;
-            const uint32_t *H = a.rhist + (b * 2 + (opens ? 0 : 1)) * 256;
             uint64_t in = 0;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) in += __ldcg(H + cbq[q]);
+            for (int q = 0; q < 16; ++q) in += __ldcg(a.rhist + rhist_at(G, opens ? 0u : 1u, cbq[q], b));
             const TileRef r0 = resolve_tile(a.batch, seg, k, ps);
             const TileRef r1 = resolve_tile(a.batch, seg, k, pe - 1);
             const uint64_t len = r1.elem0 + r1.len - r0.elem0;
@@ -282,8 +282,8 @@ __device__ __forceinline__ void count_range(const HistArgs &a, uint32_t *s_hist,
             __syncthreads();  // folds done before the next piece's counts land
             continue;
         }
-        if (ps == t_begin) a.rhist[(blockIdx.x * 2ull) * 256 + tid] = acc;
-        else if (pe == t_end) a.rhist[(blockIdx.x * 2ull + 1) * 256 + tid] = acc;
+        if (ps == t_begin) a.rhist[rhist_at(gridDim.x, 0, tid, blockIdx.x)] = acc;
+        else if (pe == t_end) a.rhist[rhist_at(gridDim.x, 1, tid, blockIdx.x)] = acc;
         if (acc) atomicAdd(&a.seg_hist[(size_t)k * 256 + tid], acc);
         __threadfence();
         __syncthreads();  // folds done before the next piece's counts land

@@ -382,6 +382,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// Raise the transaction count of the current phase by `bytes` without
+// arriving (the phase still waits for its arrivals).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -418,7 +424,7 @@ __device__ __forceinline__ void tma_load_1d(void *smem_dst, const void *gmem_src
 struct SelectCtx {
     Batch batch;
     const uint32_t *seg_hist;  // [n_segs][256]
-    const uint32_t *rhist;     // [ranges][2][256]: first, last piece of each range
+    const uint32_t *rhist;     // [2][256][ranges]: first, last piece of each range (rhist_at)
     SegMeta *meta;             // [n_segs]
     RangeRec *rrec;            // [ranges]
     uint64_t range_tiles;      // tiles per range
@@ -426,13 +432,23 @@ struct SelectCtx {
     uint32_t *hist_out;        // optional [256] (single only)
 };
 
+// Ranges of a call, and the index of the count of exponent x in the first
+// (which = 0) or last (1) piece of range b: range-minor, so that the select
+// reads one exponent's counts of consecutive ranges as consecutive words.
+__host__ __device__ inline uint64_t range_count(uint64_t n_tiles, uint64_t range_tiles) {
+    return n_tiles ? (n_tiles + range_tiles - 1) / range_tiles : 1;
+}
+__host__ __device__ inline uint64_t rhist_at(uint64_t ranges, uint32_t which, uint32_t x, uint64_t b) {
+    return ((uint64_t)which * 256 + x) * ranges + b;
+}
+
 struct HistArgs {
     SelectCtx sel;
     const uint16_t *const *pages;  // batched: page pointers
     const uint16_t *base;          // single-tensor input
     uint32_t *seg_hist;            // [n_segs][256], zero on entry
     uint32_t *seg_done;            // [n_segs] tiles counted so far, zero on entry
-    uint32_t *rhist;               // [ranges][2][256]
+    uint32_t *rhist;               // [2][256][ranges] (rhist_at)
     int32_t *status;               // [n_segs] or nullptr
     uint32_t *accum;               // accumulate mode: caller histograms [rows][256] (else nullptr)
     const uint32_t *accum_index;   // accumulate mode: row of segment k (nullptr: row k)
@@ -548,7 +564,7 @@ struct CompressScratch {
     uint32_t *seg_done;  // [1]
     uint32_t *enc_done;  // [1]
     SegMeta *meta;       // [1]
-    uint32_t *rhist;     // [ranges][2][256]
+    uint32_t *rhist;     // [2][256][ranges] (rhist_at)
     RangeRec *rrec;      // [ranges]
 };
 // Histogram kernel (with the select) and encode kernel of d_in[0..n): the
