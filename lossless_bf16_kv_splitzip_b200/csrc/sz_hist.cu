@@ -380,14 +380,20 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const uint32_t *hists,
 template <bool kAccum>
 void launch_hist_t(const HistArgs &a, bool batched, int grid, size_t smem, cudaStream_t s) {
     const bool small = a.sel.batch.page_elems <= kSub || a.sel.batch.tile_elems <= kSub;
-    if (batched && small)
+    // 65,536-element tiles: as many blocks per SM as the shared memory holds
+    // (measured 0.735 -> 0.705 ms on the 64-tensor batch); the one-sub-tile
+    // build keeps its 3 blocks per SM and the driver's carveout.
+    if (batched && small) {
         hist_kernel<true, true, kAccum><<<grid, kThreads, smem, s>>>(a);
-    else if (batched)
+    } else if (batched) {
+        prefer_max_shared<hist_kernel<true, false, kAccum>>();
         hist_kernel<true, false, kAccum><<<grid, kThreads, smem, s>>>(a);
-    else if (small)
+    } else if (small) {
         hist_kernel<false, true, kAccum><<<grid, kThreads, smem, s>>>(a);
-    else
+    } else {
+        prefer_max_shared<hist_kernel<false, false, kAccum>>();
         hist_kernel<false, false, kAccum><<<grid, kThreads, smem, s>>>(a);
+    }
 }
 
 // a.accum set: the accumulate mode

@@ -7,6 +7,7 @@
 // documented in include/splitzip.h.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -311,6 +312,26 @@ __device__ __forceinline__ void consumer_sync() {
 // next launch_after() kernel start early.
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Ask, once per device, for the largest shared-memory carveout for
+// `Kernel`: an SM then keeps room for blocks of a big-shared-memory kernel
+// next to this one's (the decode kernel starting while the index kernel
+// still runs), and a kernel whose blocks each take a slice of the shared
+// memory gets as many of them on an SM as its other limits allow.  Best
+// effort: a refusal leaves the driver's choice.
+template <auto Kernel>
+void prefer_max_shared() {
+    static std::atomic<uint64_t> done{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_relaxed) & bit) return;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess)
+        done.fetch_or(bit, std::memory_order_relaxed);
+    else
+        (void)cudaGetLastError();
+}
 
 template <typename... Params, typename... Args>
 cudaError_t launch_after(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
