@@ -305,10 +305,12 @@ __device__ __forceinline__ void count_range(const HistArgs &a, uint32_t *s_hist,
 // sub-tile (pages of at most 16,384 elements, or the one-sub-tile tiles of
 // a short single stream); that build is given registers for 3 blocks per
 // SM -- measured 0.70 -> 0.86 of the copy bandwidth on 16-token pages,
-// while the same bound costs 8 % on 65,536-element tiles, which keep the
-// default build.
+// while the same bound costs 8 % on 65,536-element tiles.  Those get a
+// bound of 5 blocks per SM (at most 51 registers; unbounded, the compiler
+// chose 32 and spilled): 0.706 -> 0.680 ms on the 64-tensor batch, with the
+// largest shared-memory carveout holding 5 blocks.
 template <bool kBatched, bool kSmallTiles, bool kAccum>
-__global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 0) hist_kernel(const HistArgs a) {
+__global__ void __launch_bounds__(kThreads, kSmallTiles ? 3 : 5) hist_kernel(const HistArgs a) {
     extern __shared__ __align__(128) uint32_t s_hist[];  // kHistWords
     __shared__ SegCache s_segc;
     __shared__ SelShared s_sel;
