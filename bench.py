@@ -413,6 +413,30 @@ def run_sweep(args):
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     peak, peak_kind = measured_peak()
     stream = torch.cuda.Stream(dev)
+    # The frame every number below sits in: the same events around an empty
+    # graph, and around a graph of one tiny kernel (a 4-element add), after
+    # the same flush.
+    tiny = torch.zeros(4, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(stream):
+        g_one = torch.cuda.CUDAGraph()
+        tiny.add_(1)
+        with torch.cuda.graph(g_one, stream=stream):
+            tiny.add_(1)
+        t0, t1 = [], []
+        for _ in range(3 + args.sweep_reps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.fill_(1)
+            ev[0].record(stream); ev[1].record(stream)
+            flush.fill_(2)
+            ev[2].record(stream); g_one.replay(); ev[3].record(stream)
+            stream.synchronize()
+            t0.append(ev[0].elapsed_time(ev[1]) / 1e3)
+            t1.append(ev[2].elapsed_time(ev[3]) / 1e3)
+        del g_one
+    print(json.dumps({"sweep_frame": "events after the flush, nothing between / one tiny kernel graph",
+                      "empty_us": round(float(np.median(t0[3:])) * 1e6, 2),
+                      "one_kernel_us": round(float(np.median(t1[3:])) * 1e6, 2), "reps": args.sweep_reps}),
+          flush=True)
     for b in sizes_b:
         n = b // 2
         x = d_flat[:n]

@@ -382,18 +382,20 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const uint32_t *hists,
 template <bool kAccum>
 void launch_hist_t(const HistArgs &a, bool batched, int grid, size_t smem, cudaStream_t s) {
     const bool small = a.sel.batch.page_elems <= kSub || a.sel.batch.tile_elems <= kSub;
-    // 65,536-element tiles: as many blocks per SM as the shared memory holds
-    // (measured 0.735 -> 0.705 ms on the 64-tensor batch); the one-sub-tile
-    // build keeps its 3 blocks per SM and the driver's carveout.
+    // 65,536-element tiles: the largest shared-memory carveout (64-tensor
+    // batch right after a decode: 0.734 -> 0.678 ms; back to back with no
+    // other kernel between it is 0.619 -> 0.671 ms, the cost of the smaller
+    // L1).  The accumulate mode keeps the driver's carveout (0.115 -> 0.099
+    // ms per 512 MiB prefill chunk), and so does the one-sub-tile build.
     if (batched && small) {
         hist_kernel<true, true, kAccum><<<grid, kThreads, smem, s>>>(a);
     } else if (batched) {
-        prefer_max_shared<hist_kernel<true, false, kAccum>>();
+        if (!kAccum) prefer_max_shared<hist_kernel<true, false, kAccum>>();
         hist_kernel<true, false, kAccum><<<grid, kThreads, smem, s>>>(a);
     } else if (small) {
         hist_kernel<false, true, kAccum><<<grid, kThreads, smem, s>>>(a);
     } else {
-        prefer_max_shared<hist_kernel<false, false, kAccum>>();
+        if (!kAccum) prefer_max_shared<hist_kernel<false, false, kAccum>>();
         hist_kernel<false, false, kAccum><<<grid, kThreads, smem, s>>>(a);
     }
 }
