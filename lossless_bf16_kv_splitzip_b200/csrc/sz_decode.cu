@@ -231,7 +231,8 @@ constexpr uint32_t kEscCap = 1024;  // escape records bulk-copied per sub-tile; 
 constexpr uint32_t kDFlagEnd = 1u;
 constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
 constexpr uint32_t kDFlagTileEnd = 4u;  // last sub-tile of its tile
-constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage
+constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage (DecEscMeta)
+constexpr uint32_t kDFlagEarly = 16u;   // described and copied before the grid dependency wait
 
 // What the producer read and copied before the grid dependency wait.
 struct DecEarly {
@@ -241,6 +242,10 @@ struct DecEarly {
     Header h;
 };
 
+// A stage's description in two parts, each published by its own arrival:
+// the values part (full[s]) needs only the container, the escape part
+// (escs[s]) needs the index kernel's sub-tile starts, so the consumers
+// decode and store a stage's values while the index may still be running.
 struct DecMeta {
     uint16_t *dst;      // global destination of the sub-tile's first element
     const uint8_t *c;   // the segment's container
@@ -248,10 +253,13 @@ struct DecMeta {
     uint64_t n, e;
     uint64_t cb_lo, cb_hi;
     uint64_t tile;      // global tile of the sub-tile
-    uint32_t seg, len, flags, lo, cnt;
+    uint32_t seg, len, flags, pad;
+};
+struct DecEscMeta {
+    uint32_t lo, cnt;   // the sub-tile's escape records [lo, lo + cnt)
     uint32_t pos_skew;  // byte offset of record lo's position inside the staged copy
     uint32_t raw_skew;  // byte offset of record lo's exponent inside the staged copy
-    uint32_t pad;
+    uint32_t flags;     // kDFlagEscSmem
 };
 
 struct __align__(128) DecShared {
@@ -260,11 +268,14 @@ struct __align__(128) DecShared {
     uint8_t pos[kDecStages][4 * kEscCap + 32];  // 16-byte aligned superset of the positions
     uint8_t raw[kDecStages][kEscCap + 32];      // 16-byte aligned superset of the exponents
     DecMeta meta[kDecStages];
-    uint64_t full[kDecStages];
+    DecEscMeta emeta[kDecStages];
+    uint64_t full[kDecStages];   // values part: sm + codes arrived, meta written
+    uint64_t escs[kDecStages];   // escape part: records arrived, emeta written
     uint64_t empty[kDecStages];
     SegCache segc;
     DecEarly early;  // producer only: what it read and copied before the grid dependency wait
     int go[2];  // stage j's data arrived (slot j & 1)
+    int eok;    // the current stage's escape part arrived
 };
 
 // Tiles are dealt round robin in groups of about kTile elements: one tile
@@ -294,14 +305,14 @@ __device__ void decode_timeout_from(const DecodeArgs &a, const SegCache &c, uint
 
 // ------------------------------------------------------------ producer
 // Before the grid dependency wait (the index kernel's end): the header of
-// the CTA's first segment and the sm + code copies of its first kDecStages
-// sub-tiles -- what the containers alone give, not the index entries or
-// status words the index kernel writes.  The containers are complete here:
-// the index kernel lets this kernel start only after its own wait for the
-// kernel that wrote them.  Stops at the first sub-tile that is short, in
-// another segment, or whose header or alignment rules out bulk copies; the
-// issued stages have their transaction count set, and the producer arrives
-// on them after the wait.  Sets no status (the index kernel writes it).
+// the CTA's first segment and the values part of its first kDecStages
+// sub-tiles (description, sm + code copies, arrival) -- what the containers
+// alone give, not the index entries or status words the index kernel
+// writes; the consumers start on those values at once.  The containers are
+// complete here: the index kernel lets this kernel start only after its own
+// wait for the kernel that wrote them.  Stops at the first sub-tile that is
+// short, in another segment, or whose header or alignment rules out bulk
+// copies.  Sets no status (the index kernel writes it).
 template <bool kBatched>
 __device__ void decode_prefetch(const DecodeArgs &a, DecShared &sh) {
     DecEarly &p = sh.early;  // the producer thread's own (shared memory: no registers held over the wait)
@@ -322,10 +333,24 @@ __device__ void decode_prefetch(const DecodeArgs &a, DecShared &sh) {
         if (!p.h.ok || (p.seg.n_elems % 16) != 0) return;
         const TileRef r = resolve_tile(a.batch, p.seg, k, t);
         const uint8_t *c = a.in + p.seg.out_offset;
+        uint16_t *dst = kBatched ? a.pages[p.seg.page_begin + r.page] + r.in_page : a.base + r.elem0;
+        if ((reinterpret_cast<uintptr_t>(dst) & 15) != 0) return;
         for (uint32_t sub = 0; sub < r.n_subs && p.n < (uint32_t)kDecStages; ++sub) {
             if (r.len - sub * kSub < kSub) return;
             const uint64_t elem0 = r.elem0 + (uint64_t)sub * kSub;
-            mbar_expect_tx(&sh.full[p.n], kSub + kSub / 2);
+            DecMeta &m = sh.meta[p.n];
+            m.dst = dst + sub * kSub;
+            m.c = c;
+            m.elem0 = elem0;
+            m.n = p.h.n;
+            m.e = p.h.e;
+            m.cb_lo = p.h.cb_lo;
+            m.cb_hi = p.h.cb_hi;
+            m.tile = t;
+            m.seg = k;
+            m.len = kSub;
+            m.flags = kDFlagInSmem | kDFlagEarly | (sub + 1 == r.n_subs ? kDFlagTileEnd : 0u);
+            mbar_arrive_expect_tx(&sh.full[p.n], kSub + kSub / 2);
             tma_load_1d(sh.sm[p.n], c + kHeader + elem0, kSub, &sh.full[p.n]);
             tma_load_1d(sh.codes[p.n], c + kHeader + p.h.n + elem0 / 2, kSub / 2, &sh.full[p.n]);
             ++p.n;
@@ -333,11 +358,12 @@ __device__ void decode_prefetch(const DecodeArgs &a, DecShared &sh) {
     }
 }
 
-// One thread: per sub-tile, wait for the stage to be free, then bulk-copy
-// the sm bytes, the codes and (when they fit and stay inside the buffer) a
-// 16-byte aligned superset of the sub-tile's escape positions and exponents
-// (the first sh.early.n sub-tiles: only the escape records, the rest was
-// copied before the wait).
+// One thread: per sub-tile, wait for the stage to be free, then publish
+// its values part (description; sm bytes and codes by bulk copy) on
+// full[s] and its escape part (record range; when they fit and stay inside
+// the buffer, a 16-byte aligned superset of its escape positions and
+// exponents by bulk copy) on escs[s] -- for the first sh.early.n sub-tiles
+// only the escape part, the values part went out before the wait.
 template <bool kBatched>
 __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
     if ((a.debug_flags & kDebugNoSignal) != 0) return;  // test hook: nothing is ever signalled
@@ -400,55 +426,51 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                 hi = lo = 0;
             }
             const uint32_t cnt = hi - lo;
-            DecMeta &m = sh.meta[s];
-            m.dst = dst_aligned ? dst + sub * kSub : nullptr;
-            m.c = c;
-            m.elem0 = elem0;
-            m.n = h.n;
-            m.e = h.e;
-            m.cb_lo = h.cb_lo;
-            m.cb_hi = h.cb_hi;
-            m.seg = k;
-            m.len = len;
-            m.lo = lo;
-            m.cnt = cnt;
-            m.tile = t;
             const bool tma = tma_ok && len == kSub;
-            uint32_t bytes = 0, f = sub + 1 == r.n_subs ? kDFlagTileEnd : 0u;
-            // escape records: aligned supersets [ps & ~15, ceil16(pe)) that
-            // must lie inside the caller's buffer
-            uint64_t p0 = 0, p1 = 0, r0 = 0, r1 = 0;
-            if (tma && cnt > 0 && cnt <= kEscCap) {
-                p0 = (pos_off + 4 * (uint64_t)lo) & ~15ull;
-                p1 = (pos_off + 4 * (uint64_t)hi + 15) & ~15ull;
-                r0 = (raw_off + lo) & ~15ull;
-                r1 = (raw_off + hi + 15) & ~15ull;
-                if (p1 <= cap && r1 <= cap) {
-                    f |= kDFlagEscSmem;
-                    m.pos_skew = (uint32_t)(pos_off + 4 * (uint64_t)lo - p0);
-                    m.raw_skew = (uint32_t)(raw_off + lo - r0);
-                    bytes += (uint32_t)(p1 - p0) + (uint32_t)(r1 - r0);
-                }
-            }
-            const bool early = j < pf.n;  // sm + codes copied before the wait (then tma holds)
-            if (tma) {
-                f |= kDFlagInSmem;
-                if (!early) bytes += kSub + kSub / 2;
-            }
-            m.flags = f;
-            if (bytes) {
-                mbar_arrive_expect_tx(&sh.full[s], bytes);
-                if (!early) {
+            if (j >= pf.n) {  // the values part (the first pf.n went out before the wait)
+                DecMeta &m = sh.meta[s];
+                m.dst = dst_aligned ? dst + sub * kSub : nullptr;
+                m.c = c;
+                m.elem0 = elem0;
+                m.n = h.n;
+                m.e = h.e;
+                m.cb_lo = h.cb_lo;
+                m.cb_hi = h.cb_hi;
+                m.tile = t;
+                m.seg = k;
+                m.len = len;
+                m.flags = (sub + 1 == r.n_subs ? kDFlagTileEnd : 0u) | (tma ? kDFlagInSmem : 0u);
+                if (tma) {
+                    mbar_arrive_expect_tx(&sh.full[s], kSub + kSub / 2);
                     tma_load_1d(sh.sm[s], c + kHeader + elem0, kSub, &sh.full[s]);
                     tma_load_1d(sh.codes[s], c + kHeader + h.n + elem0 / 2, kSub / 2, &sh.full[s]);
+                } else {
+                    mbar_arrive(&sh.full[s]);
                 }
-                if (f & kDFlagEscSmem) {
-                    tma_load_1d(sh.pos[s], c + p0, (uint32_t)(p1 - p0), &sh.full[s]);
-                    tma_load_1d(sh.raw[s], c + r0, (uint32_t)(r1 - r0), &sh.full[s]);
-                }
-            } else {
-                mbar_arrive(&sh.full[s]);
             }
+            // the escape part: aligned supersets [ps & ~15, ceil16(pe)) of
+            // the records, which must lie inside the caller's buffer
+            DecEscMeta &em = sh.emeta[s];
+            em.lo = lo;
+            em.cnt = cnt;
+            em.flags = 0;
+            uint32_t bytes = 0;
+            if (tma && cnt > 0 && cnt <= kEscCap) {
+                const uint64_t p0 = (pos_off + 4 * (uint64_t)lo) & ~15ull;
+                const uint64_t p1 = (pos_off + 4 * (uint64_t)hi + 15) & ~15ull;
+                const uint64_t r0 = (raw_off + lo) & ~15ull;
+                const uint64_t r1 = (raw_off + hi + 15) & ~15ull;
+                if (p1 <= cap && r1 <= cap) {
+                    em.flags = kDFlagEscSmem;
+                    em.pos_skew = (uint32_t)(pos_off + 4 * (uint64_t)lo - p0);
+                    em.raw_skew = (uint32_t)(raw_off + lo - r0);
+                    bytes = (uint32_t)(p1 - p0) + (uint32_t)(r1 - r0);
+                    mbar_arrive_expect_tx(&sh.escs[s], bytes);
+                    tma_load_1d(sh.pos[s], c + p0, (uint32_t)(p1 - p0), &sh.escs[s]);
+                    tma_load_1d(sh.raw[s], c + r0, (uint32_t)(r1 - r0), &sh.escs[s]);
+                }
+            }
+            if (!bytes) mbar_arrive(&sh.escs[s]);
         }
     }
     const int s = (int)(j % kDecStages);
@@ -515,18 +537,24 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
     // consumer has passed the barrier below when it is read)
     uint64_t next_tile = (uint64_t)blockIdx.x * tiles_per_group(a.batch);
     // One consumer barrier per sub-tile: after its values are stored, thread
-    // 0 waits for the next stage's data, then the barrier orders every store
-    // before the escape patches and hands the next stage's arrival to all.
+    // 0 waits for the stage's escape part and the next stage's values part,
+    // then the barrier orders every store before the escape patches and
+    // hands both arrivals to all.  The consumers do not wait for the index
+    // kernel before a stage described before the grid dependency wait (its
+    // values need only the container, and that path sets no status); every
+    // other status write comes after their own grid dependency wait.
     if (tid == 0) sh.go[0] = mbar_wait(&sh.full[0], 0u, a.wait_limit_ns) ? 1 : 0;
     consumer_sync();
     for (uint32_t j = 0;; ++j) {
         const int s = (int)(j % kDecStages);
         if (!sh.go[j & 1]) {  // the same decision in every consumer thread
+            grid_dependency_wait();
             if (tid == 0) decode_timeout_from(a, sh.segc, next_tile);
             return;
         }
         const DecMeta m = sh.meta[s];
         if (m.flags & kDFlagEnd) return;
+        if (!(m.flags & kDFlagEarly)) grid_dependency_wait();
         if (m.seg != cur) {
             T = make_tables(m.cb_lo, m.cb_hi);
 #pragma unroll
@@ -546,22 +574,33 @@ __device__ void decode_consumers(const DecodeArgs &a, DecShared &sh) {
         for (int q = 0; q < kChunks; ++q) decode_store_chunk(m, sh, s, T, q, tid, status);
 
         const int s_next = (int)((j + 1) % kDecStages);
-        if (tid == 0) sh.go[(j + 1) & 1] = mbar_wait(&sh.full[s_next], ((j + 1) / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
+        if (tid == 0) {
+            const bool e_ok = mbar_wait(&sh.escs[s], (j / kDecStages) & 1u, a.wait_limit_ns);
+            sh.eok = e_ok ? 1 : 0;
+            sh.go[(j + 1) & 1] =
+                e_ok && mbar_wait(&sh.full[s_next], ((j + 1) / kDecStages) & 1u, a.wait_limit_ns) ? 1 : 0;
+        }
         consumer_sync();
+        grid_dependency_wait();  // returns at once: the escape part was published after it
+        if (!sh.eok) {  // the same decision in every consumer thread
+            if (tid == 0) decode_timeout_from(a, sh.segc, next_tile);
+            return;
+        }
 
         // ---- escapes, one per thread, after every chunk store of the
         // sub-tile: check the record and overwrite its value's exponent
-        if (m.cnt) {
-            const bool es = (m.flags & kDFlagEscSmem) != 0;
+        const DecEscMeta em = sh.emeta[s];
+        if (em.cnt) {
+            const bool es = (em.flags & kDFlagEscSmem) != 0;
             const bool ss = (m.flags & kDFlagInSmem) != 0;
             const uint8_t *gpos = m.c + kHeader + m.n + (m.n + 1) / 2;
             const uint8_t *graw = gpos + 4 * m.e;
-            const uint8_t *spos = sh.pos[s] + m.pos_skew;
-            const uint8_t *sraw = sh.raw[s] + m.raw_skew;
+            const uint8_t *spos = sh.pos[s] + em.pos_skew;
+            const uint8_t *sraw = sh.raw[s] + em.raw_skew;
             const uint8_t *gsm = m.c + kHeader + m.elem0;
             const uint8_t *gcodes = m.c + kHeader + m.n;
-            for (uint32_t i = tid; i < m.cnt; i += kThreads) {
-                const uint64_t g = (uint64_t)m.lo + i;
+            for (uint32_t i = tid; i < em.cnt; i += kThreads) {
+                const uint64_t g = (uint64_t)em.lo + i;
                 const uint64_t p = es ? *reinterpret_cast<const uint32_t *>(spos + 4 * i) : load_u32_any(gpos + 4 * g);
                 const uint32_t x = es ? sraw[i] : graw[g];
                 bool bad = p < m.elem0 || p - m.elem0 >= m.len || in_set8(cbset, x);
@@ -596,17 +635,20 @@ __global__ void __launch_bounds__(kPipeThreads, 3) decode_kernel(const DecodeArg
     if (tid == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.escs[s], 1);
             mbar_init(&sh.empty[s], kWarps);
         }
         fence_mbar_init();
     }
     seg_cache_fill(sh.segc, a.batch);  // all threads (the caller's table); ends with __syncthreads
-    if (tid == kThreads) decode_prefetch<kBatched>(a, sh);
-    grid_dependency_wait();  // the index kernel before it has finished
     if (tid >= kThreads) {
-        if (tid == kThreads) decode_producer<kBatched>(a, sh);
+        if (tid == kThreads) {
+            decode_prefetch<kBatched>(a, sh);
+            grid_dependency_wait();  // the index kernel before it has finished
+            decode_producer<kBatched>(a, sh);
+        }
     } else {
-        decode_consumers<kBatched>(a, sh);
+        decode_consumers<kBatched>(a, sh);  // waits for the index kernel itself, where it must
     }
 }
 
