@@ -161,7 +161,7 @@ sz_status sz_encode(const uint16_t *d_in, uint64_t n, const uint8_t *d_codebook1
 /*
  * sz_compress -- histogram, codebook and container of d_in[0..n) in one call
  * (sz_histogram_codebook + sz_encode with the codebook chosen there).  A
- * stream of at most 2^21 elements is compressed by blocks of 4,096
+ * stream of at most 2^20 elements is compressed by blocks of 4,096
  * elements in two launches after one memset; a longer one by the
  * histogram kernel and the encode kernel.
  *   d_out, out_cap  container buffer, 16-byte aligned; out_cap at least
@@ -193,9 +193,9 @@ sz_status sz_compress(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t
  *                   d_out holds no meaningful data unless it reads SZ_OK.
  *   d_ws, ws_bytes  workspace of sz_plan's size (the first escape index of
  *                   every 16,384-element sub-tile, found by binary search).
- * A stream of at most 2^21 elements is decoded by blocks of 4,096 elements
+ * A stream of at most 2^17 elements is decoded by blocks of 4,096 elements
  * in one launch after the status memset (no index kernel), with the same
- * checks.
+ * checks; a longer one by the index kernel and the pipelined decode.
  */
 sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uint64_t n,
                     int32_t *d_status, void *d_ws, uint64_t ws_bytes, void *stream);

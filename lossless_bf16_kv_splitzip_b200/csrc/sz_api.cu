@@ -29,8 +29,8 @@ namespace {
 
 constexpr uint64_t kMaxElems = 0xFFFFFFFFull;  // largest n: positions are u32, n < 2^32
 constexpr uint64_t kAlign = 256;
-constexpr uint64_t kSmallEncodeMax = 1ull << 21;  // sz_compress: 4,096-element blocks up to this many elements (measured crossover 4-8 MiB)
-constexpr uint64_t kSmallDecodeMax = 1ull << 21;  // sz_decode: one launch of 4,096-element blocks up to this (measured crossover 4-8 MiB)
+constexpr uint64_t kSmallEncodeMax = 1ull << 20;  // sz_compress: 4,096-element blocks up to this many elements (measured crossover 2-4 MiB)
+constexpr uint64_t kSmallDecodeMax = 1ull << 17;  // sz_decode: one launch of 4,096-element blocks up to this (measured crossover 256-512 KiB)
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
 std::atomic<uint32_t> g_debug_flags{0};

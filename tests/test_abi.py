@@ -58,7 +58,7 @@ def test_plan_worst_case_bound(n):
     # escape starts
     need = 1024 + 4 + 4 + 32 + 2048 * ranges + 16 * ranges + 4 * ((tile // 16384) * tiles + 1)
     assert need <= ws
-    if n <= 1 << 21:  # also the one-call compression's scratch: counts of every 4,096-element slice
+    if n <= 1 << 20:  # also the one-call compression's scratch: counts of every 4,096-element slice
         nb = max(1, -(-n // 4096))
         small = -(-(-(-(1536 + 4 * nb) // 256) * 256 + 1024 * nb) // 256) * 256
         assert small <= ws <= max(small, need + 6 * 256)

@@ -29,7 +29,9 @@ if not torch.cuda.is_available():  # pragma: no cover
 
 H = 48
 DEV = "cuda:0"
-SHORT = 1 << 21  # streams up to this many elements take the short-stream encode / decode
+SHORT_ENC = 1 << 20  # sz_compress: streams up to this many elements take the short-stream encode
+SHORT_DEC = 1 << 17  # sz_decode: streams up to this many elements take the short-stream decode
+SHORT = 1 << 21  # past both limits
 
 
 def to_dev(x_np):
@@ -311,7 +313,8 @@ def corruptions(blob, n):
 
 # short streams take the one-launch decode, longer ones the index +
 # pipelined decode: both must reject every corruption
-@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11, 65536 + 3001, SHORT + 3001, SHORT + 16 * 17])
+@pytest.mark.parametrize("n", [3001, 40000, 3 * 16384 + 11, 65536 + 3001, SHORT_DEC, SHORT_DEC + 3001,
+                               SHORT + 3001, SHORT + 16 * 17])
 def test_corrupt_containers_rejected(n):
     x = kvgen.mixed_small(n, seed=21 + n)
     blob = gpu_encode(x)
@@ -336,7 +339,8 @@ def test_odd_tail_nibble_rejected():
 
 
 # -------------------------------------------------- one-call compression
-@pytest.mark.parametrize("n", [0, 1, 17, 4095, 4096, 4097, 32769, 65537, 3 * 65536 + 100, SHORT, SHORT + 1,
+@pytest.mark.parametrize("n", [0, 1, 17, 4095, 4096, 4097, 32769, 65537, 3 * 65536 + 100, SHORT_ENC,
+                               SHORT_ENC + 1, SHORT, SHORT + 1,
                                (1 << 23) + 7, (1 << 25) + 12345, (1 << 26) + 33, (1 << 27) - 5, (1 << 27) + 16])
 def test_compress_one_call_equals_oracle(n):
     """sz_compress: short streams by 4,096-element blocks in two launches,
