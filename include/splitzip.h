@@ -447,7 +447,10 @@ sz_status sz_set_wait_limit_ns(uint64_t limit_ns);
  * sz_debug_set_flags -- test hook.  Bit 0: the encode and decode kernels'
  * copy threads issue no bulk copy, so every stage wait of their consumer
  * threads runs out (exercises the timeout path without faulting
- * anything).  0 restores normal operation.
+ * anything).  Bit 1: the decode kernel's copy thread publishes the values
+ * part of its stages but never their escape part, so the consumers' wait
+ * for escape records runs out after the values are stored.  0 restores
+ * normal operation.
  */
 sz_status sz_debug_set_flags(uint32_t flags);
 

@@ -233,6 +233,7 @@ constexpr uint32_t kDFlagInSmem = 2u;   // sm + codes came by TMA into the stage
 constexpr uint32_t kDFlagTileEnd = 4u;  // last sub-tile of its tile
 constexpr uint32_t kDFlagEscSmem = 8u;  // the escape records came by TMA into the stage (DecEscMeta)
 constexpr uint32_t kDFlagEarly = 16u;   // described and copied before the grid dependency wait
+constexpr uint32_t kDebugNoEscapeSignal = 2u;  // test hook: the producer publishes values parts only
 
 // What the producer read and copied before the grid dependency wait.
 struct DecEarly {
@@ -448,6 +449,8 @@ __device__ void decode_producer(const DecodeArgs &a, DecShared &sh) {
                     mbar_arrive(&sh.full[s]);
                 }
             }
+            // test hook: the escape parts are never published
+            if ((a.debug_flags & kDebugNoEscapeSignal) != 0) return;
             // the escape part: aligned supersets [ps & ~15, ceil16(pe)) of
             // the records, which must lie inside the caller's buffer
             DecEscMeta &em = sh.emeta[s];

@@ -468,6 +468,50 @@ def test_compress_wait_times_out_cleanly(n):
     assert out[: int(size.item())].cpu().numpy().tobytes() == oracle.encode(x)
 
 
+def test_decode_escape_wait_times_out_cleanly():
+    """The decode's values are stored before the index is ready; a wait for
+    a stage's escape part that runs out (bit 1: only values parts are ever
+    published) gives SZ_ERR_DEVICE_TIMEOUT for the stream and for every
+    segment of a batch, and the next call is bit-exact."""
+    x = kvgen.mixed_small(SHORT + 5, seed=33)
+    blob = oracle.encode(x)
+    c = torch.from_numpy(np.frombuffer(blob, np.uint8).copy()).to(DEV)
+    lens = [300000, 5 * 65536 + 11, 65536]
+    streams = [kvgen.mixed_small(m, seed=40 + i) for i, m in enumerate(lens)]
+    starts = [0]
+    for m in lens[:-1]:
+        starts.append(starts[-1] + -(-m // 64) * 64)  # 16-byte aligned pages
+    flat = np.zeros(starts[-1] + lens[-1], np.uint16)
+    for s_, x_ in zip(starts, streams):
+        flat[s_: s_ + x_.size] = x_
+    pool = torch.from_numpy(flat.view(np.int16)).to(DEV)
+    plan = sz.BatchPlan(lens, max(lens), device=DEV)
+    ptrs = torch.from_numpy((np.array(starts) * 2 + pool.data_ptr()).astype(np.int64)).to(DEV)
+    plan.encode(ptrs)
+    torch.cuda.synchronize()
+    assert plan.enc_status.abs().sum().item() == 0
+    dst = torch.zeros_like(pool)
+    dptrs = torch.from_numpy((np.array(starts) * 2 + dst.data_ptr()).astype(np.int64)).to(DEV)
+    try:
+        sz.sz_set_wait_limit_ns(2_000_000)
+        sz.sz_debug_set_flags(2)
+        _, status = sz.decode(c, x.size)
+        plan.decode(dptrs)
+        torch.cuda.synchronize()
+        assert int(status.item()) == sz.SZ_ERR_DEVICE_TIMEOUT
+        assert all(int(v) == sz.SZ_ERR_DEVICE_TIMEOUT for v in plan.dec_status.cpu().tolist())
+    finally:
+        sz.sz_debug_set_flags(0)
+        sz.sz_set_wait_limit_ns(1_000_000_000)
+    y, status = sz.decode(c, x.size)
+    plan.decode(dptrs)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert np.array_equal(y.cpu().numpy().view(np.uint16), x)
+    assert plan.dec_status.abs().sum().item() == 0
+    assert torch.equal(dst, pool)
+
+
 def test_decode_stage_wait_times_out_cleanly():
     x = kvgen.mixed_small(SHORT + 5, seed=32)  # the pipelined decode (it has the waits)
     blob = oracle.encode(x)
