@@ -19,7 +19,7 @@ cudaError_t launch_small_encode(const uint16_t *in, uint64_t n, const SmallWs &w
 cudaError_t launch_small_decode(const uint8_t *c, uint64_t cap, uint16_t *out, uint64_t n, int32_t *status,
                                 cudaStream_t s);
 cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s);
-cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs &a, bool batched, int grid, int sms, cudaStream_t s);
 int decode_blocks_per_sm();
 }  // namespace sz
 
@@ -382,7 +382,7 @@ sz_status sz_decode(const uint8_t *d_in, uint64_t in_bytes, uint16_t *d_out, uin
     a.wait_limit_ns = wait_limit_ns();
     a.debug_flags = debug_flags();
     SZ_TRY_CUDA(launch_esc_index(a, false, s));
-    return cuda_status(launch_decode(a, false, dev.sms * dev.dec_occ, s));
+    return cuda_status(launch_decode(a, false, dev.sms * dev.dec_occ, dev.sms, s));
 }
 
 sz_status sz_compress(const uint16_t *d_in, uint64_t n, uint8_t *d_out, uint64_t out_cap, uint64_t *d_out_bytes,
@@ -527,7 +527,7 @@ sz_status sz_decode_batched(uint32_t n_segs, const sz_segment *d_segs, uint64_t 
     a.wait_limit_ns = wait_limit_ns();
     a.debug_flags = debug_flags();
     SZ_TRY_CUDA(launch_esc_index(a, true, s));
-    return cuda_status(launch_decode(a, true, dev.sms * dev.dec_occ, s));
+    return cuda_status(launch_decode(a, true, dev.sms * dev.dec_occ, dev.sms, s));
 }
 
 sz_status sz_plan_one_pass(uint64_t n_elems, uint64_t *max_compressed_bytes, uint64_t *workspace_bytes) {

@@ -783,12 +783,25 @@ cudaError_t launch_esc_index(const DecodeArgs &a, bool batched, cudaStream_t s) 
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs &a0, bool batched, int grid, int sms, cudaStream_t s) {
     DecodeArgs a = a0;
     if (a.batch.n_tiles == 0) return cudaSuccess;
     const size_t smem = sizeof(DecShared);
+    const uint64_t groups = div_up(a.batch.n_tiles, tiles_per_group(a.batch));
+    // A short index kernel (its warp build) holds one SM slot of this kernel
+    // per block while it runs.  When the CTAs left beside it take at most
+    // 1.5 groups each on average, leaving those slots out lets every CTA
+    // start at once and copy its first stages while the index runs (16 MiB
+    // stream: 20.5 -> 18.4 us, no CTA starting after the index's end instead
+    // of 64; at 20 MiB, 1.76 groups each, it was no better).
+    const uint64_t entries = (uint64_t)a.batch.tile_subs * a.batch.n_tiles + (batched ? a.batch.n_segs : 1u);
+    if (entries <= kWarpIndexMax) {
+        const uint64_t index_blocks = div_up(entries, 256 / 32);
+        const uint64_t beside = umax64((uint64_t)sms, (uint64_t)grid > index_blocks ? (uint64_t)grid - index_blocks : 0);
+        if (2 * groups <= 3 * beside) grid = (int)umin64((uint64_t)grid, beside);
+    }
     // groups of tiles are dealt round robin: CTA b decodes groups b, b + grid, ...
-    grid = (int)umax64(1, umin64((uint64_t)grid, div_up(a.batch.n_tiles, tiles_per_group(a.batch))));
+    grid = (int)umax64(1, umin64((uint64_t)grid, groups));
     cudaError_t e;
     if (batched) {
         e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
