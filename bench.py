@@ -492,6 +492,78 @@ def run_sweep(args):
         print(json.dumps(line), flush=True)
 
 
+def single_streams(d_flat, sz, dev, peak, reps=10):
+    """Mid-size single streams in the headline line: the first 16 and 64 MiB
+    of the workload's buffer as ONE stream each, sz_compress and sz_decode
+    captured in CUDA graphs and replayed between two events after a 512 MiB
+    write that flushes L2 (median of `reps`), as in the latency sweep; also
+    the frame, the same events around a graph of one tiny kernel."""
+    import torch
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    n_max = (64 << 20) // 2
+    cap, wsb = sz.sz_plan(n_max)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    dec = torch.empty(n_max, dtype=torch.int16, device=dev)
+    cb = torch.empty(16, dtype=torch.uint8, device=dev)
+    size = torch.zeros(1, dtype=torch.int64, device=dev)
+    est = torch.zeros(1, dtype=torch.int32, device=dev)
+    dst = torch.zeros(1, dtype=torch.int32, device=dev)
+    tiny = torch.zeros(4, dtype=torch.int32, device=dev)
+
+    def timed(graphs):
+        t = [[] for _ in graphs]
+        for r in range(3 + reps):
+            for i, g in enumerate(graphs):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                flush.fill_(r & 255)
+                e0.record(stream); g.replay(); e1.record(stream)
+                stream.synchronize()
+                if r >= 3:
+                    t[i].append(e0.elapsed_time(e1) * 1e3)
+        return [float(np.median(v)) for v in t]
+
+    res = {}
+    with torch.cuda.stream(stream):
+        g1 = torch.cuda.CUDAGraph()
+        tiny.add_(1)
+        with torch.cuda.graph(g1, stream=stream):
+            tiny.add_(1)
+        res["frame_one_kernel_us"] = round(timed([g1])[0], 2)
+        del g1
+        for mib in (16, 64):
+            b = mib << 20
+            n = b // 2
+            x = d_flat[:n]
+            c_cap, w_need = sz.sz_plan(n)
+
+            def enc():
+                sz.sz_compress(x, n, out, c_cap, size, cb, est, ws, w_need, stream)
+
+            def dcd():
+                sz.sz_decode(out, c_cap, dec, n, dst, ws, w_need, stream)
+
+            enc(); dcd()
+            ge, gd = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ge, stream=stream):
+                enc()
+            with torch.cuda.graph(gd, stream=stream):
+                dcd()
+            te, td = timed([ge, gd])
+            stream.synchronize()
+            comp = int(size.item())
+            ok = int(est.item()) == 0 and int(dst.item()) == 0 and bool(torch.equal(dec[:n], x))
+            res["%dMiB" % mib] = {"compress_us": round(te, 2), "decode_us": round(td, 2),
+                                  "compress_frac": round((b + comp) / (te * 1e-6) / 1e9 / peak, 4),
+                                  "decode_frac": round((b + comp) / (td * 1e-6) / 1e9 / peak, 4),
+                                  "ratio": round(b / comp, 5), "round_trip": ok}
+            del ge, gd
+    res["timing"] = ("CUDA graph replay between events after a 512 MiB L2 flush, median of %d; fractions of the "
+                     "peak over 2N + container bytes" % reps)
+    return res
+
+
 # ---------------------------------------------------------------- transfer
 def run_transfer(args):
     """The cache handed from one place to another over a link: here PCIe
@@ -949,9 +1021,13 @@ def main():
         cpu = cpu_baseline(inp, args.cpu_seconds)
         cpu.update(host_facts())
 
-    # ---- the other workloads, fewer steps each (rank 0, one GPU)
+    # ---- mid-size single streams and the other workloads, fewer steps
+    # each (rank 0, one GPU)
     workloads = None
+    streams = None
     if rank == 0 and world == 1 and not args.no_workloads and args.tensors <= 0:
+        if inp.contiguous:
+            streams = single_streams(inp.d_in.view(-1), sz, dev, peak)
         del inp, plan, flush
         torch.cuda.empty_cache()
         workloads = {}
@@ -970,7 +1046,7 @@ def main():
             "decode_roofline_frac": roof["decode"]["frac"],
             "encode_roofline_frac_of_spec": round(enc_e2e_bytes / encode_s / 1e9 / SPEC_HBM_GBS, 4),
             "decode_roofline_frac_of_spec": roof["decode"]["frac_of_spec"],
-            "encode_read_once": read_once, "codebook_reuse": reuse,
+            "encode_read_once": read_once, "codebook_reuse": reuse, "single_streams": streams,
             "ratio": round(U / comp, 5), "escape_frac": round(esc / (U // 2), 6),
             "roofline": roofline, "roofline_phases": roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * args.steps,  # hist, encode, esc_index, decode
